@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Routed FP4 MoE layer benchmark on B200.
+
+One step = one pass of the whole layer (route -> sort -> INT8 quant -> W1 ->
+SwiGLU + requant -> W2 -> combine) over one batch of seeded synthetic input,
+through the library's one-call entry point moe_layer_forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moe|reference]
+
+Prints one JSON line on rank 0.  `value` is tokens/s of the whole job with
+inputs resident in HBM; `e2e` is the same through host buffers (pinned H2D of
+x and logits, D2H of y, inside the timed region).  Multi-GPU runs are
+independent replicas (weak scaling), timed as the max over ranks.
+The reference arm (--impl reference) times the CPU oracle on the same
+workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+# Algorithmic HBM bytes of one expert's weights (codes + scales, W1 and W2).
+def expert_bytes(H: int, I: int) -> int:
+    return (2 * I * H + H * I) * 17 // 32
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["moe", "reference"], default="moe")
+    ap.add_argument("--workload", default="decode_T8")
+    ap.add_argument("--prefill-workload", default="prefill_T4604")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing (replicas: barrier + max-over-ranks only, no data-path collective)
+
+class Dist:
+    def __init__(self, n_expected: int):
+        import torch
+        import torch.distributed as dist
+        self.torch, self.dist = torch, dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            import datetime
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        else:
+            torch.cuda.set_device(0)
+        if n_expected != self.world:
+            print(f"warning: --gpus {n_expected} but WORLD_SIZE {self.world}", file=sys.stderr)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def profiled_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch of the streaming GEMM from a committed ncu summary,
+    valid only while the kernel source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", f"gemv_{workload}_traffic.json")
+    src = os.path.join(ROOT, "fp4_routed_mixture_b200", "csrc", kernel_file)
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    if d.get("kernel_sha256") != h:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------
+
+def run_gpu_workload(name: str, steps: int, warmup: int, dist: Dist, want_e2e: bool,
+                     want_clocks: bool):
+    import torch
+
+    import fp4_routed_mixture_b200 as moe
+
+    w = synth.WORKLOADS[name]
+    T, H, I, E, k = w.T, w.H, w.I, w.E, w.k
+    d = synth.make(w)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    canon = [cu(d[n]) for n in ("w1_codes", "w1_scales", "w2_codes", "w2_scales")]
+    packed = moe.moe_pack_weights(*canon)
+    del canon
+    logits = cu(d["logits"])
+    x = cu(d["x"]).view(torch.bfloat16)
+    ws = torch.empty(moe.moe_layer_workspace_bytes(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    # touched experts of this batch (outside the timed region)
+    idx, _ = moe.moe_route(logits, k)
+    touched = int(torch.unique(idx).numel())
+    alg_bytes_step = touched * expert_bytes(H, I)
+    alg_flop_step = 6.0 * T * k * I * H
+
+    def step(dbg=None):
+        moe.moe_layer_forward(logits, x, packed, H, I, E, k, ws=ws, y=y, dbg=dbg, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # per-step GEMM events (W1 start/end, W2 start/end) for the live kernel roofline
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    dbgs = [moe.make_debug(None, e) for e in ev]
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(torch.cuda.current_device()) if want_clocks else None
+    launches0 = moe.moe_launch_count()
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s in range(steps):
+        step(dbgs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    launches = moe.moe_launch_count() - launches0
+    clk = clocks.stop() if clocks else None
+    ms = dist.max(t0.elapsed_time(t1))
+    gemm_ms = sum(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev)
+    w1_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    w2_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
+    flag = moe.moe_check_device_flag(ws)
+    assert flag == 0, f"device error word {flag:#x}"
+
+    res = dict(workload=w, T=T, ms=ms, steps=steps, launches=launches, clocks=clk, touched=touched,
+               alg_bytes_step=alg_bytes_step, alg_flop_step=alg_flop_step, gemm_ms=gemm_ms,
+               w1_ms=w1_ms, w2_ms=w2_ms)
+
+    if want_e2e:
+        xh = torch.from_numpy(d["x"]).view(torch.bfloat16).pin_memory()
+        lh = torch.from_numpy(d["logits"]).pin_memory()
+        yh = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(x)
+        ld = torch.empty_like(logits)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            ld.copy_(lh, non_blocking=True)
+            moe.moe_layer_forward(ld, xd, packed, H, I, E, k, ws=ws, y=y, stream=stream)
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(max(3, warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        res["e2e_ms"] = dist.max(e0.elapsed_time(e1))
+        res["h2d"] = xh.numel() * 2 + lh.numel() * 4
+        res["d2h"] = yh.numel() * 2
+    del packed, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(name: str, seconds: float) -> dict:
+    import oracle
+    w = synth.WORKLOADS[name]
+    d = synth.make(w)
+    t0 = time.time()
+    reps = 0
+    if w.T <= 64:
+        # the whole step (all T tokens) per repetition
+        while True:
+            oracle.forward(d["x"], d["logits"], d["w1_codes"], d["w1_scales"], d["w2_codes"],
+                           d["w2_scales"], w.k)
+            reps += 1
+            if time.time() - t0 >= seconds:
+                break
+        toks = reps * w.T
+        sample = f"{reps} full steps of {name} ({w.T} tokens each)"
+    else:
+        tok = 0
+        while time.time() - t0 < seconds:
+            oracle.forward_tokens(d["x"], d["logits"], d["w1_codes"], d["w1_scales"],
+                                  d["w2_codes"], d["w2_scales"], w.k, [tok % w.T])
+            tok += 1
+        toks = tok
+        sample = f"{tok} single-token layer evaluations of {name}"
+    dt = time.time() - t0
+    return {"value": toks / dt, "unit": "tokens/s", "cores": oracle.nthreads(), "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 2)}
+
+
+def roofline_hbm(r: dict, peaks: dict, traffic):
+    n_launch = 2 * r["steps"]
+    bytes_per_launch = r["alg_bytes_step"] / 2.0
+    achieved = (r["alg_bytes_step"] * r["steps"]) / (r["gemm_ms"] * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "k_gemv (W1 and W2 launches)", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic, "launches": n_launch, "alg_bytes_per_launch": bytes_per_launch,
+            "peak_source": peaks["source"] + " (hbm_gbs: stream copy)"}
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        return main_reference(a)
+    steps = a.steps if a.steps is not None else 2000
+    warmup = a.warmup if a.warmup is not None else 20
+    assert warmup >= 3 or a.warmup is not None
+    dist = Dist(a.gpus)
+    import torch
+    rank0 = dist.rank == 0
+    peaks = measured_peaks()
+    r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
+    w = r["workload"]
+    N = dist.world
+    value = N * w.T * steps / (r["ms"] * 1e-3)
+    out = {
+        "metric": "routed-MoE layer tokens/s (T=8 decode, T=4604 prefill); % HBM / TC roofline",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": N, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(r["ms"] / steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8 x e2m1 -> int32 block sums, fp64 acc",
+        "data": "synthetic (seeded SplitMix64; random MXFP4 weights, N(0,1) activations)",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k,
+                   "seed": w.seed, "parallelism": f"replicas x{N}",
+                   "touched_experts": r["touched"],
+                   "l2": "inputs larger than L2: %.2f GB of expert weights streamed per step "
+                         "vs 126 MB L2" % (r["alg_bytes_step"] / 1e9)},
+        "roofline": roofline_hbm(r, peaks, profiled_traffic("gemv.cu", w.name)),
+        "e2e": {"value": round(N * w.T * steps / (r["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+        "kernel_ms_per_step": {"w1": round(r["w1_ms"] / steps, 5), "w2": round(r["w2_ms"] / steps, 5)},
+    }
+    if not a.no_prefill:
+        pw = synth.WORKLOADS[a.prefill_workload]
+        psteps = max(3, min(20, steps // 100))
+        rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=False)
+        ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        out["prefill"] = {
+            "workload": pw.name, "T": pw.T, "steps": psteps,
+            "value": round(N * pw.T * psteps / (rp["ms"] * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(rp["ms"] / psteps, 4),
+            "roofline": {"bound": "tensor", "kernel": "k_gemv (CUDA-core fallback)",
+                         "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
+                         "frac": round(ptf / fp8_peak, 5),
+                         "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
+                         "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1)},
+        }
+    if rank0 and N == 1 and not a.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)
+    if rank0:
+        print(json.dumps(out), flush=True)
+    dist.close()
+
+
+def main_reference(a):
+    """The oracle, timed on this host's cores, on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    steps = a.steps if a.steps is not None else 5
+    warmup = a.warmup if a.warmup is not None else 1
+    w = synth.WORKLOADS[a.workload]
+    d = synth.make(w)
+    # each step is a bounded sample: the layer for one token of the batch
+    def step(i):
+        oracle.forward_tokens(d["x"], d["logits"], d["w1_codes"], d["w1_scales"], d["w2_codes"],
+                              d["w2_scales"], w.k, [i % w.T])
+    for i in range(warmup):
+        step(i)
+    t0 = time.time()
+    for i in range(steps):
+        step(i)
+    dt = time.time() - t0
+    value = steps / dt
+    out = {"metric": "routed-MoE layer tokens/s (T=8 decode, T=4604 prefill); % HBM / TC roofline",
+           "value": round(value, 4), "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+           "steps": steps, "warmup": warmup, "ms_per_step": round(dt * 1e3 / steps, 2),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded SplitMix64)", "impl": "reference",
+           "config": {"workload": w.name, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "k": w.k},
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": oracle.nthreads(),
+                            "kind": "oracle",
+                            "sample": f"each step: the whole layer for one token of {w.name}"},
+           "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,319 @@
+// C-ABI layer: argument checks, workspace layout, launch sequence.
+// Declarations and the meaning of every argument are in include/moe.h.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/moe.h"
+#include "kernels.cuh"
+#include "moe_common.cuh"
+
+#include <atomic>
+
+namespace moe {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+}  // namespace moe
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int check_dims(const moe_dims* d, bool need_T) {
+    if (!d) return fail(MOE_ERR_INVALID_ARG, "dims is NULL");
+    if (need_T && d->T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0 (got %d)", d->T);
+    if (d->H <= 0 || d->I <= 0 || d->H % 128 || d->I % 128)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "H and I must be positive multiples of 128 (H=%d I=%d)",
+                    d->H, d->I);
+    if (d->E < 1 || d->E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 1024] (got %d)", d->E);
+    if (d->k < 1 || d->k > 16 || d->k > d->E)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "k must be in [1, min(E, 16)] (got %d)", d->k);
+    if (need_T && (long long)d->T * d->k >= (1LL << 31))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T*k must be < 2^31");
+    return MOE_OK;
+}
+
+struct WsLayout {
+    size_t flag, uoff1, uoff2, sx, xq, xinit, hq, sh, hinit, gacc, yacc, total;
+};
+
+WsLayout ws_layout(const moe_dims& d, long long T) {
+    using moe::align_up;
+    const size_t P = (size_t)T * d.k;
+    WsLayout L;
+    size_t o = 0;
+    L.flag = o; o += 256;
+    L.uoff1 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.uoff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.sx = o; o += align_up(4 * (size_t)T, 256);
+    L.xq = o; o += align_up((size_t)T * d.H, 256);
+    L.xinit = o; o += align_up(4 * (size_t)T * (d.H / 32), 256);
+    L.hq = o; o += align_up(P * d.I, 256);
+    L.sh = o; o += align_up(4 * P, 256);
+    L.hinit = o; o += align_up(4 * P * (d.I / 32), 256);
+    L.gacc = o; o += align_up(8 * P * 2 * d.I, 256);   // gacc and yacc are adjacent:
+    L.yacc = o; o += align_up(8 * P * d.H, 256);        // one memset clears both
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_last_error(char* buf, size_t n) {
+    if (buf && n) {
+        const size_t c = std::min(n - 1, g_last_error.size());
+        std::memcpy(buf, g_last_error.data(), c);
+        buf[c] = 0;
+    }
+    return g_last_error.size();
+}
+
+size_t moe_packed_bytes(const moe_dims* d) {
+    if (check_dims(d, false) != MOE_OK) return 0;
+    return moe::packed_layout(d->H, d->I, d->E).total;
+}
+
+int moe_pack_weights(const moe_dims* d, const uint8_t* w1_codes, const uint8_t* w1_scales,
+                     const uint8_t* w2_codes, const uint8_t* w2_scales, void* packed,
+                     cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, false)) return rc;
+    if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !packed)
+        return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: NULL pointer");
+    if (!aligned(w1_codes, 16) || !aligned(w2_codes, 16) || !aligned(packed, 256))
+        return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: codes need 16-byte, packed 256-byte alignment");
+    cudaError_t e = moe::launch_pack(d->H, d->I, d->E, w1_codes, w1_scales, w2_codes, w2_scales,
+                                     packed, true, nullptr, nullptr, nullptr, nullptr, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_pack_weights launch");
+    int32_t flag = 0;
+    e = cudaMemcpyAsync(&flag, moe::packed_flag_ptr(packed), sizeof(flag), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_pack_weights");
+    if (flag & MOE_FLAG_BAD_SCALE)
+        return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: scale byte 0xFF (E8M0 NaN) in the input");
+    return MOE_OK;
+}
+
+int moe_unpack_weights(const moe_dims* d, const void* packed, uint8_t* w1_codes, uint8_t* w1_scales,
+                       uint8_t* w2_codes, uint8_t* w2_scales, cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, false)) return rc;
+    if (!w1_codes || !w1_scales || !w2_codes || !w2_scales || !packed)
+        return fail(MOE_ERR_INVALID_ARG, "moe_unpack_weights: NULL pointer");
+    if (!aligned(w1_codes, 16) || !aligned(w2_codes, 16) || !aligned(packed, 256))
+        return fail(MOE_ERR_INVALID_ARG, "moe_unpack_weights: codes need 16-byte, packed 256-byte alignment");
+    cudaError_t e = moe::launch_pack(d->H, d->I, d->E, nullptr, nullptr, nullptr, nullptr,
+                                     const_cast<void*>(packed), false, w1_codes, w1_scales, w2_codes,
+                                     w2_scales, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_unpack_weights launch");
+}
+
+int moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
+              cudaStream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_route: T < 0");
+    if (E < 1 || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_route: E must be in [1, 1024]");
+    if (k < 1 || k > 16 || k > E) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_route: k must be in [1, min(E,16)]");
+    if (T > 0 && (!logits || !topk_idx || !gates)) return fail(MOE_ERR_INVALID_ARG, "moe_route: NULL pointer");
+    cudaError_t e = moe::launch_route(logits, T, E, k, topk_idx, gates, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+}
+
+size_t moe_sort_workspace_bytes(int T_max, int k, int E) {
+    if (T_max < 0 || k < 1 || E < 1) return 0;
+    return moe::sort_workspace_bytes(T_max, k, E);
+}
+
+int moe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
+             int32_t* offsets, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_sort: T < 0");
+    if (E < 1 || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_sort: E must be in [1, 1024]");
+    if (k < 1 || k > 16 || k > E) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_sort: k must be in [1, min(E,16)]");
+    if ((long long)T * k >= (1LL << 31)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_sort: T*k too large");
+    if (!offsets || !ws || (T > 0 && (!topk_idx || !perm || !pos)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_sort: NULL pointer");
+    if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "moe_sort: ws must be 256-byte aligned");
+    if (ws_bytes < moe::sort_workspace_bytes(T, k, E))
+        return fail(MOE_ERR_INVALID_ARG, "moe_sort: ws_bytes %zu < %zu", ws_bytes,
+                    moe::sort_workspace_bytes(T, k, E));
+    cudaError_t e = moe::launch_sort(topk_idx, T, k, E, perm, pos, offsets, ws, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort launch");
+}
+
+size_t moe_workspace_bytes(const moe_dims* d, int T_max) {
+    if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
+    return ws_layout(*d, T_max).total;
+}
+
+int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, const float* gates,
+                const int32_t* perm, const int32_t* pos, const int32_t* offsets, const void* packed,
+                void* y_bf16, void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, true)) return rc;
+    if (!ws || !packed || !offsets) return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
+    if (d->T > 0 && (!x_bf16 || !topk_idx || !gates || !perm || !pos || !y_bf16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
+    if (!aligned(ws, 256) || !aligned(packed, 256) || !aligned(x_bf16, 16) || !aligned(y_bf16, 16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws/packed need 256-byte, x/y 16-byte alignment");
+    const WsLayout L = ws_layout(*d, d->T);
+    if (ws_bytes < L.total)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws_bytes %zu < %zu", ws_bytes, L.total);
+    char* w = (char*)ws;
+    int32_t* flag = (int32_t*)(w + L.flag);
+    cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int32_t), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_forward memset");
+    if (d->T == 0) return MOE_OK;
+
+    const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k, P = T * k;
+    const moe::PackedLayout PL = moe::packed_layout(H, I, E);
+    const uint8_t* pk = (const uint8_t*)packed;
+    int32_t* uoff1 = (int32_t*)(w + L.uoff1);
+    int32_t* uoff2 = (int32_t*)(w + L.uoff2);
+    float* sx = (float*)(w + L.sx);
+    int8_t* xq = (int8_t*)(w + L.xq);
+    int32_t* xinit = (int32_t*)(w + L.xinit);
+    int8_t* hq = (int8_t*)(w + L.hq);
+    float* sh = (float*)(w + L.sh);
+    int32_t* hinit = (int32_t*)(w + L.hinit);
+    double* gacc = (double*)(w + L.gacc);
+    double* yacc = (double*)(w + L.yacc);
+
+#define MOE_TRY(call, what)                          \
+    do {                                             \
+        cudaError_t _e = (call);                     \
+        if (_e != cudaSuccess) return cuda_fail(_e, what); \
+    } while (0)
+    MOE_TRY(moe::launch_check_header(packed, H, I, E, flag, stream), "header check");
+    MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, dbg ? dbg->xq : nullptr,
+                               dbg ? dbg->sx : nullptr, stream), "x quant");
+    MOE_TRY(moe::launch_plan(offsets, E, 2 * I / 32, H / 32, uoff1, uoff2, stream), "plan");
+    MOE_TRY(cudaMemsetAsync(gacc, 0, L.total - L.gacc, stream), "accumulator clear");
+    cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
+    if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
+    MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
+                             uoff1, E, gacc, flag, stream), "W1");
+    if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
+    MOE_TRY(moe::launch_swiglu_hquant(gacc, sx, perm, P, k, I, hq, sh, hinit,
+                                      dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, stream),
+            "SwiGLU + h quant");
+    if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
+    MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
+                             uoff2, E, yacc, flag, stream), "W2");
+    if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
+    MOE_TRY(moe::launch_combine(yacc, sh, gates, pos, T, k, H, y_bf16, stream), "combine");
+#undef MOE_TRY
+    return MOE_OK;
+}
+
+// Whole-layer workspace: forward workspace, then idx/gates/perm/pos/offsets,
+// then the sort scratch.
+struct LayerWs {
+    size_t fwd, idx, gates, perm, pos, offsets, sortws, sort_bytes, total;
+};
+
+static LayerWs layer_ws(const moe_dims& d, long long T) {
+    using moe::align_up;
+    LayerWs L;
+    const size_t P = (size_t)T * d.k;
+    size_t o = 0;
+    L.fwd = o; o += ws_layout(d, T).total;
+    L.idx = o; o += align_up(4 * P, 256);
+    L.gates = o; o += align_up(4 * P, 256);
+    L.perm = o; o += align_up(4 * P, 256);
+    L.pos = o; o += align_up(4 * P, 256);
+    L.offsets = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.sortws = o;
+    L.sort_bytes = moe::sort_workspace_bytes((int)T, d.k, d.E);
+    o += L.sort_bytes;
+    L.total = o;
+    return L;
+}
+
+size_t moe_layer_workspace_bytes(const moe_dims* d, int T_max) {
+    if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
+    return layer_ws(*d, T_max).total;
+}
+
+int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16, const void* packed,
+                      void* y_bf16, void* ws, size_t ws_bytes, const moe_debug* dbg,
+                      cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, true)) return rc;
+    if (!ws || !packed || (d->T > 0 && (!logits || !x_bf16 || !y_bf16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: NULL pointer");
+    if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: ws must be 256-byte aligned");
+    const LayerWs L = layer_ws(*d, d->T);
+    if (ws_bytes < L.total)
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: ws_bytes %zu < %zu", ws_bytes, L.total);
+    char* w = (char*)ws;
+    int32_t* idx = (int32_t*)(w + L.idx);
+    float* gates = (float*)(w + L.gates);
+    int32_t* perm = (int32_t*)(w + L.perm);
+    int32_t* pos = (int32_t*)(w + L.pos);
+    int32_t* offsets = (int32_t*)(w + L.offsets);
+    if (int rc = moe_route(logits, d->T, d->E, d->k, idx, gates, stream)) return rc;
+    if (int rc = moe_sort(idx, d->T, d->k, d->E, perm, pos, offsets, w + L.sortws, L.sort_bytes, stream))
+        return rc;
+    return moe_forward(d, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
+                       L.idx - L.fwd, dbg, stream);
+}
+
+int moe_quant_rows_f32(const float* v, int rows, int cols, int8_t* q, float* s, cudaStream_t stream) {
+    g_last_error.clear();
+    if (rows < 0 || cols <= 0) return fail(MOE_ERR_INVALID_ARG, "moe_quant_rows_f32: bad shape");
+    if (rows > 0 && (!v || !q || !s)) return fail(MOE_ERR_INVALID_ARG, "moe_quant_rows_f32: NULL pointer");
+    cudaError_t e = moe::launch_quant_rows(v, rows, cols, q, s, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_quant_rows_f32 launch");
+}
+
+int moe_exp_f32(const float* x, float* y, int64_t n, cudaStream_t stream) {
+    g_last_error.clear();
+    if (n < 0 || (n > 0 && (!x || !y))) return fail(MOE_ERR_INVALID_ARG, "moe_exp_f32: bad arguments");
+    cudaError_t e = moe::launch_exp(x, y, n, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_exp_f32 launch");
+}
+
+int moe_swiglu_f32(const float* g, const float* u, float* h, int64_t n, cudaStream_t stream) {
+    g_last_error.clear();
+    if (n < 0 || (n > 0 && (!g || !u || !h))) return fail(MOE_ERR_INVALID_ARG, "moe_swiglu_f32: bad arguments");
+    cudaError_t e = moe::launch_swiglu(g, u, h, n, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_swiglu_f32 launch");
+}
+
+unsigned long long moe_launch_count(void) { return moe::g_launches.load(); }
+
+int moe_check_device_flag(const void* ws, int32_t* out_flag, cudaStream_t stream) {
+    g_last_error.clear();
+    if (!ws || !out_flag) return fail(MOE_ERR_INVALID_ARG, "moe_check_device_flag: NULL pointer");
+    int32_t f = 0;
+    cudaError_t e = cudaMemcpyAsync(&f, ws, sizeof(f), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_check_device_flag");
+    *out_flag = f;
+    if (f) return fail(MOE_ERR_DEVICE_FLAG, "device error word 0x%x", f);
+    return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Launch wrappers shared between the kernel files and the C-ABI layer.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cstddef>
+
+namespace moe {
+
+// Number of kernels this library has launched in the process (diagnostics).
+void count_launches(int n);
+
+struct PackedLayout {
+    size_t header, w1, w1_expert_bytes, w2, w2_expert_bytes, total;
+};
+PackedLayout packed_layout(int H, int I, int E);
+
+cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
+                         cudaStream_t st);
+
+size_t sort_workspace_bytes(int T_max, int k, int E);
+cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
+                        int32_t* offsets, void* ws, cudaStream_t st);
+
+cudaError_t launch_pack(int H, int I, int E, const uint8_t* w1c, const uint8_t* w1s,
+                        const uint8_t* w2c, const uint8_t* w2s, void* packed, bool forward,
+                        uint8_t* out_w1c, uint8_t* out_w1s, uint8_t* out_w2c, uint8_t* out_w2s,
+                        cudaStream_t st);
+const int32_t* packed_flag_ptr(const void* packed);
+cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t* flag,
+                                cudaStream_t st);
+
+cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
+                          int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
+cudaError_t launch_swiglu_hquant(const double* gacc, const float* sx, const int32_t* perm, int P,
+                                 int k, int I, int8_t* hq, float* sh, int32_t* hinit,
+                                 int8_t* dbg_hq, float* dbg_sh, cudaStream_t st);
+cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
+cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
+cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
+                              cudaStream_t st);
+
+cudaError_t launch_plan(const int32_t* offsets, int E, int tiles1, int tiles2, int32_t* unit_off1,
+                        int32_t* unit_off2, cudaStream_t st);
+cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
+                        const int32_t* act_init, const int32_t* perm, int k_div,
+                        const int32_t* offsets, const int32_t* unit_off, int E, double* out,
+                        const int32_t* flag, cudaStream_t st);
+
+cudaError_t launch_combine(const double* yacc, const float* sh, const float* gates,
+                           const int32_t* pos, int T, int k, int H, void* y, cudaStream_t st);
+
+}  // namespace moe

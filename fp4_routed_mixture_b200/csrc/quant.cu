@@ -1,0 +1,206 @@
+// INT8 activation quantisation ("DeepSeek-V4-Flash on AMD gfx90a", abstract:
+// INT8 activations feeding the packed-FP4 expert GEMMs).
+//
+//   k_xquant        x [T,H] bf16 -> xq [T,H] int8, sx [T], xinit [T,H/32]
+//   k_swiglu_hquant G accumulators (fp64, sorted rows) -> SwiGLU -> hq, sh, hinit
+//   k_quant_rows    fp32 rows -> int8 + scale (stage entry point)
+//
+// Rule for every row: a = max|v| (exact), s = fp32(a/127) by IEEE division,
+// q = clamp(rne(fp32(v/s)), -127, 127), and q = 0, s = 0 for an all-zero row.
+// xinit/hinit hold -12 * (sum of the 32 codes of each K block): the streaming
+// GEMM decodes weight nibbles to 2*e2m1 + 12 (an unsigned byte), so this term
+// cancels the +12 bias of every block's integer dot product.
+#include "kernels.cuh"
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kQThreads = 256;
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+    v = warp_max(v);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    if (w == 0) {
+        v = (lane < (int)(blockDim.x >> 5)) ? red[lane] : 0.0f;
+        v = warp_max(v);
+        if (lane == 0) red[32] = v;
+    }
+    __syncthreads();
+    const float r = red[32];
+    __syncthreads();
+    return r;
+}
+
+// One CTA per token; each thread handles chunks of 8 consecutive elements.
+__global__ void __launch_bounds__(kQThreads)
+    k_xquant(const __nv_bfloat16* __restrict__ x, int T, int H, int8_t* __restrict__ xq,
+             float* __restrict__ sx, int32_t* __restrict__ xinit, int8_t* __restrict__ dbg_xq,
+             float* __restrict__ dbg_sx) {
+    __shared__ float red[33];
+    const int t = blockIdx.x;
+    const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    const int nchunk = H / 8;
+    float a = 0.0f;
+    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+        const uint4 v = __ldg(row + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            a = fmaxf(a, fabsf(__uint_as_float(w[j] << 16)));
+            a = fmaxf(a, fabsf(__uint_as_float(w[j] & 0xffff0000u)));
+        }
+    }
+    a = block_max(a, red);
+    const float s = quant_scale(a);
+    if (threadIdx.x == 0) {
+        sx[t] = s;
+        if (dbg_sx) dbg_sx[t] = s;
+    }
+    // chunks are handed out round-robin, so the 4 chunks of one 32-element
+    // block sit in 4 consecutive lanes of one warp (nchunk % 4 == 0)
+    for (int c0 = 0; c0 < nchunk; c0 += blockDim.x) {
+        const int c = c0 + threadIdx.x;
+        int bsum = 0;
+        if (c < nchunk) {
+            const uint4 v = __ldg(row + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int q0 = quant_code(__uint_as_float(w[j] << 16), a, s);
+                const int q1 = quant_code(__uint_as_float(w[j] & 0xffff0000u), a, s);
+                bsum += q0 + q1;
+                packed[j >> 1] |= ((uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8))
+                                  << (16 * (j & 1));
+            }
+            const uint2 pv = make_uint2(packed[0], packed[1]);
+            reinterpret_cast<uint2*>(xq + (size_t)t * H)[c] = pv;
+            if (dbg_xq) reinterpret_cast<uint2*>(dbg_xq + (size_t)t * H)[c] = pv;
+        }
+        bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
+        bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
+        if (c < nchunk && (c & 3) == 0) xinit[(size_t)t * (H / 32) + (c >> 2)] = -12 * bsum;
+    }
+}
+
+// One CTA per sorted row i.  G values are the exact fp64 sums of the W1
+// product; the fp32 G of the definition is fp32(fp64(sx[t]) * sum).
+__global__ void __launch_bounds__(kQThreads)
+    k_swiglu_hquant(const double* __restrict__ gacc, const float* __restrict__ sx,
+                    const int32_t* __restrict__ perm, int k, int I, int8_t* __restrict__ hq,
+                    float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
+                    float* __restrict__ dbg_sh) {
+    extern __shared__ float h[];  // [I]
+    __shared__ float red[33];
+    const int i = blockIdx.x;
+    const int t = perm[i] / k;
+    const double s = (double)sx[t];
+    const double* g = gacc + (size_t)i * 2 * I;
+    float a = 0.0f;
+    for (int j = threadIdx.x; j < I; j += blockDim.x) {
+        const float gv = (float)__dmul_rn(s, g[j]);
+        const float uv = (float)__dmul_rn(s, g[I + j]);
+        const float hv = swiglu(gv, uv);
+        h[j] = hv;
+        a = fmaxf(a, fabsf(hv));
+    }
+    a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
+    const float sc = quant_scale(a);
+    if (threadIdx.x == 0) {
+        sh[i] = sc;
+        if (dbg_sh) dbg_sh[i] = sc;
+    }
+    // 4 codes per thread-step; 8 consecutive lanes cover one 32-element block
+    for (int j0 = 0; j0 < I; j0 += 4 * blockDim.x) {
+        const int j = j0 + 4 * threadIdx.x;
+        int bsum = 0;
+        if (j < I) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int q = quant_code(h[j + u], a, sc);
+                bsum += q;
+                packed |= (uint32_t)(q & 0xff) << (8 * u);
+            }
+            *reinterpret_cast<uint32_t*>(hq + (size_t)i * I + j) = packed;
+            if (dbg_hq) *reinterpret_cast<uint32_t*>(dbg_hq + (size_t)i * I + j) = packed;
+        }
+        bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
+        bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
+        bsum += __shfl_xor_sync(0xffffffffu, bsum, 4);
+        if (j < I && (j & 31) == 0) hinit[(size_t)i * (I / 32) + (j >> 5)] = -12 * bsum;
+    }
+}
+
+__global__ void __launch_bounds__(kQThreads)
+    k_quant_rows(const float* __restrict__ v, int cols, int8_t* __restrict__ q, float* __restrict__ s) {
+    __shared__ float red[33];
+    const int r = blockIdx.x;
+    const float* row = v + (size_t)r * cols;
+    float a = 0.0f;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x) a = fmaxf(a, fabsf(row[c]));
+    a = block_max(a, red);
+    const float sc = quant_scale(a);
+    if (threadIdx.x == 0) s[r] = sc;
+    for (int c = threadIdx.x; c < cols; c += blockDim.x)
+        q[(size_t)r * cols + c] = (int8_t)quant_code(row[c], a, sc);
+}
+
+__global__ void k_exp(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        y[i] = layer_exp(x[i]);
+}
+
+__global__ void k_swiglu(const float* __restrict__ g, const float* __restrict__ u,
+                         float* __restrict__ h, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        h[i] = swiglu(g[i], u[i]);
+}
+
+cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+    k_exp<<<grid, 256, 0, st>>>(x, y, n);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, 148 * 16);
+    k_swiglu<<<grid, 256, 0, st>>>(g, u, h, n);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
+                          int8_t* dbg_xq, float* dbg_sx, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    k_xquant<<<T, kQThreads, 0, st>>>((const __nv_bfloat16*)x, T, H, xq, sx, xinit, dbg_xq, dbg_sx);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_hquant(const double* gacc, const float* sx, const int32_t* perm, int P,
+                                 int k, int I, int8_t* hq, float* sh, int32_t* hinit,
+                                 int8_t* dbg_hq, float* dbg_sh, cudaStream_t st) {
+    if (P == 0) return cudaSuccess;
+    k_swiglu_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, sx, perm, k, I, hq, sh,
+                                                                      hinit, dbg_hq, dbg_sh);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
+                              cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    k_quant_rows<<<rows, kQThreads, 0, st>>>(v, cols, q, s);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,198 @@
+// Expert sorting: stable counting sort of token-expert pairs by expert.
+//
+// "DeepSeek-V4-Flash on AMD gfx90a" (abstract) groups the routed pairs by
+// expert before the expert GEMMs and retunes that sort for prefill.  Here the
+// sort is an atomic histogram in shared memory, a prefix scan, and a stable
+// scatter:
+//   k_sort_count   (one CTA per chunk of 1024 pairs): per-chunk histogram
+//   k_sort_scatter (one CTA per chunk): every CTA rebuilds the global offsets
+//                  and its chunk's starting cursor per expert from the chunk
+//                  histograms, then one warp walks the chunk in pair order;
+//                  __match_any_sync ranks equal experts inside each 32-pair
+//                  step, which keeps the sort stable.
+// A single chunk (P <= 1024, the decode case) runs both phases in one launch.
+// Expert ids outside [0, E) raise FLAG_BAD_EXPERT and are skipped.
+#include "kernels.cuh"
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int kSortChunk = 1024;
+constexpr int kSortThreads = 256;
+
+__device__ __forceinline__ bool valid_expert(int e, int E) { return (unsigned)e < (unsigned)E; }
+
+// Exclusive scan of smem[0..E) in place (blockDim == kSortThreads, E <= 1024);
+// returns the total.  Uses `tmp` [kSortThreads + 1] of shared scratch.
+__device__ int block_exclusive_scan(int* vals, int E, int* tmp) {
+    const int tid = threadIdx.x;
+    const int per = (E + kSortThreads - 1) / kSortThreads;  // <= 4
+    int local[4];
+    int s = 0;
+    for (int j = 0; j < per; ++j) {
+        const int e = tid * per + j;
+        local[j] = (e < E) ? vals[e] : 0;
+        s += local[j];
+    }
+    tmp[tid] = s;
+    __syncthreads();
+    // Hillis-Steele over kSortThreads partial sums
+    for (int o = 1; o < kSortThreads; o <<= 1) {
+        const int v = (tid >= o) ? tmp[tid - o] : 0;
+        __syncthreads();
+        tmp[tid] += v;
+        __syncthreads();
+    }
+    int run = (tid == 0) ? 0 : tmp[tid - 1];
+    const int total = tmp[kSortThreads - 1];
+    __syncthreads();
+    for (int j = 0; j < per; ++j) {
+        const int e = tid * per + j;
+        if (e < E) {
+            vals[e] = run;
+            run += local[j];
+        }
+    }
+    __syncthreads();
+    return total;
+}
+
+// Stable scatter of pairs [p0, p1) by one warp; cursor[e] is the next free
+// sorted slot of expert e and is advanced in place.
+__device__ void warp_stable_scatter(const int32_t* __restrict__ topk_idx, int p0, int p1, int E,
+                                    int* cursor, int32_t* __restrict__ perm,
+                                    int32_t* __restrict__ pos) {
+    const int lane = threadIdx.x & 31;
+    for (int base = p0; base < p1; base += 32) {
+        const int p = base + lane;
+        const bool in = p < p1;
+        int e = in ? __ldg(topk_idx + p) : -1;
+        if (!valid_expert(e, E)) e = -1 - lane;  // unique key: never grouped, never written
+        const uint32_t same = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        const int leader = __ffs(same) - 1;
+        int slot = 0;
+        if (e >= 0) slot = cursor[e];  // all lanes of a group read the same value
+        __syncwarp();
+        if (e >= 0) {
+            const int dst = slot + rank;
+            perm[dst] = p;
+            pos[p] = dst;
+            if (lane == leader) cursor[e] = slot + __popc(same);
+        }
+        __syncwarp();
+    }
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+    k_sort_count(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ chunk_hist,
+                 int32_t* flag) {
+    extern __shared__ int hist[];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    const int p0 = blockIdx.x * kSortChunk, p1 = min(P, p0 + kSortChunk);
+    bool bad = false;
+    for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+        const int e = __ldg(topk_idx + p);
+        if (valid_expert(e, E))
+            atomicAdd(&hist[e], 1);
+        else
+            bad = true;
+    }
+    if (bad) raise_flag(flag, FLAG_BAD_EXPERT);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+__global__ void __launch_bounds__(kSortThreads)
+    k_sort_scatter(const int32_t* __restrict__ topk_idx, int P, int E,
+                   const int32_t* __restrict__ chunk_hist, int32_t* __restrict__ perm,
+                   int32_t* __restrict__ pos, int32_t* __restrict__ offsets) {
+    extern __shared__ int sm[];
+    int* total = sm;           // [E] -> exclusive offsets
+    int* cursor = sm + E;      // [E]
+    int* tmp = sm + 2 * E;     // [kSortThreads + 1]
+    const int nchunks = gridDim.x, c = blockIdx.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int tot = 0, before = 0;
+        for (int j = 0; j < nchunks; ++j) {
+            const int v = chunk_hist[(size_t)j * E + e];
+            tot += v;
+            if (j < c) before += v;
+        }
+        total[e] = tot;
+        cursor[e] = before;
+    }
+    __syncthreads();
+    const int all = block_exclusive_scan(total, E, tmp);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cursor[e] += total[e];
+    if (c == 0) {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = total[e];
+        if (threadIdx.x == 0) offsets[E] = all;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int p0 = c * kSortChunk, p1 = min(P, p0 + kSortChunk);
+        warp_stable_scatter(topk_idx, p0, p1, E, cursor, perm, pos);
+    }
+}
+
+// P <= kSortChunk: histogram, scan and scatter in one CTA.
+__global__ void __launch_bounds__(kSortThreads)
+    k_sort_single(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ perm,
+                  int32_t* __restrict__ pos, int32_t* __restrict__ offsets, int32_t* flag) {
+    extern __shared__ int sm[];
+    int* hist = sm;
+    int* tmp = sm + E;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int p = threadIdx.x; p < P; p += blockDim.x) {
+        const int e = __ldg(topk_idx + p);
+        if (valid_expert(e, E))
+            atomicAdd(&hist[e], 1);
+        else
+            bad = true;
+    }
+    if (bad) raise_flag(flag, FLAG_BAD_EXPERT);
+    __syncthreads();
+    const int all = block_exclusive_scan(hist, E, tmp);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = hist[e];
+    if (threadIdx.x == 0) offsets[E] = all;
+    __syncthreads();
+    if (threadIdx.x < 32) warp_stable_scatter(topk_idx, 0, P, E, hist, perm, pos);
+}
+
+size_t sort_workspace_bytes(int T_max, int k, int E) {
+    const size_t P = (size_t)T_max * k;
+    const size_t chunks = (P + kSortChunk - 1) / kSortChunk;
+    return 256 + align_up(std::max<size_t>(chunks, 1) * E * sizeof(int32_t), 256);
+}
+
+cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
+                        int32_t* offsets, void* ws, cudaStream_t st) {
+    int32_t* flag = (int32_t*)ws;
+    int32_t* chunk_hist = (int32_t*)((char*)ws + 256);
+    const int P = T * k;
+    cudaError_t err = cudaMemsetAsync(flag, 0, sizeof(int32_t), st);
+    if (err != cudaSuccess) return err;
+    if (P <= kSortChunk) {
+        const size_t smem = (size_t)(E + kSortThreads + 1) * sizeof(int);
+        k_sort_single<<<1, kSortThreads, smem, st>>>(topk_idx, P, E, perm, pos, offsets, flag);
+        count_launches(1);
+        return cudaGetLastError();
+    }
+    const int chunks = (P + kSortChunk - 1) / kSortChunk;
+    k_sort_count<<<chunks, kSortThreads, (size_t)E * sizeof(int), st>>>(topk_idx, P, E, chunk_hist,
+                                                                        flag);
+    count_launches(1);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const size_t smem = (size_t)(2 * E + kSortThreads + 1) * sizeof(int);
+    k_sort_scatter<<<chunks, kSortThreads, smem, st>>>(topk_idx, P, E, chunk_hist, perm, pos,
+                                                       offsets);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe
