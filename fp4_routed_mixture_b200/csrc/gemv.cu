@@ -4,16 +4,21 @@
 // GEMMs from packed FP4 weights and INT8 activations with integer
 // dot-product instructions, and names memory bandwidth and low M as the
 // limits.  On B200 the same regime is HBM-bound: every touched expert's FP4
-// weights are read exactly once, with 128-bit coalesced loads, while the few
-// token rows of that expert are reused from L1.
+// weights are read exactly once, in coalesced 16-byte pieces.
 //
 // Work: for every expert e with M_e > 0, units (tile of 32 weight rows, group
 // of up to kGroup tokens); each unit is K/128 items of 4 scale blocks.  The
 // flat item range is split evenly over all warps of the grid (stream-K), so
 // the load is balanced to within one item whatever the expert counts are.
+//
+// Every warp runs its own kStages-deep ring in shared memory: the cp.async
+// copies of item i + 1 -- the weights (every lane copies its own 16-byte code
+// slices, a warp-wide 512-byte coalesced access per block), the group's
+// activation bytes and block terms -- are in flight while item i is computed.
+//
 // Lane l of a warp owns weight row 32*tile + l and the full dot products of
 // that row with the group's token rows:
-//   * a 16-byte code load gives the lane one 32-element block (one scale);
+//   * a 16-byte code slice gives the lane one 32-element block (one scale);
 //   * nibbles become bytes 2*e2m1 + 12 in [0, 24] through two byte
 //     permutes (positive and negative code tables) and an OR;
 //   * __dp4a against the int8 activation bytes, started from -12 * (sum of
@@ -28,9 +33,25 @@
 
 namespace moe {
 
-constexpr int kGroup = 8;        // token rows per unit
-constexpr int kGemvWarps = 8;    // warps per CTA
+// Tuning (measured on B200, decode T=8 and T=64): a 2-deep ring per warp and
+// 8 warps per CTA (5 CTAs per SM) stream at ~96% of the measured copy
+// bandwidth.  Giving a warp two 32-row tiles per item (two weight streams 69 KB
+// apart) or deeper rings with fewer warps, and TMA bulk copies in place of the
+// per-lane 16-byte copies, were all slower.
+constexpr int kGroup = 4;          // token rows per unit
+constexpr int kGemvWarps = 8;      // warps per CTA; every warp runs its own pipeline
+constexpr int kStages = 2;         // shared-memory ring depth per warp
 constexpr int kGroupBytes = 2176;  // 4 scale blocks of 32 rows: 128 B scales + 4 x 512 B codes
+
+// One ring slot: one K group (4 blocks of 32 elements) of one 32-row tile,
+// plus the group's activation bytes and block terms.
+struct alignas(16) Slot {
+    uint8_t w[kGroupBytes];
+    int8_t x[kGroup][128];
+    int32_t init[kGroup][4];
+};
+constexpr int kSlotBytes = (int)sizeof(Slot);
+constexpr int kSmemBytes = kGemvWarps * kStages * kSlotBytes;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
@@ -44,25 +65,42 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // is 0 for every table byte.  So the positive table answers for sign 0 codes,
 // the negative table (selected with the sign bit flipped) for sign 1 codes,
 // and the other table returns 0.
-__device__ __forceinline__ void decode8(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    constexpr uint32_t kPos0 = 0x0F0E0D0Cu, kPos1 = 0x18141210u;  // 12 + {0,1,2,3,4,6,8,12}
-    constexpr uint32_t kNeg0 = 0x090A0B0Cu, kNeg1 = 0x00040608u;  // 12 - {0,1,2,3,4,6,8,12}
+constexpr uint32_t kPos0 = 0x0F0E0D0Cu, kPos1 = 0x18141210u;  // 12 + {0,1,2,3,4,6,8,12}
+constexpr uint32_t kNeg0 = 0x090A0B0Cu, kNeg1 = 0x00040608u;  // 12 - {0,1,2,3,4,6,8,12}
+
+// The four table words, held in registers for the whole kernel.  They are
+// derived from a kernel argument that is always zero, so that the compiler
+// keeps them in registers instead of re-materialising the immediates before
+// every byte permute.
+struct Tables {
+    uint32_t p0, p1, n0, n1;
+    __device__ __forceinline__ explicit Tables(uint32_t zero)
+        : p0(kPos0 ^ zero), p1(kPos1 ^ zero), n0(kNeg0 ^ zero), n1(kNeg1 ^ zero) {}
+};
+
+__device__ __forceinline__ void decode8(const Tables& t, uint32_t w, uint32_t& lo, uint32_t& hi) {
     const uint32_t wf = w ^ 0x88888888u;
-    lo = prmt(kPos0, kPos1, w) | prmt(kNeg0, kNeg1, wf);
-    hi = prmt(kPos0, kPos1, w >> 16) | prmt(kNeg0, kNeg1, wf >> 16);
+    lo = prmt(t.p0, t.p1, w) | prmt(t.n0, t.n1, wf);
+    hi = prmt(t.p0, t.p1, w >> 16) | prmt(t.n0, t.n1, wf >> 16);
 }
 
-__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
+// High word of the double 2^(S-128) for scale byte bb of the packed word sw:
+// one byte permute and one multiply-add ((S + 895) << 20).
+__device__ __forceinline__ double block_scale(uint32_t sw, int bb) {
+    const uint32_t S = __byte_perm(sw, 0u, 0x4440u + (uint32_t)bb);
+    return __hiloint2double((int)(S * 1048576u + 895u * 1048576u), 0);
 }
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+
+__device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 struct GemvArgs {
@@ -79,88 +117,198 @@ struct GemvArgs {
     int E;
     double* out;               // [P, N] fp64 accumulators, zeroed
     const int32_t* flag;       // device error word: a layout mismatch stops the kernel
+    uint32_t zero;             // always 0 (see Tables)
 };
 
+// A unit: expert, tile, first sorted row, number of rows.
+struct Unit {
+    int id, e, tile, i0, mc;
+};
+
+__device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
+    int lo = 0, hi = a.E;  // last e with unit_off[e] <= unit
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a.unit_off + mid) <= unit) lo = mid; else hi = mid;
+    }
+    Unit u;
+    u.id = unit;
+    u.e = lo;
+    const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
+    const int ngroups = (r1 - r0 + kGroup - 1) / kGroup;
+    const int local = unit - __ldg(a.unit_off + lo);
+    u.tile = local / ngroups;
+    u.i0 = r0 + (local % ngroups) * kGroup;
+    u.mc = min(kGroup, r1 - u.i0);
+    return u;
+}
+
+__device__ __forceinline__ int act_row(const GemvArgs& a, int i) {
+    return a.k_div ? __ldg(a.perm + i) / a.k_div : i;
+}
+
+// Integer dot product of one 32-element block (8 decoded words) with one
+// token's 32 activation bytes, started from the block term.
+__device__ __forceinline__ int block_dot(const uint32_t (&v)[8], const uint4& x0, const uint4& x1,
+                                         int init) {
+    int d0 = init, d1 = 0;
+    d0 = __dp4a((int)v[0], (int)x0.x, d0);
+    d1 = __dp4a((int)v[1], (int)x0.y, d1);
+    d0 = __dp4a((int)v[2], (int)x0.z, d0);
+    d1 = __dp4a((int)v[3], (int)x0.w, d1);
+    d0 = __dp4a((int)v[4], (int)x1.x, d0);
+    d1 = __dp4a((int)v[5], (int)x1.y, d1);
+    d0 = __dp4a((int)v[6], (int)x1.z, d0);
+    d1 = __dp4a((int)v[7], (int)x1.w, d1);
+    return d0 + d1;
+}
+
+// Single-token variant: the positive- and negative-table bytes of each word
+// feed two dot products instead of being merged first (the merge moves from
+// the ALU pipe to dp4a), worthwhile when one token carries the whole decode.
+__device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, const uint4& x0,
+                                               const uint4& x1, int init) {
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    int d0 = init, d1 = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t w = cw[j], wf = w ^ 0x88888888u;
+        d0 = __dp4a((int)prmt(t.p0, t.p1, w), (int)xw[2 * j], d0);
+        d1 = __dp4a((int)prmt(t.n0, t.n1, wf), (int)xw[2 * j], d1);
+        d0 = __dp4a((int)prmt(t.p0, t.p1, w >> 16), (int)xw[2 * j + 1], d0);
+        d1 = __dp4a((int)prmt(t.n0, t.n1, wf >> 16), (int)xw[2 * j + 1], d1);
+    }
+    return d0 + d1;
+}
+
 __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
-    const int lane = threadIdx.x & 31;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // packed weights built for other dims may be smaller than the offsets used here
     if (*(volatile const int32_t*)a.flag & FLAG_LAYOUT) return;
-    const long long gw = (long long)blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
+    const Tables tb(a.zero);
+    Slot* ring = reinterpret_cast<Slot*>(smem) + warp * kStages;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const long long gw = (long long)blockIdx.x * kGemvWarps + warp;
     const long long nw = (long long)gridDim.x * kGemvWarps;
     const int KG = a.K / 128;
-    const long long U = a.unit_off[a.E];
-    const long long W = U * KG;
-    const long long it1 = W * (gw + 1) / nw;
-    long long it = W * gw / nw;
-    while (it < it1) {
-        const int unit = (int)(it / KG);
-        const int kg0 = (int)(it % KG);
-        const long long rem = it1 - it;
-        const int kg1 = rem < (long long)(KG - kg0) ? kg0 + (int)rem : KG;
-        // expert of this unit: last e with unit_off[e] <= unit
-        int lo = 0, hi = a.E;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (__ldg(a.unit_off + mid) <= unit) lo = mid; else hi = mid;
+    const size_t tile_bytes = (size_t)KG * kGroupBytes;
+    const long long W = (long long)__ldg(a.unit_off + a.E) * KG;
+    const int it0 = (int)(W * gw / nw), it1 = (int)(W * (gw + 1) / nw);
+    if (it0 >= it1) return;
+
+    // per-lane byte offsets inside a slot: own scale word, own code slices, the
+    // 16-byte activation chunk (token lane/8, chunk lane%8) and block terms
+    // (token lane%4) this lane copies
+    const uint32_t o_sc = lane * 4, o_code = 128 + lane * 16;
+    const uint32_t o_x = (uint32_t)offsetof(Slot, x) + (lane >> 3) * 128 + (lane & 7) * 16;
+    const uint32_t o_init = (uint32_t)offsetof(Slot, init) + (lane & (kGroup - 1)) * 16;
+
+    // ---- fetch side: cp.async copies of one item into its slot ----
+    int f_left = it1 - it0;
+    int f_kg = it0 % KG, f_slot = 0;
+    Unit fu = unit_at(a, it0 / KG);
+    const uint8_t* f_w = nullptr;  // this lane's sources for the current item
+    const int8_t* f_x = nullptr;
+    const int32_t* f_i = nullptr;
+    auto start_unit = [&](int kg) {
+        f_w = a.w + (size_t)fu.e * a.expert_bytes + (size_t)fu.tile * tile_bytes + (size_t)kg * kGroupBytes;
+        f_x = a.act + (size_t)act_row(a, fu.i0 + min(lane >> 3, fu.mc - 1)) * a.K + kg * 128 + (lane & 7) * 16;
+        f_i = a.act_init + (size_t)act_row(a, fu.i0 + min(lane & (kGroup - 1), fu.mc - 1)) * (a.K / 32) +
+              kg * 4;
+    };
+    start_unit(f_kg);
+    auto issue = [&]() {
+        const uint32_t sb = ring_s + f_slot * kSlotBytes;
+        cp_async4(sb + o_sc, f_w + o_sc);
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) cp_async16(sb + o_code + bb * 512, f_w + o_code + bb * 512);
+        if ((lane >> 3) < fu.mc) cp_async16(sb + o_x, f_x);
+        if (lane < fu.mc) cp_async16(sb + o_init, f_i);
+        cp_async_commit();
+        --f_left;
+        f_slot = (f_slot + 1 == kStages) ? 0 : f_slot + 1;
+        if (++f_kg == KG) {
+            if (f_left > 0) {
+                f_kg = 0;
+                fu = unit_at(a, fu.id + 1);
+                start_unit(0);
+            }
+        } else {
+            f_w += kGroupBytes;
+            f_x += 128;
+            f_i += 4;
         }
-        const int e = lo;
-        const int r0 = __ldg(a.offsets + e), r1 = __ldg(a.offsets + e + 1);
-        const int ngroups = (r1 - r0 + kGroup - 1) / kGroup;
-        const int local = unit - __ldg(a.unit_off + e);
-        const int tile = local / ngroups;
-        const int i0 = r0 + (local % ngroups) * kGroup;
-        const int mc = min(kGroup, r1 - i0);
-        int arow[kGroup];
+    };
+
 #pragma unroll
-        for (int m = 0; m < kGroup; ++m) {
-            const int i = i0 + min(m, mc - 1);
-            arow[m] = a.k_div ? __ldg(a.perm + i) / a.k_div : i;
-        }
-        const uint8_t* tb = a.w + (size_t)e * a.expert_bytes + (size_t)tile * KG * kGroupBytes;
-        double acc[kGroup];
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (f_left > 0) issue();
+        else cp_async_commit();
+    }
+
+    // ---- compute side ----
+    Unit cu = unit_at(a, it0 / KG);
+    int c_kg = it0 % KG, c_slot = 0;
+    double acc[kGroup];
 #pragma unroll
-        for (int m = 0; m < kGroup; ++m) acc[m] = 0.0;
-        for (int kg = kg0; kg < kg1; ++kg) {
-            const uint8_t* gb = tb + (size_t)kg * kGroupBytes;
-            const uint32_t sw = ldg_u32(gb + lane * 4);
-            uint4 c[4];
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) c[bb] = ldg_stream(gb + 128 + bb * 512 + lane * 16);
+    for (int m = 0; m < kGroup; ++m) acc[m] = 0.0;
+    for (int it = it0; it < it1; ++it) {
+        if (f_left > 0) issue();
+        else cp_async_commit();
+        cp_async_wait<kStages - 1>();  // item `it` has landed (this lane's copies) ...
+        __syncwarp();                  // ... and every other lane's
+        const Slot& sl = ring[c_slot];
+        const uint32_t sw = *reinterpret_cast<const uint32_t*>(sl.w + o_sc);
+#ifndef MOE_GEMV_SPLIT
+#define MOE_GEMV_SPLIT 1
+#endif
+        if (MOE_GEMV_SPLIT && cu.mc == 1) {
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                const double sc = pow2_scale_minus128((sw >> (8 * bb)) & 0xffu);
+                const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + bb * 512);
+                const uint4 x0 = *reinterpret_cast<const uint4*>(&sl.x[0][bb * 32]);
+                const uint4 x1 = *reinterpret_cast<const uint4*>(&sl.x[0][bb * 32 + 16]);
+                const int d = block_dot_split(tb, c, x0, x1, sl.init[0][bb]);
+                acc[0] = __fma_rn((double)d, block_scale(sw, bb), acc[0]);
+            }
+        } else {
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + bb * 512);
                 uint32_t v[8];
-                decode8(c[bb].x, v[0], v[1]);
-                decode8(c[bb].y, v[2], v[3]);
-                decode8(c[bb].z, v[4], v[5]);
-                decode8(c[bb].w, v[6], v[7]);
-                const int blk = kg * 4 + bb;
+                decode8(tb, c.x, v[0], v[1]);
+                decode8(tb, c.y, v[2], v[3]);
+                decode8(tb, c.z, v[4], v[5]);
+                decode8(tb, c.w, v[6], v[7]);
+                const double sc = block_scale(sw, bb);
 #pragma unroll
                 for (int m = 0; m < kGroup; ++m) {
-                    if (m < mc) {
-                        const uint4* xp = reinterpret_cast<const uint4*>(a.act + (size_t)arow[m] * a.K +
-                                                                         blk * 32);
-                        const uint4 x0 = __ldg(xp), x1 = __ldg(xp + 1);
-                        int d = __ldg(a.act_init + (size_t)arow[m] * (a.K / 32) + blk);
-                        d = __dp4a((int)v[0], (int)x0.x, d);
-                        d = __dp4a((int)v[1], (int)x0.y, d);
-                        d = __dp4a((int)v[2], (int)x0.z, d);
-                        d = __dp4a((int)v[3], (int)x0.w, d);
-                        d = __dp4a((int)v[4], (int)x1.x, d);
-                        d = __dp4a((int)v[5], (int)x1.y, d);
-                        d = __dp4a((int)v[6], (int)x1.z, d);
-                        d = __dp4a((int)v[7], (int)x1.w, d);
-                        acc[m] = __fma_rn((double)d, sc, acc[m]);
+                    if (m < cu.mc) {
+                        const uint4 x0 = *reinterpret_cast<const uint4*>(&sl.x[m][bb * 32]);
+                        const uint4 x1 = *reinterpret_cast<const uint4*>(&sl.x[m][bb * 32 + 16]);
+                        acc[m] = __fma_rn((double)block_dot(v, x0, x1, sl.init[m][bb]), sc, acc[m]);
                     }
                 }
             }
         }
-        const int n = tile * 32 + lane;
+        __syncwarp();  // every lane is done with the slot before it is refilled
+        c_slot = (c_slot + 1 == kStages) ? 0 : c_slot + 1;
+        if (++c_kg == KG || it + 1 == it1) {
+            const int n = cu.tile * 32 + lane;
 #pragma unroll
-        for (int m = 0; m < kGroup; ++m)
-            if (m < mc) atomicAdd(a.out + (size_t)(i0 + m) * a.N + n, acc[m]);
-        it += kg1 - kg0;
+            for (int m = 0; m < kGroup; ++m) {
+                if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.i0 + m) * a.N + n, acc[m]);
+                acc[m] = 0.0;
+            }
+            if (c_kg == KG && it + 1 < it1) {
+                c_kg = 0;
+                cu = unit_at(a, cu.id + 1);
+            }
+        }
     }
+    cp_async_wait<0>();
 }
 
 // Units per expert for both matrices and their exclusive scans (one warp;
@@ -205,7 +353,8 @@ static int gemv_grid() {
         int dev = 0, sms = 0, per_sm = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv, kGemvWarps * 32, 0);
+        cudaFuncSetAttribute(k_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv, kGemvWarps * 32, kSmemBytes);
         grid = sms * (per_sm > 0 ? per_sm : 1);
     }
     return grid;
@@ -222,8 +371,8 @@ cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, con
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
                         const int32_t* flag, cudaStream_t st) {
-    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag};
-    k_gemv<<<gemv_grid(), kGemvWarps * 32, 0, st>>>(a);
+    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag, 0u};
+    k_gemv<<<gemv_grid(), kGemvWarps * 32, kSmemBytes, st>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -196,7 +196,9 @@ def test_sort_parity(moe, name):
                                    (1025, 1, 16), (683, 3, 1024), (20000, 6, 256), (0, 6, 256)])
 def test_sort_sizes(moe, T, k, E):
     rng = np.random.default_rng(T + k + E)
-    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32).reshape(T, k)
+    idx = np.zeros((T, k), np.int32)
+    for t in range(T):
+        idx[t] = rng.permutation(E)[:k]
     if T >= 100:  # skew: half the pairs on one expert
         idx[: T // 2, 0] = E - 1 if k == 1 else idx[: T // 2, 0]
     perm, pos, offsets = moe.moe_sort(cu(idx), E)
