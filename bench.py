@@ -49,6 +49,11 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-run", action="store_true",
+                    help="no timing, no JSON: pack the workload and run --steps layer calls "
+                         "(the command profiled under ncu)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="with --profile-run: override E (a smaller capture of the same kernels)")
     return ap.parse_args()
 
 
@@ -294,8 +299,32 @@ def roofline_hbm(r: dict, peaks: dict, traffic):
             "peak_source": peaks["source"] + " (hbm_gbs: stream copy)"}
 
 
+def profile_run(a):
+    import dataclasses
+
+    import torch
+
+    import fp4_routed_mixture_b200 as moe
+    w = synth.WORKLOADS[a.workload]
+    if a.experts:
+        w = dataclasses.replace(w, name=f"{w.name}_E{a.experts}", E=a.experts)
+    d = synth.make(w)
+    cu = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    packed = moe.moe_pack_weights(*[cu(d[n]) for n in ("w1_codes", "w1_scales", "w2_codes", "w2_scales")])
+    torch.cuda.empty_cache()
+    logits, x = cu(d["logits"]), cu(d["x"]).view(torch.bfloat16)
+    ws = torch.empty(moe.moe_layer_workspace_bytes(w.T, w.H, w.I, w.E, w.k), dtype=torch.uint8, device="cuda")
+    for _ in range(a.steps or 3):
+        y = moe.moe_layer_forward(logits, x, packed, w.H, w.I, w.E, w.k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_check_device_flag(ws) == 0
+    print(f"profile run ok: {w.name}, {a.steps or 3} steps, max|y| = {float(y.float().abs().max())}")
+
+
 def main():
     a = parse()
+    if a.profile_run:
+        return profile_run(a)
     if a.impl == "reference":
         return main_reference(a)
     steps = a.steps if a.steps is not None else 2000
