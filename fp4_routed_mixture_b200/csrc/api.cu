@@ -213,14 +213,14 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                             uoff1, E, gacc, flag, stream), "W1");
+                             uoff1, E, gacc, flag, I, stream), "W1");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_swiglu_hquant(gacc, sx, perm, P, k, I, hq, sh, hinit,
                                       dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, stream),
             "SwiGLU + h quant");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                             uoff2, E, yacc, flag, stream), "W2");
+                             uoff2, E, yacc, flag, 0, stream), "W2");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, sh, gates, pos, T, k, H, y_bf16, stream), "combine");
 #undef MOE_TRY

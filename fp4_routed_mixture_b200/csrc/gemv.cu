@@ -19,6 +19,8 @@
 // Lane l of a warp owns weight row 32*tile + l and the full dot products of
 // that row with the group's token rows:
 //   * a 16-byte code slice gives the lane one 32-element block (one scale);
+//     the warp's 32 slices of a block are one contiguous 512-byte piece of the
+//     packed chunk (layout in pack.cu);
 //   * nibbles become bytes 2*e2m1 + 12 in [0, 24] through two byte
 //     permutes (positive and negative code tables) and an OR;
 //   * __dp4a against the int8 activation bytes, started from -12 * (sum of
@@ -42,6 +44,7 @@ constexpr int kGroup = 4;          // token rows per unit
 constexpr int kGemvWarps = 8;      // warps per CTA; every warp runs its own pipeline
 constexpr int kStages = 2;         // shared-memory ring depth per warp
 constexpr int kGroupBytes = 2176;  // 4 scale blocks of 32 rows: 128 B scales + 4 x 512 B codes
+constexpr int kChunkBytes = 8704;  // packed chunk: 4 scale blocks of 128 rows (see pack.cu)
 
 // One ring slot: one K group (4 blocks of 32 elements) of one 32-row tile,
 // plus the group's activation bytes and block terms.
@@ -117,8 +120,16 @@ struct GemvArgs {
     int E;
     double* out;               // [P, N] fp64 accumulators, zeroed
     const int32_t* flag;       // device error word: a layout mismatch stops the kernel
+    int gate_up_half;          // > 0 (= I) for W1: device rows interleave gate and up rows
     uint32_t zero;             // always 0 (see Tables)
 };
+
+// Canonical row (output column) of a device row (see the layout in pack.cu).
+__device__ __forceinline__ int canonical_row(int d, int gate_up_half) {
+    if (gate_up_half <= 0) return d;
+    const int rb = d >> 7, r = d & 127;
+    return (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
+}
 
 // A unit: expert, tile, first sorted row, number of rows.
 struct Unit {
@@ -182,7 +193,7 @@ __device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, 
     return d0 + d1;
 }
 
-__global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // packed weights built for other dims may be smaller than the offsets used here
@@ -193,14 +204,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
     const long long gw = (long long)blockIdx.x * kGemvWarps + warp;
     const long long nw = (long long)gridDim.x * kGemvWarps;
     const int KG = a.K / 128;
-    const size_t tile_bytes = (size_t)KG * kGroupBytes;
     const long long W = (long long)__ldg(a.unit_off + a.E) * KG;
     const int it0 = (int)(W * gw / nw), it1 = (int)(W * (gw + 1) / nw);
     if (it0 >= it1) return;
 
     // per-lane byte offsets inside a slot: own scale word, own code slices, the
     // 16-byte activation chunk (token lane/8, chunk lane%8) and block terms
-    // (token lane%4) this lane copies
+    // (token lane%4) this lane copies.  In the packed chunk of 8704 bytes the
+    // lane's scale word of tile t is at lane*16 + t*4 and its code slice of
+    // block j at 512 + j*2048 + t*512 + lane*16.
     const uint32_t o_sc = lane * 4, o_code = 128 + lane * 16;
     const uint32_t o_x = (uint32_t)offsetof(Slot, x) + (lane >> 3) * 128 + (lane & 7) * 16;
     const uint32_t o_init = (uint32_t)offsetof(Slot, init) + (lane & (kGroup - 1)) * 16;
@@ -212,8 +224,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
     const uint8_t* f_w = nullptr;  // this lane's sources for the current item
     const int8_t* f_x = nullptr;
     const int32_t* f_i = nullptr;
+    uint32_t g_sc = 0, g_code = 0;  // this lane's offsets inside a packed chunk (tile dependent)
     auto start_unit = [&](int kg) {
-        f_w = a.w + (size_t)fu.e * a.expert_bytes + (size_t)fu.tile * tile_bytes + (size_t)kg * kGroupBytes;
+        const int rb = fu.tile >> 2, t = fu.tile & 3;
+        g_sc = lane * 16 + t * 4;
+        g_code = 512 + t * 512 + lane * 16;
+        f_w = a.w + (size_t)fu.e * a.expert_bytes + ((size_t)rb * KG + kg) * kChunkBytes;
         f_x = a.act + (size_t)act_row(a, fu.i0 + min(lane >> 3, fu.mc - 1)) * a.K + kg * 128 + (lane & 7) * 16;
         f_i = a.act_init + (size_t)act_row(a, fu.i0 + min(lane & (kGroup - 1), fu.mc - 1)) * (a.K / 32) +
               kg * 4;
@@ -221,9 +237,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
     start_unit(f_kg);
     auto issue = [&]() {
         const uint32_t sb = ring_s + f_slot * kSlotBytes;
-        cp_async4(sb + o_sc, f_w + o_sc);
+        cp_async4(sb + o_sc, f_w + g_sc);
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) cp_async16(sb + o_code + bb * 512, f_w + o_code + bb * 512);
+        for (int bb = 0; bb < 4; ++bb) cp_async16(sb + o_code + bb * 512, f_w + g_code + bb * 2048);
         if ((lane >> 3) < fu.mc) cp_async16(sb + o_x, f_x);
         if (lane < fu.mc) cp_async16(sb + o_init, f_i);
         cp_async_commit();
@@ -236,7 +252,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
                 start_unit(0);
             }
         } else {
-            f_w += kGroupBytes;
+            f_w += kChunkBytes;
             f_x += 128;
             f_i += 4;
         }
@@ -296,7 +312,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k_gemv(GemvArgs a) {
         __syncwarp();  // every lane is done with the slot before it is refilled
         c_slot = (c_slot + 1 == kStages) ? 0 : c_slot + 1;
         if (++c_kg == KG || it + 1 == it1) {
-            const int n = cu.tile * 32 + lane;
+            const int n = canonical_row(cu.tile * 32 + lane, a.gate_up_half);
 #pragma unroll
             for (int m = 0; m < kGroup; ++m) {
                 if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.i0 + m) * a.N + n, acc[m]);
@@ -370,8 +386,9 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int tiles1, int tiles2, i
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, cudaStream_t st) {
-    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag, 0u};
+                        const int32_t* flag, int gate_up_half, cudaStream_t st) {
+    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
+               gate_up_half, 0u};
     k_gemv<<<gemv_grid(), kGemvWarps * 32, kSmemBytes, st>>>(a);
     count_launches(1);
     return cudaGetLastError();

@@ -46,7 +46,7 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int tiles1, int tiles2, i
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, cudaStream_t st);
+                        const int32_t* flag, int gate_up_half, cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* sh, const float* gates,
                            const int32_t* pos, int T, int k, int H, void* y, cudaStream_t st);

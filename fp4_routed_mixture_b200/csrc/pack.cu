@@ -6,17 +6,25 @@
 // is checked by the exact inverse, moe_unpack_weights, whose output must
 // reproduce the canonical bytes.
 //
-// Streaming device layout of one expert matrix with N rows and K inputs (per
-// expert, experts back to back; W1 region then W2 region):
-//   tile tau = 32 consecutive rows (row n = 32*tau + lane), tiles back to back;
-//   inside a tile, K/128 groups of 4 scale blocks, each 2176 bytes:
-//     [  0, 128)  32 lanes x 4 bytes: the lane's UE8M0 scales of blocks 4g..4g+3
-//     [128, 640)  32 lanes x 16 bytes: codes of block 4g   (32 nibbles, canonical order)
-//     [640,1152)  block 4g+1, [1152,1664) block 4g+2, [1664,2176) block 4g+3
-// A warp reading one 512-byte code slice hands each lane one 32-element block
-// of its own row, so weight loads are fully coalesced 128-bit loads and no
-// cross-lane reduction is needed.  The layout is the canonical bytes moved,
-// so its size equals the canonical size.
+// Device layout (one layout serves both the CUDA-core streaming GEMM and the
+// tensor-core GEMM).  Per expert, W1 region then W2 region; one expert matrix
+// with N rows and K inputs is split into 128-row blocks rb and 128-input
+// groups g, chunk (rb, g) at byte offset (rb * K/128 + g) * 8704:
+//   [   0,  512)  scales: byte l*16 + t*4 + j = UE8M0 scale of device row
+//                 rb*128 + t*32 + l, input block 4g + j (l < 32, t < 4, j < 4);
+//                 the tensor cores' 128-row x 4-block scale-factor atom
+//   [ 512, 8704)  codes:  16 bytes at 512 + j*2048 + t*512 + l*16 = the 32 E2M1
+//                 codes (canonical nibble order) of that row and block; i.e. for
+//                 every block j the 128 rows' 16-byte pieces back to back, the
+//                 no-swizzle K-major core-matrix order of the tensor cores
+// A warp of the streaming GEMM (lane = row of a 32-row tile t) reads one
+// 512-byte contiguous slice per block; the tensor-core producer fetches a whole
+// chunk with one bulk copy.
+// Device rows of W2 are its canonical rows.  Device rows of W1 interleave gate
+// and up per 128-row block: device row rb*128 + r is gate row rb*64 + r for
+// r < 64 and up row I + rb*64 + (r - 64) otherwise, so every 128-row block
+// holds the gate and up rows of the same 64 outputs.
+// The layout moves the canonical bytes, so its size equals the canonical size.
 #include "kernels.cuh"
 #include "moe_common.cuh"
 
@@ -29,24 +37,27 @@ struct PackHeader {
 };
 
 constexpr uint32_t kPackMagic = 0x34454F4Du;  // "MOE4"
-constexpr uint32_t kPackVersion = 1;
+constexpr uint32_t kPackVersion = 2;
 
 __host__ __device__ inline size_t matrix_bytes(int N, int K) { return (size_t)N * K * 17 / 32; }
 
-// byte offset, inside one expert matrix, of the scale byte / first code byte of (row n, block b)
-__host__ __device__ inline size_t dl_scale_off(int n, int b, int K) {
-    const int tau = n >> 5, lane = n & 31, g = b >> 2, bb = b & 3;
-    return (size_t)tau * (K / 128) * 2176 + (size_t)g * 2176 + lane * 4 + bb;
+// byte offsets, inside one expert matrix, of the scale byte / first code byte of
+// (device row d, input block b)
+__host__ __device__ inline size_t dl_scale_off(int d, int b, int K) {
+    const int rb = d >> 7, t = (d >> 5) & 3, l = d & 31, g = b >> 2, j = b & 3;
+    return ((size_t)rb * (K / 128) + g) * 8704 + l * 16 + t * 4 + j;
 }
-__host__ __device__ inline size_t dl_code_off(int n, int b, int K) {
-    const int tau = n >> 5, lane = n & 31, g = b >> 2, bb = b & 3;
-    return (size_t)tau * (K / 128) * 2176 + (size_t)g * 2176 + 128 + bb * 512 + lane * 16;
+__host__ __device__ inline size_t dl_code_off(int d, int b, int K) {
+    const int rb = d >> 7, t = (d >> 5) & 3, l = d & 31, g = b >> 2, j = b & 3;
+    return ((size_t)rb * (K / 128) + g) * 8704 + 512 + j * 2048 + t * 512 + l * 16;
 }
 
-// One thread per (expert, row, 32-element block).  forward: canonical -> device.
+// One thread per (expert, device row, 32-element block).  forward: canonical ->
+// device.  gate_up_half > 0 selects the W1 row interleave with that I.
 template <bool kForward>
 __global__ void k_pack_matrix(uint8_t* __restrict__ dev, uint8_t* __restrict__ codes,
-                              uint8_t* __restrict__ scales, int E, int N, int K, int32_t* flag) {
+                              uint8_t* __restrict__ scales, int E, int N, int K, int gate_up_half,
+                              int32_t* flag) {
     const int nb = K / 32;
     const size_t total = (size_t)E * N * nb;
     const size_t mbytes = matrix_bytes(N, K);
@@ -54,14 +65,20 @@ __global__ void k_pack_matrix(uint8_t* __restrict__ dev, uint8_t* __restrict__ c
     for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
          id += (size_t)gridDim.x * blockDim.x) {
         const int b = (int)(id % nb);
-        const size_t rn = id / nb;
-        const int n = (int)(rn % N);
-        const int e = (int)(rn / N);
+        const size_t rd = id / nb;
+        const int drow = (int)(rd % N);
+        const int e = (int)(rd / N);
+        int crow = drow;  // canonical row of this device row
+        if (gate_up_half > 0) {
+            const int rb = drow >> 7, r = drow & 127;
+            crow = (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
+        }
+        const size_t rn = (size_t)e * N + crow;
         uint8_t* d = dev + (size_t)e * mbytes;
         uint4* cc = reinterpret_cast<uint4*>(codes + rn * (K / 2) + (size_t)b * 16);
         uint8_t* cs = scales + rn * nb + b;
-        uint4* dc = reinterpret_cast<uint4*>(d + dl_code_off(n, b, K));
-        uint8_t* ds = d + dl_scale_off(n, b, K);
+        uint4* dc = reinterpret_cast<uint4*>(d + dl_code_off(drow, b, K));
+        uint8_t* ds = d + dl_scale_off(drow, b, K);
         if (kForward) {
             const uint8_t s = *cs;
             if (s == 0xFF) bad = true;
@@ -123,18 +140,18 @@ cudaError_t launch_pack(int H, int I, int E, const uint8_t* w1c, const uint8_t* 
         count_launches(1);
         const size_t n1 = (size_t)E * 2 * I * (H / 32), n2 = (size_t)E * H * (I / 32);
         k_pack_matrix<true><<<grid_for(n1), 256, 0, st>>>(base + L.w1, (uint8_t*)w1c, (uint8_t*)w1s,
-                                                          E, 2 * I, H, &hdr->flag);
+                                                          E, 2 * I, H, I, &hdr->flag);
         count_launches(1);
         k_pack_matrix<true><<<grid_for(n2), 256, 0, st>>>(base + L.w2, (uint8_t*)w2c, (uint8_t*)w2s,
-                                                          E, H, I, &hdr->flag);
+                                                          E, H, I, 0, &hdr->flag);
         count_launches(1);
     } else {
         const size_t n1 = (size_t)E * 2 * I * (H / 32), n2 = (size_t)E * H * (I / 32);
         k_pack_matrix<false><<<grid_for(n1), 256, 0, st>>>(base + L.w1, out_w1c, out_w1s, E, 2 * I,
-                                                           H, nullptr);
+                                                           H, I, nullptr);
         count_launches(1);
         k_pack_matrix<false><<<grid_for(n2), 256, 0, st>>>(base + L.w2, out_w2c, out_w2s, E, H, I,
-                                                           nullptr);
+                                                           0, nullptr);
         count_launches(1);
     }
     return cudaGetLastError();

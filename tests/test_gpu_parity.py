@@ -125,14 +125,16 @@ def test_mispermuted_w2_layout_is_caught(moe, workload_data):
     d, w = workload_data(name), synth.WORKLOADS[name]
     r = run_layer(moe, d, w, debug=False)
     packed = r["packed"]
-    # swap lanes 0 and 1 of every 16-byte code chunk of one used expert's W2 tiles
+    # swap the code pieces of rows 0 and 1 of every 128-row block of one used
+    # expert's W2 (packed chunk of 8704 bytes: 512 scale bytes, then for each
+    # of 4 blocks the 128 rows' 16-byte pieces)
     e = int(r["idx"][0, 0])
     w2_off = 256 + w.E * (2 * w.I * w.H * 17 // 32) + e * (w.H * w.I * 17 // 32)
-    tile_bytes = (w.I // 128) * 2176
-    for tile in range(w.H // 32):
-        for g in range(w.I // 128):
-            for bb in range(4):
-                o = w2_off + tile * tile_bytes + g * 2176 + 128 + bb * 512
+    KG = w.I // 128
+    for rb in range(w.H // 128):
+        for g in range(KG):
+            for j in range(4):
+                o = w2_off + (rb * KG + g) * 8704 + 512 + j * 2048
                 a = packed[o:o + 16].clone()
                 packed[o:o + 16] = packed[o + 16:o + 32]
                 packed[o + 16:o + 32] = a
