@@ -25,7 +25,7 @@ FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_LAYOUT, FLAG_TIMEOUT, FLAG_BOUNDS = 1, 2, 
 SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack_weights",
            "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_workspace_bytes",
            "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
-           "moe_launch_count", "moe_check_device_flag"]
+           "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
 
 
 class MoeError(RuntimeError):
@@ -65,6 +65,8 @@ def _load():
         "moe_quant_rows_f32": ([vp, i32, i32, vp, vp, vp], i32),
         "moe_exp_f32": ([vp, vp, ctypes.c_int64, vp], i32),
         "moe_swiglu_f32": ([vp, vp, vp, ctypes.c_int64, vp], i32),
+        "moe_set_option": ([i32, i32], i32),
+        "moe_get_option": ([i32], i32),
         "moe_launch_count": ([], ctypes.c_ulonglong),
         "moe_check_device_flag": ([vp, ctypes.POINTER(ctypes.c_int32), vp], i32),
     }
@@ -260,6 +262,17 @@ def moe_swiglu_f32(g, u, stream=None):
     h = torch.empty_like(g)
     _check(lib.moe_swiglu_f32(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream(stream)))
     return h
+
+
+MOE_OPT_TC_MIN_ROWS = 1
+
+
+def moe_set_option(option: int, value: int):
+    _check(lib.moe_set_option(option, value))
+
+
+def moe_get_option(option: int) -> int:
+    return int(lib.moe_get_option(option))
 
 
 def moe_launch_count() -> int:

@@ -52,8 +52,13 @@ int check_dims(const moe_dims* d, bool need_T) {
     return MOE_OK;
 }
 
+// Experts with at least this many rows use the tensor-core GEMM (see
+// moe_set_option); the others the streaming GEMM.
+int g_tc_min_rows = 32;
+
 struct WsLayout {
-    size_t flag, uoff1, uoff2, sx, xq, xinit, hq, sh, hinit, gacc, yacc, total;
+    size_t flag, uoff1, uoff2, toff1, toff2, sx, xq, xinit, hq, sh, hinit, px, ph, gacc, yacc, total;
+    int P_pad;
 };
 
 WsLayout ws_layout(const moe_dims& d, long long T) {
@@ -64,12 +69,19 @@ WsLayout ws_layout(const moe_dims& d, long long T) {
     L.flag = o; o += 256;
     L.uoff1 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.uoff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.toff1 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.toff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.sx = o; o += align_up(4 * (size_t)T, 256);
     L.xq = o; o += align_up((size_t)T * d.H, 256);
     L.xinit = o; o += align_up(4 * (size_t)T * (d.H / 32), 256);
     L.hq = o; o += align_up(P * d.I, 256);
     L.sh = o; o += align_up(4 * P, 256);
     L.hinit = o; o += align_up(4 * P * (d.I / 32), 256);
+    // digit planes of the tensor-core GEMM: 3 x [K/32][P_pad][16 bytes]; the
+    // last tile of an expert may read up to 128 rows past the end
+    L.P_pad = (int)P + 128;
+    L.px = o; o += align_up(3 * (size_t)(d.H / 32) * L.P_pad * 16, 256);
+    L.ph = o; o += align_up(3 * (size_t)(d.I / 32) * L.P_pad * 16, 256);
     L.gacc = o; o += align_up(8 * P * 2 * d.I, 256);   // gacc and yacc are adjacent:
     L.yacc = o; o += align_up(8 * P * d.H, 256);        // one memset clears both
     L.total = o;
@@ -208,19 +220,36 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     MOE_TRY(moe::launch_check_header(packed, H, I, E, flag, stream), "header check");
     MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, dbg ? dbg->xq : nullptr,
                                dbg ? dbg->sx : nullptr, stream), "x quant");
-    MOE_TRY(moe::launch_plan(offsets, E, 2 * I / 32, H / 32, uoff1, uoff2, stream), "plan");
+    int32_t* toff1 = (int32_t*)(w + L.toff1);
+    int32_t* toff2 = (int32_t*)(w + L.toff2);
+    uint8_t* px = (uint8_t*)(w + L.px);
+    uint8_t* ph = (uint8_t*)(w + L.ph);
+    const size_t px_stride = (size_t)(H / 32) * L.P_pad * 16, ph_stride = (size_t)(I / 32) * L.P_pad * 16;
+    // an expert has at most T rows, so the tensor-core path is skipped without
+    // reading any count when T < tc_min
+    const bool use_tc = T >= g_tc_min_rows;
+    MOE_TRY(moe::launch_plan(offsets, E, 2 * I, H, use_tc ? g_tc_min_rows : 0x7fffffff, uoff1, uoff2,
+                             toff1, toff2, stream), "plan");
+    if (use_tc) MOE_TRY(moe::launch_planes(xq, H, perm, k, P, L.P_pad, px, px_stride, stream), "x planes");
     MOE_TRY(cudaMemsetAsync(gacc, 0, L.total - L.gacc, stream), "accumulator clear");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
                              uoff1, E, gacc, flag, I, stream), "W1");
+    if (use_tc)
+        MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, px_stride, L.P_pad,
+                                    offsets, toff1, E, gacc, flag, stream), "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_swiglu_hquant(gacc, sx, perm, P, k, I, hq, sh, hinit,
                                       dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, stream),
             "SwiGLU + h quant");
+    if (use_tc) MOE_TRY(moe::launch_planes(hq, I, perm, 0, P, L.P_pad, ph, ph_stride, stream), "h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
                              uoff2, E, yacc, flag, 0, stream), "W2");
+    if (use_tc)
+        MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, ph_stride, L.P_pad, offsets,
+                                    toff2, E, yacc, flag, stream), "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, sh, gates, pos, T, k, H, y_bf16, stream), "combine");
 #undef MOE_TRY
@@ -303,6 +332,21 @@ int moe_swiglu_f32(const float* g, const float* u, float* h, int64_t n, cudaStre
 }
 
 unsigned long long moe_launch_count(void) { return moe::g_launches.load(); }
+
+int moe_set_option(int option, int value) {
+    g_last_error.clear();
+    if (option == MOE_OPT_TC_MIN_ROWS) {
+        if (value < 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_MIN_ROWS must be >= 1");
+        g_tc_min_rows = value;
+        return MOE_OK;
+    }
+    return fail(MOE_ERR_INVALID_ARG, "moe_set_option: unknown option %d", option);
+}
+
+int moe_get_option(int option) {
+    if (option == MOE_OPT_TC_MIN_ROWS) return g_tc_min_rows;
+    return -1;
+}
 
 int moe_check_device_flag(const void* ws, int32_t* out_flag, cudaStream_t stream) {
     g_last_error.clear();

@@ -327,40 +327,56 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
     cp_async_wait<0>();
 }
 
-// Units per expert for both matrices and their exclusive scans (one warp;
-// lane l owns a contiguous slice of experts).
-__global__ void k_plan(const int32_t* __restrict__ offsets, int E, int tiles1, int tiles2,
-                       int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2) {
+// Work split per expert: experts with at least tc_min rows go to the
+// tensor-core GEMM (tiles of 128 weight rows x 128 token rows), the others to
+// the streaming GEMM (units of 32 weight rows x kGroup tokens).  Writes the
+// exclusive scans over experts of the streaming units of W1/W2 and of the
+// tensor-core tiles of W1/W2.  One warp; lane l owns a contiguous slice of
+// experts.
+__global__ void k_plan(const int32_t* __restrict__ offsets, int E, int n1, int n2, int tc_min,
+                       int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
+                       int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2) {
     const int lane = threadIdx.x;
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-    int s1 = 0, s2 = 0;
+    auto counts = [&](int e, int& u1, int& u2, int& t1, int& t2) {
+        const int m = offsets[e + 1] - offsets[e];
+        const bool tc = m >= tc_min;
+        const int g = tc ? 0 : (m + kGroup - 1) / kGroup;
+        const int nb = tc ? (m + 127) / 128 : 0;
+        u1 = g * (n1 / 32);
+        u2 = g * (n2 / 32);
+        t1 = nb * (n1 / 128);
+        t2 = nb * (n2 / 128);
+    };
+    int s[4] = {0, 0, 0, 0};
     for (int e = e0; e < e1; ++e) {
-        const int g = (offsets[e + 1] - offsets[e] + kGroup - 1) / kGroup;
-        s1 += g * tiles1;
-        s2 += g * tiles2;
+        int c[4];
+        counts(e, c[0], c[1], c[2], c[3]);
+        for (int j = 0; j < 4; ++j) s[j] += c[j];
     }
-    int x1 = s1, x2 = s2;
+    int x[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y1 = __shfl_up_sync(0xffffffffu, x1, o), y2 = __shfl_up_sync(0xffffffffu, x2, o);
-        if (lane >= o) {
-            x1 += y1;
-            x2 += y2;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int y = __shfl_up_sync(0xffffffffu, x[j], o);
+            if (lane >= o) x[j] += y;
         }
     }
-    int r1 = x1 - s1, r2 = x2 - s2;  // exclusive prefix
+    int r[4];
+    for (int j = 0; j < 4; ++j) r[j] = x[j] - s[j];  // exclusive prefix
+    int32_t* outs[4] = {unit_off1, unit_off2, tile_off1, tile_off2};
     for (int e = e0; e < e1; ++e) {
-        unit_off1[e] = r1;
-        unit_off2[e] = r2;
-        const int g = (offsets[e + 1] - offsets[e] + kGroup - 1) / kGroup;
-        r1 += g * tiles1;
-        r2 += g * tiles2;
+        int c[4];
+        counts(e, c[0], c[1], c[2], c[3]);
+        for (int j = 0; j < 4; ++j) {
+            outs[j][e] = r[j];
+            r[j] += c[j];
+        }
     }
-    if (lane == 31) {
-        unit_off1[E] = x1;
-        unit_off2[E] = x2;
-    }
+    if (lane == 31)
+        for (int j = 0; j < 4; ++j) outs[j][E] = x[j];
 }
 
 static int gemv_grid() {
@@ -376,9 +392,9 @@ static int gemv_grid() {
     return grid;
 }
 
-cudaError_t launch_plan(const int32_t* offsets, int E, int tiles1, int tiles2, int32_t* unit_off1,
-                        int32_t* unit_off2, cudaStream_t st) {
-    k_plan<<<1, 32, 0, st>>>(offsets, E, tiles1, tiles2, unit_off1, unit_off2);
+cudaError_t launch_plan(const int32_t* offsets, int E, int n1, int n2, int tc_min, int32_t* unit_off1,
+                        int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, cudaStream_t st) {
+    k_plan<<<1, 32, 0, st>>>(offsets, E, n1, n2, tc_min, unit_off1, unit_off2, tile_off1, tile_off2);
     count_launches(1);
     return cudaGetLastError();
 }

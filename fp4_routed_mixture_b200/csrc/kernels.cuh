@@ -41,12 +41,20 @@ cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, c
 cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
                               cudaStream_t st);
 
-cudaError_t launch_plan(const int32_t* offsets, int E, int tiles1, int tiles2, int32_t* unit_off1,
-                        int32_t* unit_off2, cudaStream_t st);
+cudaError_t launch_plan(const int32_t* offsets, int E, int n1, int n2, int tc_min, int32_t* unit_off1,
+                        int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, cudaStream_t st);
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
                         const int32_t* flag, int gate_up_half, cudaStream_t st);
+
+size_t tc_smem_bytes();
+cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
+                          int P_pad, uint8_t* planes, size_t plane_stride, cudaStream_t st);
+cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
+                           const uint8_t* planes, size_t plane_stride, int P_pad,
+                           const int32_t* offsets, const int32_t* tile_off, int E, double* out,
+                           int32_t* flag, cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* sh, const float* gates,
                            const int32_t* pos, int T, int k, int H, void* y, cudaStream_t st);

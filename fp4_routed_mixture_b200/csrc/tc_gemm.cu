@@ -1,0 +1,473 @@
+// Tensor-core grouped GEMM for experts with many rows (prefill).
+//
+// "DeepSeek-V4-Flash on AMD gfx90a" (abstract) moves its prefill expert GEMMs
+// onto matrix-core kernels with better reuse of the packed weights.  On B200
+// the same step runs on the 5th-generation tensor cores with the FP4 weights
+// consumed natively: tcgen05.mma kind::mxf4 with block scaling (E2M1 operands,
+// one UE8M0 scale per 32 inputs), operands staged in shared memory by TMA bulk
+// copies, accumulators in tensor memory.
+//
+// Operands (swap-AB: the weights take the 128-row M side, tokens the N side):
+//   A = one 128-row block of an expert's weights; each 128-input group is one
+//       packed chunk (pack.cu): 512 scale bytes in the tensor cores' 128 x 4
+//       scale-factor atom, then 8 KB of codes in no-swizzle K-major
+//       core-matrix order.  One bulk copy per chunk.
+//   B = the INT8 activations of the expert's sorted rows, written exactly as
+//       three E2M1 digit planes: q = 64*a + 8*b + c with a, b, c in [-4, 3]
+//       (balanced base-8 digits; every digit is an E2M1 value).  Plane p has
+//       the constant scale 2^(6 - 3p).  Each plane is stored chunk-major
+//       ([K/32][rows][16 bytes]) so that the N rows of a tile are contiguous.
+//   D (TMEM, fp32) = sum over planes of A * SFA * B_p * SFB_p = sum_k w * q:
+//       the same exact sum the CUDA-core kernel forms (every product is an
+//       integer multiple of the row's smallest weight scale).
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      producer: bulk copies of A and the three B planes into a
+//               6-stage ring (mbarrier transaction counts);
+//   warp 1      MMA issuer: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs per
+//               stage, tcgen05.commit frees the stage / publishes the tile;
+//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld) -> fp64 accumulators
+//               in global memory, one thread per weight row; two accumulator
+//               buffers in TMEM let the epilogue overlap the next tile's MMAs.
+// Every wait is bounded in time; a wait that gives up raises FLAG_TIMEOUT and
+// the roles wind down (copies in flight are waited for, TMEM is freed).
+#include "kernels.cuh"
+#include "moe_common.cuh"
+
+namespace moe {
+
+constexpr int TC_BM = 128;                     // weight rows per tile (MMA M)
+constexpr int TC_BN = 128;                     // token rows per tile (largest MMA N used)
+constexpr int TC_STAGES = 6;
+constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
+constexpr int TC_B_PLANE_BYTES = TC_BN * 64;   // 128 rows x 128 inputs, 4 bits each
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + 3 * TC_B_PLANE_BYTES;
+constexpr int TC_THREADS = 192;
+constexpr int TC_TMEM_COLS = 512;
+constexpr int TC_SFA_COL = 2 * TC_BN;          // 4 columns per stage
+constexpr int TC_SFB_COL = TC_SFA_COL + 4 * TC_STAGES;  // 4 columns per plane
+
+struct TcShared {
+    uint8_t stage[TC_STAGES][TC_STAGE_BYTES];
+    uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once
+    uint64_t full[TC_STAGES], empty[TC_STAGES], acc_full[2], acc_empty[2];
+    uint32_t tmem_base;
+    int32_t abort;
+};
+
+struct TcArgs {
+    const uint8_t* w;          // matrix region of the packed buffer
+    size_t expert_bytes;
+    int K;                     // inputs per weight row
+    int N;                     // weight rows per expert
+    int gate_up_half;          // W1: I (gate/up interleave), W2: 0
+    const uint8_t* planes;     // 3 digit planes, [K/32][P_pad][16] each
+    size_t plane_stride;       // bytes per plane
+    int P_pad;
+    const int32_t* offsets;    // [E+1]
+    const int32_t* tile_off;   // [E+1] exclusive scan of tiles per expert
+    int E;
+    double* out;               // [P, N] fp64 accumulators
+    int32_t* flag;
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Bounded wait (about one second; a stage lands in microseconds).  Gives up
+// early when another role has aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > 1000000000ull) return false;
+    }
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > 1000000000ull) return false;
+    return true;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, no swizzle, K-major: 8-row x 16-byte core
+// matrices; lbo = byte distance between the two K-adjacent core matrices of one
+// MMA, sbo = byte distance between 8-row groups.  Bit 46 marks the sm100 format.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    return d;
+}
+
+// Instruction descriptor of kind::mxf4 block-scaled MMA: E2M1 x E2M1, UE8M0
+// scales, fp32 accumulate, both operands K-major, M = 128, K = 64.
+__device__ __forceinline__ uint32_t make_idesc(int n, int a_sf_id, int b_sf_id) {
+    uint32_t d = 0;
+    d |= (uint32_t)(b_sf_id & 3) << 4;
+    d |= 1u << 7;                          // A format: E2M1
+    d |= 1u << 10;                         // B format: E2M1
+    d |= (uint32_t)(n >> 3) << 17;         // N / 8
+    d |= 1u << 23;                         // scale format UE8M0
+    d |= (uint32_t)(TC_BM >> 4) << 24;     // M / 16
+    d |= (uint32_t)(a_sf_id & 3) << 29;
+    return d;
+}
+
+struct TcTile {
+    int e, rb, i0, n_valid, n_mma;
+};
+
+__device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
+    int lo = 0, hi = a.E;  // last e with tile_off[e] <= t
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(a.tile_off + mid) <= t) lo = mid; else hi = mid;
+    }
+    TcTile tt;
+    tt.e = lo;
+    const int RB = a.N / TC_BM;
+    const int local = t - __ldg(a.tile_off + lo);
+    const int nb = local / RB;
+    tt.rb = local % RB;
+    const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
+    tt.i0 = r0 + nb * TC_BN;
+    tt.n_valid = min(TC_BN, r1 - tt.i0);
+    tt.n_mma = (tt.n_valid + 15) & ~15;
+    return tt;
+}
+
+__device__ __forceinline__ int canonical_row_tc(int d, int gate_up_half) {
+    if (gate_up_half <= 0) return d;
+    const int rb = d >> 7, r = d & 127;
+    return (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
+    extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
+    TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KG = a.K / 128;
+    const int total = __ldg(a.tile_off + a.E);
+    if (*(volatile int32_t*)a.flag & FLAG_LAYOUT) return;
+    if (total == 0) return;
+
+    // ---- set-up: barriers, constant plane scales, TMEM ----
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(smem_u32(&sh.full[s]), 1);
+            mbar_init(smem_u32(&sh.empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&sh.acc_full[b]), 1);
+            mbar_init(smem_u32(&sh.acc_empty[b]), 4);
+        }
+        sh.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    for (int i = threadIdx.x; i < 3 * 512; i += TC_THREADS)
+        sh.sfb[i / 512][i % 512] = (uint8_t)(133 - 3 * (i / 512));  // 2^6, 2^3, 2^0
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sh.tmem_base)),
+                     "r"(TC_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int32_t* abort = &sh.abort;
+    auto give_up = [&]() {
+        *abort = 1;
+        raise_flag(a.flag, FLAG_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        int stage = 0;
+        uint32_t phase = 0;
+        bool filled[TC_STAGES] = {};
+        uint32_t fill_parity[TC_STAGES] = {};
+        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+            const TcTile tt = tile_at(a, t);
+            const uint8_t* wsrc = a.w + (size_t)tt.e * a.expert_bytes + (size_t)tt.rb * KG * TC_A_BYTES;
+            const uint32_t bbytes = 16u * (uint32_t)tt.n_mma;  // one 32-input chunk of one plane
+            for (int g = 0; g < KG; ++g) {
+                const uint32_t fb = smem_u32(&sh.full[stage]), eb = smem_u32(&sh.empty[stage]);
+                if (!mbar_wait(eb, phase ^ 1u, abort)) {
+                    give_up();
+                    break;
+                }
+                const uint32_t sbase = smem_u32(sh.stage[stage]);
+                if (lane == 0) mbar_expect_tx(fb, TC_A_BYTES + 12u * bbytes);
+                __syncwarp();
+                if (lane == 0) {
+                    bulk_g2s(sbase, wsrc + (size_t)g * TC_A_BYTES, TC_A_BYTES, fb);
+                } else if (lane <= 12) {
+                    const int p = (lane - 1) >> 2, cc = (lane - 1) & 3;
+                    const uint8_t* src = a.planes + (size_t)p * a.plane_stride +
+                                         ((size_t)(4 * g + cc) * a.P_pad + tt.i0) * 16;
+                    bulk_g2s(sbase + TC_A_BYTES + p * TC_B_PLANE_BYTES + cc * bbytes, src, bbytes, fb);
+                }
+                __syncwarp();
+                filled[stage] = true;
+                fill_parity[stage] = phase;
+                if (++stage == TC_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // let every copy this warp issued land before the CTA can exit (on the
+        // normal path the MMA warp has already waited for all of them)
+        for (int s = 0; s < TC_STAGES; ++s)
+            if (filled[s]) mbar_wait_bounded(smem_u32(&sh.full[s]), fill_parity[s]);
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            for (int p = 0; p < 3; ++p)
+                tc_cp_sf(tmem + TC_SFB_COL + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
+        }
+        __syncwarp();
+        int stage = 0;
+        uint32_t phase = 0;
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+            const TcTile tt = tile_at(a, t);
+            if (!mbar_wait(smem_u32(&sh.acc_empty[buf]), acc_phase ^ 1u, abort)) {
+                give_up();
+                break;
+            }
+            tc_fence_after();
+            const uint32_t dcol = tmem + buf * TC_BN;
+            const uint32_t bbytes = 16u * (uint32_t)tt.n_mma;
+            bool ok = true;
+            for (int g = 0; g < KG; ++g) {
+                if (!mbar_wait(smem_u32(&sh.full[stage]), phase, abort)) {
+                    give_up();
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t sbase = smem_u32(sh.stage[stage]);
+                    const uint32_t sfa = tmem + TC_SFA_COL + 4 * stage;
+                    tc_cp_sf(sfa, make_sdesc(sbase, 0, 128));
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const uint64_t adesc = make_sdesc(sbase + 512 + ks * 2 * 2048, 2048, 128);
+#pragma unroll
+                        for (int p = 0; p < 3; ++p) {
+                            const uint64_t bdesc = make_sdesc(
+                                sbase + TC_A_BYTES + p * TC_B_PLANE_BYTES + ks * 2 * bbytes, bbytes, 128);
+                            const uint32_t idesc = make_idesc(tt.n_mma, 2 * ks, 0);
+                            tc_mma_mxf4(dcol, adesc, bdesc, idesc, sfa,
+                                        tmem + TC_SFB_COL + 4 * p, (g | ks | p) != 0);
+                        }
+                    }
+                    tc_commit(smem_u32(&sh.empty[stage]));
+                }
+                __syncwarp();
+                if (++stage == TC_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) tc_commit(smem_u32(&sh.acc_full[buf]));
+            __syncwarp();
+            if (++buf == 2) {
+                buf = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;            // TMEM lane quadrant this warp may access
+        const int m = q * 32 + lane;       // weight row within the tile
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+            const TcTile tt = tile_at(a, t);
+            if (!mbar_wait(smem_u32(&sh.acc_full[buf]), acc_phase, abort)) {
+                give_up();
+                break;
+            }
+            tc_fence_after();
+            const int crow = canonical_row_tc(tt.rb * TC_BM + m, a.gate_up_half);
+            double* out = a.out + (size_t)tt.i0 * a.N + crow;
+            for (int n0 = 0; n0 < tt.n_mma; n0 += 32) {
+                uint32_t r[32];
+                tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * TC_BN + n0, r);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (n0 + j < tt.n_valid) out[(size_t)(n0 + j) * a.N] = (double)__uint_as_float(r[j]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[buf]));
+            if (++buf == 2) {
+                buf = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
+                     : "memory");
+}
+
+// Writes the three E2M1 digit planes of INT8 rows in chunk-major order:
+// plane p, input chunk c (32 inputs), row i -> 16 bytes at
+// planes + p*plane_stride + (c*P_pad + i)*16; element 2j of the chunk in the
+// low nibble of byte j.  Source row of sorted row i: perm[i] / k_div (k_div > 0)
+// or i.  One thread per (row, chunk).
+__global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm,
+                         int k_div, int rows, int P_pad, uint8_t* __restrict__ planes,
+                         size_t plane_stride) {
+    const int nc = K / 32;
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= (long long)rows * nc) return;
+    const int i = (int)(id / nc), c = (int)(id % nc);
+    const int srow = k_div > 0 ? __ldg(perm + i) / k_div : i;
+    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
+    const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    // E2M1 code of a digit d in [-4, 3]
+    auto code = [](int d) -> uint32_t {
+        const uint32_t mag[5] = {0u, 2u, 4u, 5u, 6u};  // 0, 1.0, 2.0, 3.0, 4.0
+        return d < 0 ? (8u | mag[-d]) : mag[d];
+    };
+    uint32_t out[3][4] = {};
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int qv = (int)(int8_t)(w[e >> 2] >> (8 * (e & 3)));
+        const int c0 = ((qv + 4) & 7) - 4;          // least significant digit
+        const int q1 = (qv - c0) >> 3;
+        const int b0 = ((q1 + 4) & 7) - 4;
+        const int a0 = (q1 - b0) >> 3;              // in [-2, 2]
+        const int d[3] = {a0, b0, c0};
+#pragma unroll
+        for (int p = 0; p < 3; ++p) out[p][e >> 3] |= code(d[p]) << (4 * (e & 7));
+    }
+#pragma unroll
+    for (int p = 0; p < 3; ++p)
+        *reinterpret_cast<uint4*>(planes + (size_t)p * plane_stride + ((size_t)c * P_pad + i) * 16) =
+            make_uint4(out[p][0], out[p][1], out[p][2], out[p][3]);
+}
+
+static int tc_grid() {
+    static int grid = 0;
+    if (!grid) {
+        int dev = 0, sms = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaFuncSetAttribute(k_tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
+        grid = sms;
+    }
+    return grid;
+}
+
+size_t tc_smem_bytes() { return sizeof(TcShared); }
+
+cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
+                          int P_pad, uint8_t* planes, size_t plane_stride, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    const long long n = (long long)rows * (K / 32);
+    k_planes<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, K, perm, k_div, rows, P_pad, planes,
+                                                          plane_stride);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
+                           const uint8_t* planes, size_t plane_stride, int P_pad,
+                           const int32_t* offsets, const int32_t* tile_off, int E, double* out,
+                           int32_t* flag, cudaStream_t st) {
+    TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_stride, P_pad, offsets, tile_off, E, out, flag};
+    k_tc_gemm<<<tc_grid(), TC_THREADS, sizeof(TcShared), st>>>(a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

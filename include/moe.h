@@ -192,6 +192,17 @@ int moe_quant_rows_f32(const float *v, int rows, int cols, int8_t *q, float *s,
 int moe_exp_f32(const float *x, float *y, int64_t n, cudaStream_t stream);
 int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStream_t stream);
 
+/* Process-wide tuning options (not thread-safe; set them before launching work).
+ *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
+ *   run on the tensor-core grouped GEMM (tcgen05, tiles of 128 weight rows x
+ *   128 token rows); experts with fewer rows run on the CUDA-core streaming
+ *   GEMM.  Default 32; must be >= 1.  Both paths give the same results.
+ * moe_set_option returns MOE_OK or MOE_ERR_INVALID_ARG; moe_get_option returns
+ * the current value (-1 for an unknown option). */
+#define MOE_OPT_TC_MIN_ROWS 1
+int moe_set_option(int option, int value);
+int moe_get_option(int option);
+
 /* Number of CUDA kernels this library has launched in the calling process
  * (a diagnostic counter; memsets and event records are not counted). */
 unsigned long long moe_launch_count(void);

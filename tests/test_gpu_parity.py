@@ -355,3 +355,43 @@ def test_swiglu_bit_identical_to_oracle(moe):
     ref = np.array([oracle.swiglu(float(a), float(b)) for a, b in zip(g[:20000], u[:20000])],
                    np.float32)
     assert np.array_equal(h[:20000].view(np.uint32), ref.view(np.uint32))
+
+
+# ---- the tensor-core grouped GEMM, forced on for every expert ------------------
+
+@pytest.fixture
+def tc_everywhere(moe):
+    old = moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS)
+    moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
+    yield
+    moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, old)
+
+
+@pytest.mark.parametrize("T,H,E,k,I,seed", [
+    (40, 256, 2, 1, 128, 51),      # one n-block per expert, ragged (19/21 rows)
+    (300, 512, 4, 2, 256, 52),     # several n-blocks per expert, ragged tails
+    (13, 384, 9, 3, 256, 42),      # tiny experts: n_mma = 16
+    (9, 256, 16, 16, 128, 43),     # k = E
+    (257, 128, 1, 1, 128, 53),     # E = 1, 257 rows: three n-blocks, last holds one row
+])
+def test_tc_forward_parity_shapes(moe, tc_everywhere, T, H, E, k, I, seed):
+    w = synth.custom("tc", T, H, E, k, I, seed)
+    d = synth.make(w)
+    o = oracle.forward(d["x"], d["logits"], d["w1_codes"], d["w1_scales"], d["w2_codes"],
+                       d["w2_scales"], k)
+    _check_layer(moe, d, w, o)
+
+
+def test_tc_forward_parity_decode_T64(moe, workload_data, tc_everywhere):
+    # decode-shaped experts (1-7 rows) through the tensor-core path
+    name = "decode_T64"
+    d, w = workload_data(name), synth.WORKLOADS[name]
+    _check_layer(moe, d, w, oracle_full(name, d))
+
+
+def test_tc_option_validation(moe):
+    with pytest.raises(moe.MoeError):
+        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 0)
+    with pytest.raises(moe.MoeError):
+        moe.moe_set_option(99, 1)
+    assert moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS) >= 1
