@@ -23,7 +23,7 @@ FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_LAYOUT, FLAG_TIMEOUT, FLAG_BOUNDS = 1, 2, 
 
 # Exported symbols of include/moe.h, in declaration order.
 SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack_weights",
-           "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_workspace_bytes",
+           "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_sort_static", "moe_workspace_bytes",
            "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
            "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
 
@@ -58,6 +58,7 @@ def _load():
         "moe_route": ([vp, i32, i32, i32, vp, vp, vp], i32),
         "moe_sort_workspace_bytes": ([i32, i32, i32], sz),
         "moe_sort": ([vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
+        "moe_sort_static": ([vp, i32, i32, i32, vp, vp, vp, vp], i32),
         "moe_workspace_bytes": ([D, i32], sz),
         "moe_forward": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
         "moe_layer_workspace_bytes": ([D, i32], sz),
@@ -185,6 +186,21 @@ def moe_sort(topk_idx, E: int, ws=None, out=None, stream=None):
     perm, pos, offsets = out
     _check(lib.moe_sort(_ptr(topk_idx), T, k, E, _ptr(perm), _ptr(pos), _ptr(offsets), _ptr(ws),
                         ws.numel(), _stream(stream)))
+    return perm, pos, offsets
+
+
+def moe_sort_static(topk_idx, E: int, out=None, stream=None):
+    """moe_sort using the library's own fixed scratch (no workspace argument);
+    T*k <= 65536 and E <= 1024."""
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if out is None:
+        out = (torch.empty(T * k, dtype=torch.int32, device=dev),
+               torch.empty(T * k, dtype=torch.int32, device=dev),
+               torch.empty(E + 1, dtype=torch.int32, device=dev))
+    perm, pos, offsets = out
+    _check(lib.moe_sort_static(_ptr(topk_idx), T, k, E, _ptr(perm), _ptr(pos), _ptr(offsets),
+                               _stream(stream)))
     return perm, pos, offsets
 
 

@@ -174,6 +174,23 @@ int moe_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort launch");
 }
 
+int moe_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
+                    int32_t* offsets, cudaStream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_sort_static: T < 0");
+    if (E < 1 || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_sort_static: E must be in [1, 1024]");
+    if (k < 1 || k > 16 || k > E)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_sort_static: k must be in [1, min(E,16)]");
+    if (!moe::sort_static_fits(T, k, E))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                    "moe_sort_static: T*k = %lld exceeds the static scratch limit of 65536 pairs "
+                    "(use moe_sort with a caller workspace)", (long long)T * k);
+    if (!offsets || (T > 0 && (!topk_idx || !perm || !pos)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_sort_static: NULL pointer");
+    cudaError_t e = moe::launch_sort_static(topk_idx, T, k, E, perm, pos, offsets, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_sort_static");
+}
+
 size_t moe_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
     return ws_layout(*d, T_max).total;

@@ -23,6 +23,10 @@ size_t sort_workspace_bytes(int T_max, int k, int E);
 cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
                         int32_t* offsets, void* ws, cudaStream_t st);
 
+int sort_static_fits(int T, int k, int E);
+cudaError_t launch_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* perm,
+                               int32_t* pos, int32_t* offsets, cudaStream_t st);
+
 cudaError_t launch_pack(int H, int I, int E, const uint8_t* w1c, const uint8_t* w1s,
                         const uint8_t* w2c, const uint8_t* w2s, void* packed, bool forward,
                         uint8_t* out_w1c, uint8_t* out_w1s, uint8_t* out_w2c, uint8_t* out_w2s,

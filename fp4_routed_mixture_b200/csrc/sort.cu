@@ -12,6 +12,8 @@
 //                  step, which keeps the sort stable.
 // A single chunk (P <= 1024, the decode case) runs both phases in one launch.
 // Expert ids outside [0, E) raise FLAG_BAD_EXPERT and are skipped.
+#include <mutex>
+
 #include "kernels.cuh"
 #include "moe_common.cuh"
 
@@ -193,6 +195,55 @@ cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* p
                                                        offsets);
     count_launches(1);
     return cudaGetLastError();
+}
+
+// ---- the same sort with library-owned scratch (moe_sort_static) -------------
+// For callers that are handed only input and output pointers and have no way
+// to obtain a device workspace: the scratch (error word + per-chunk
+// histograms) lives in this file-scope device array.  Every GPU that loads the
+// library holds it until the process exits; every call shares it, so calls
+// that overlap on a GPU race.  It keeps the previous call's contents: the
+// error word is cleared by every call and every histogram entry a call reads
+// is written by that same call first.
+constexpr int kSortStaticMaxPairs = 65536;
+constexpr int kSortStaticMaxExperts = 1024;
+constexpr size_t kSortStaticBytes =
+    256 + (size_t)(kSortStaticMaxPairs / kSortChunk) * kSortStaticMaxExperts * sizeof(int32_t);
+static __device__ __align__(256) uint8_t g_sort_scratch[kSortStaticBytes];
+
+static_assert(kSortStaticMaxPairs % kSortChunk == 0, "whole chunks");
+
+// Device address of g_sort_scratch on the current device, looked up once per
+// device (the host-side name is only a stand-in for it).
+static cudaError_t sort_static_scratch(void** out) {
+    constexpr int kMaxDevices = 64;
+    static void* ptrs[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_sort_scratch);
+        if (e != cudaSuccess) return e;
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return cudaSuccess;
+}
+
+int sort_static_fits(int T, int k, int E) {
+    return (long long)T * k <= kSortStaticMaxPairs && E <= kSortStaticMaxExperts;
+}
+
+cudaError_t launch_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* perm,
+                               int32_t* pos, int32_t* offsets, cudaStream_t st) {
+    void* ws = nullptr;
+    cudaError_t e = sort_static_scratch(&ws);
+    if (e != cudaSuccess) return e;
+    return launch_sort(topk_idx, T, k, E, perm, pos, offsets, ws, st);
 }
 
 }  // namespace moe

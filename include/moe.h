@@ -142,6 +142,25 @@ size_t moe_sort_workspace_bytes(int T_max, int k, int E);
 int moe_sort(const int32_t *topk_idx, int T, int k, int E, int32_t *perm, int32_t *pos,
              int32_t *offsets, void *ws, size_t ws_bytes, cudaStream_t stream);
 
+/* moe_sort without a workspace argument.  The paper has no counterpart: this
+ * entry point exists for callers that are handed only input and output
+ * buffers -- for example code embedded in a host framework that owns all
+ * device memory and offers no way to request a scratch buffer -- and so cannot
+ * call cudaMalloc or size a workspace themselves.  Same arguments (minus ws)
+ * and same results as moe_sort; nothing is allocated.
+ *   - Scratch is a fixed 256 KB array inside the library (held on every GPU
+ *     that loads it, until process exit): T*k <= 65536 pairs and E <= 1024;
+ *     larger calls return MOE_ERR_UNSUPPORTED_SHAPE (use moe_sort).
+ *   - The first call on a device looks up that array's device address for the
+ *     current device (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - All calls share the array: calls that overlap on a GPU race.  Each call
+ *     clears and rewrites what it reads.
+ *   - Expert ids outside [0, E) are skipped as in moe_sort; the error word is
+ *     internal to this variant (use moe_sort to observe it). */
+int moe_sort_static(const int32_t *topk_idx, int T, int k, int E, int32_t *perm, int32_t *pos,
+                    int32_t *offsets, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------
  * The expert computation ([A]: INT8 activation quantisation, packed FP4
  * expert GEMMs W1 and W2; routed mixture combine).
