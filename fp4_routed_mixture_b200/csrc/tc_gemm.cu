@@ -401,22 +401,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
 // plane p, input chunk c (32 inputs), row i -> 16 bytes at
 // planes + p*plane_stride + (c*P_pad + i)*16; element 2j of the chunk in the
 // low nibble of byte j.  Source row of sorted row i: perm[i] / k_div (k_div > 0)
-// or i.  One thread per (row, chunk).
+// or i.  One thread per (row, chunk), rows fastest: consecutive threads write
+// consecutive 16-byte pieces of a plane.
 __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm,
                          int k_div, int rows, int P_pad, uint8_t* __restrict__ planes,
                          size_t plane_stride) {
     const int nc = K / 32;
     const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (id >= (long long)rows * nc) return;
-    const int i = (int)(id / nc), c = (int)(id % nc);
+    const int i = (int)(id % rows), c = (int)(id / rows);
     const int srow = k_div > 0 ? __ldg(perm + i) / k_div : i;
     const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
     const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    // E2M1 code of a digit d in [-4, 3]
+    // E2M1 code of a digit d in [-4, 3]: magnitudes 0, 1, 2, 3, 4 are the codes
+    // 0, 2, 4, 5, 6 (nibbles packed in 0x65420), the sign is bit 3
     auto code = [](int d) -> uint32_t {
-        const uint32_t mag[5] = {0u, 2u, 4u, 5u, 6u};  // 0, 1.0, 2.0, 3.0, 4.0
-        return d < 0 ? (8u | mag[-d]) : mag[d];
+        const uint32_t mag = (0x65420u >> (4 * (d < 0 ? -d : d))) & 0xFu;
+        return d < 0 ? (8u | mag) : mag;
     };
     uint32_t out[3][4] = {};
 #pragma unroll
@@ -426,9 +428,9 @@ __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* _
         const int q1 = (qv - c0) >> 3;
         const int b0 = ((q1 + 4) & 7) - 4;
         const int a0 = (q1 - b0) >> 3;              // in [-2, 2]
-        const int d[3] = {a0, b0, c0};
-#pragma unroll
-        for (int p = 0; p < 3; ++p) out[p][e >> 3] |= code(d[p]) << (4 * (e & 7));
+        out[0][e >> 3] |= code(a0) << (4 * (e & 7));
+        out[1][e >> 3] |= code(b0) << (4 * (e & 7));
+        out[2][e >> 3] |= code(c0) << (4 * (e & 7));
     }
 #pragma unroll
     for (int p = 0; p < 3; ++p)
