@@ -121,14 +121,15 @@ struct GemvArgs {
     double* out;               // [P, N] fp64 accumulators, zeroed
     const int32_t* flag;       // device error word: a layout mismatch stops the kernel
     int gate_up_half;          // > 0 (= I) for W1: device rows interleave gate and up rows
+    int P;                     // pairs (rows of the sorted tables)
     uint32_t zero;             // always 0 (see Tables)
 };
 
 // Canonical row (output column) of a device row (see the layout in pack.cu).
 __device__ __forceinline__ int canonical_row(int d, int gate_up_half) {
     if (gate_up_half <= 0) return d;
-    const int rb = d >> 7, r = d & 127;
-    return (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
+    const int tau = d >> 5, r = d & 31;
+    return (r < 16) ? tau * 16 + r : gate_up_half + tau * 16 + (r - 16);
 }
 
 // A unit: expert, tile, first sorted row, number of rows.
@@ -155,7 +156,7 @@ __device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
 }
 
 __device__ __forceinline__ int act_row(const GemvArgs& a, int i) {
-    return a.k_div ? __ldg(a.perm + i) / a.k_div : i;
+    return a.k_div ? checked_index(__ldg(a.perm + i), a.P, const_cast<int32_t*>(a.flag)) / a.k_div : i;
 }
 
 // Integer dot product of one 32-element block (8 decoded words) with one
@@ -331,16 +332,23 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
 // tensor-core GEMM (tiles of 128 weight rows x 128 token rows), the others to
 // the streaming GEMM (units of 32 weight rows x kGroup tokens).  Writes the
 // exclusive scans over experts of the streaming units of W1/W2 and of the
-// tensor-core tiles of W1/W2.  One warp; lane l owns a contiguous slice of
-// experts.
-__global__ void k_plan(const int32_t* __restrict__ offsets, int E, int n1, int n2, int tc_min,
+// tensor-core tiles of W1/W2, and expert_tc[e] = 1 for tensor-core experts.
+// One warp; lane l owns a contiguous slice of experts.
+__global__ void k_plan(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
                        int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
-                       int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2) {
+                       int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
+                       int32_t* __restrict__ expert_tc, int32_t* flag) {
     const int lane = threadIdx.x;
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    // offsets must run from 0 up to at most P without decreasing; otherwise no
+    // expert gets any work (and FLAG_BOUNDS is raised)
+    bool bad = (lane == 0 && offsets[0] != 0) || (lane == 31 && offsets[E] > P);
+    for (int e = e0; e < e1; ++e) bad |= offsets[e + 1] < offsets[e];
+    const bool any_bad = __any_sync(0xffffffffu, bad);
+    if (any_bad && lane == 0) raise_flag(flag, FLAG_BOUNDS);
     auto counts = [&](int e, int& u1, int& u2, int& t1, int& t2) {
-        const int m = offsets[e + 1] - offsets[e];
+        const int m = any_bad ? 0 : offsets[e + 1] - offsets[e];
         const bool tc = m >= tc_min;
         const int g = tc ? 0 : (m + kGroup - 1) / kGroup;
         const int nb = tc ? (m + 127) / 128 : 0;
@@ -374,6 +382,7 @@ __global__ void k_plan(const int32_t* __restrict__ offsets, int E, int n1, int n
             outs[j][e] = r[j];
             r[j] += c[j];
         }
+        expert_tc[e] = (!any_bad && (offsets[e + 1] - offsets[e]) >= tc_min) ? 1 : 0;
     }
     if (lane == 31)
         for (int j = 0; j < 4; ++j) outs[j][E] = x[j];
@@ -392,9 +401,11 @@ static int gemv_grid() {
     return grid;
 }
 
-cudaError_t launch_plan(const int32_t* offsets, int E, int n1, int n2, int tc_min, int32_t* unit_off1,
-                        int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, cudaStream_t st) {
-    k_plan<<<1, 32, 0, st>>>(offsets, E, n1, n2, tc_min, unit_off1, unit_off2, tile_off1, tile_off2);
+cudaError_t launch_plan(const int32_t* offsets, int E, int P, int n1, int n2, int tc_min,
+                        int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2,
+                        int32_t* expert_tc, int32_t* flag, cudaStream_t st) {
+    k_plan<<<1, 32, 0, st>>>(offsets, E, P, n1, n2, tc_min, unit_off1, unit_off2, tile_off1, tile_off2,
+                             expert_tc, flag);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -402,9 +413,9 @@ cudaError_t launch_plan(const int32_t* offsets, int E, int n1, int n2, int tc_mi
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, cudaStream_t st) {
+                        const int32_t* flag, int gate_up_half, int P, cudaStream_t st) {
     GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
-               gate_up_half, 0u};
+               gate_up_half, P, 0u};
     k_gemv<<<gemv_grid(), kGemvWarps * 32, kSmemBytes, st>>>(a);
     count_launches(1);
     return cudaGetLastError();

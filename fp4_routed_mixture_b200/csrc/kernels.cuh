@@ -37,30 +37,38 @@ cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
                           int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
-cudaError_t launch_swiglu_hquant(const double* gacc, const float* sx, const int32_t* perm, int P,
-                                 int k, int I, int8_t* hq, float* sh, int32_t* hinit,
-                                 int8_t* dbg_hq, float* dbg_sh, cudaStream_t st);
+cudaError_t launch_hquant(const double* gacc, const float* hbuf, const uint32_t* amax,
+                          const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
+                          const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
+                          int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st);
+cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
+                                int P, int E, int I, int H, uint32_t* amax, double* gacc, double* yacc,
+                                int32_t* flag, cudaStream_t st);
 cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
 cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
                               cudaStream_t st);
 
-cudaError_t launch_plan(const int32_t* offsets, int E, int n1, int n2, int tc_min, int32_t* unit_off1,
-                        int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, cudaStream_t st);
+cudaError_t launch_plan(const int32_t* offsets, int E, int P, int n1, int n2, int tc_min,
+                        int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2,
+                        int32_t* expert_tc, int32_t* flag, cudaStream_t st);
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, cudaStream_t st);
+                        const int32_t* flag, int gate_up_half, int P, cudaStream_t st);
 
 size_t tc_smem_bytes();
 cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
-                          int P_pad, uint8_t* planes, size_t plane_stride, cudaStream_t st);
+                          int P_pad, uint8_t* planes, size_t plane_stride, int32_t* flag, cudaStream_t st);
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, size_t plane_stride, int P_pad,
-                           const int32_t* offsets, const int32_t* tile_off, int E, double* out,
-                           int32_t* flag, cudaStream_t st);
+                           const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
+                           const float* row_scale, const int32_t* perm, int k_div, float* out,
+                           uint32_t* amax, cudaStream_t st);
 
-cudaError_t launch_combine(const double* yacc, const float* sh, const float* gates,
-                           const int32_t* pos, int T, int k, int H, void* y, cudaStream_t st);
+cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
+                           const int32_t* topk_idx, const float* sh, const float* gates,
+                           const int32_t* pos, int T, int k, int E, int H, void* y, int32_t* flag,
+                           cudaStream_t st);
 
 }  // namespace moe

@@ -24,6 +24,15 @@ __device__ __forceinline__ void raise_flag(int32_t* flag, int32_t bit) {
     if (flag) atomicOr(flag, bit);
 }
 
+// An index read from a caller-provided table (perm, pos, topk_idx): values
+// outside [0, n) raise FLAG_BOUNDS and are replaced by 0, so a bad table can
+// give wrong results but never an out-of-bounds access.
+__device__ __forceinline__ int checked_index(int v, int n, int32_t* flag) {
+    if ((unsigned)v < (unsigned)n) return v;
+    raise_flag(flag, FLAG_BOUNDS);
+    return 0;
+}
+
 // ---- The layer's fp32 exp ---------------------------------------------------
 // Specification (the CPU reference implements the same one separately):
 //   NaN -> NaN; x > 88.8 -> +inf; x < -104 -> 0;

@@ -21,9 +21,9 @@
 // 512-byte contiguous slice per block; the tensor-core producer fetches a whole
 // chunk with one bulk copy.
 // Device rows of W2 are its canonical rows.  Device rows of W1 interleave gate
-// and up per 128-row block: device row rb*128 + r is gate row rb*64 + r for
-// r < 64 and up row I + rb*64 + (r - 64) otherwise, so every 128-row block
-// holds the gate and up rows of the same 64 outputs.
+// and up rows per 32-row tile: device row 32*tau + r is gate row 16*tau + r
+// for r < 16 and up row I + 16*tau + (r - 16) otherwise, so every warp-sized
+// group of rows holds the gate and up rows of the same 16 outputs.
 // The layout moves the canonical bytes, so its size equals the canonical size.
 #include "kernels.cuh"
 #include "moe_common.cuh"
@@ -37,7 +37,7 @@ struct PackHeader {
 };
 
 constexpr uint32_t kPackMagic = 0x34454F4Du;  // "MOE4"
-constexpr uint32_t kPackVersion = 2;
+constexpr uint32_t kPackVersion = 3;
 
 __host__ __device__ inline size_t matrix_bytes(int N, int K) { return (size_t)N * K * 17 / 32; }
 
@@ -70,8 +70,8 @@ __global__ void k_pack_matrix(uint8_t* __restrict__ dev, uint8_t* __restrict__ c
         const int e = (int)(rd / N);
         int crow = drow;  // canonical row of this device row
         if (gate_up_half > 0) {
-            const int rb = drow >> 7, r = drow & 127;
-            crow = (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
+            const int tau = drow >> 5, r = drow & 31;
+            crow = (r < 16) ? tau * 16 + r : gate_up_half + tau * 16 + (r - 16);
         }
         const size_t rn = (size_t)e * N + crow;
         uint8_t* d = dev + (size_t)e * mbytes;

@@ -2,7 +2,9 @@
 // INT8 activations feeding the packed-FP4 expert GEMMs).
 //
 //   k_xquant        x [T,H] bf16 -> xq [T,H] int8, sx [T], xinit [T,H/32]
-//   k_swiglu_hquant G accumulators (fp64, sorted rows) -> SwiGLU -> hq, sh, hinit
+//   k_hquant        h of every sorted row (SwiGLU of the streaming GEMM's fp64
+//                   sums, or h from the tensor-core epilogue) -> hq, sh, hinit
+//   k_prepare_rows  clears per-row state before the W1/W2 GEMMs
 //   k_quant_rows    fp32 rows -> int8 + scale (stage entry point)
 //
 // Rule for every row: a = max|v| (exact), s = fp32(a/127) by IEEE division,
@@ -85,28 +87,42 @@ __global__ void __launch_bounds__(kQThreads)
     }
 }
 
-// One CTA per sorted row i.  G values are the exact fp64 sums of the W1
-// product; the fp32 G of the definition is fp32(fp64(sx[t]) * sum).
+// One CTA per sorted row i: the row's h values and |h| maximum, then its INT8
+// codes.  Rows of experts on the streaming GEMM arrive as exact fp64 sums of
+// the W1 product (gate and up): G = fp32(fp64(sx[t]) * sum), h = SwiGLU(g, u)
+// here.  Rows of experts on the tensor-core GEMM arrive as h itself plus the
+// bits of max |h| (formed in that GEMM's epilogue).
 __global__ void __launch_bounds__(kQThreads)
-    k_swiglu_hquant(const double* __restrict__ gacc, const float* __restrict__ sx,
-                    const int32_t* __restrict__ perm, int k, int I, int8_t* __restrict__ hq,
-                    float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
-                    float* __restrict__ dbg_sh) {
+    k_hquant(const double* __restrict__ gacc, const float* __restrict__ hbuf,
+             const uint32_t* __restrict__ amax_bits, const int32_t* __restrict__ expert_tc,
+             const int32_t* __restrict__ topk_idx, const float* __restrict__ sx,
+             const int32_t* __restrict__ perm, int P, int k, int E, int I, int8_t* __restrict__ hq,
+             float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
+             float* __restrict__ dbg_sh, int32_t* flag) {
     extern __shared__ float h[];  // [I]
     __shared__ float red[33];
     const int i = blockIdx.x;
-    const int t = perm[i] / k;
-    const double s = (double)sx[t];
-    const double* g = gacc + (size_t)i * 2 * I;
-    float a = 0.0f;
-    for (int j = threadIdx.x; j < I; j += blockDim.x) {
-        const float gv = (float)__dmul_rn(s, g[j]);
-        const float uv = (float)__dmul_rn(s, g[I + j]);
-        const float hv = swiglu(gv, uv);
-        h[j] = hv;
-        a = fmaxf(a, fabsf(hv));
+    const int p = checked_index(perm[i], P, flag);
+    const bool tc = expert_tc[checked_index(topk_idx[p], E, flag)] != 0;
+    float a;
+    if (tc) {
+        const float* hr = hbuf + (size_t)i * I;
+        for (int j = threadIdx.x; j < I; j += blockDim.x) h[j] = hr[j];
+        a = __uint_as_float(amax_bits[i]);
+        __syncthreads();
+    } else {
+        const double s = (double)sx[p / k];
+        const double* g = gacc + (size_t)i * 2 * I;
+        a = 0.0f;
+        for (int j = threadIdx.x; j < I; j += blockDim.x) {
+            const float gv = (float)__dmul_rn(s, g[j]);
+            const float uv = (float)__dmul_rn(s, g[I + j]);
+            const float hv = swiglu(gv, uv);
+            h[j] = hv;
+            a = fmaxf(a, fabsf(hv));
+        }
+        a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
     }
-    a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
     const float sc = quant_scale(a);
     if (threadIdx.x == 0) {
         sh[i] = sc;
@@ -131,6 +147,23 @@ __global__ void __launch_bounds__(kQThreads)
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 4);
         if (j < I && (j & 31) == 0) hinit[(size_t)i * (I / 32) + (j >> 5)] = -12 * bsum;
+    }
+}
+
+// Per sorted row: clears the row's |h| maximum and, for rows of experts on
+// the streaming GEMM, its fp64 accumulators (that GEMM adds partial sums into
+// them).  Rows of tensor-core experts are written whole by that GEMM.
+__global__ void __launch_bounds__(256)
+    k_prepare_rows(const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
+                   const int32_t* __restrict__ perm, int P, int E, int I, int H, uint32_t* __restrict__ amax,
+                   double* __restrict__ gacc, double* __restrict__ yacc, int32_t* flag) {
+    for (int i = blockIdx.x; i < P; i += gridDim.x) {
+        if (threadIdx.x == 0) amax[i] = 0u;
+        if (expert_tc[checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag)]) continue;
+        double2* g = reinterpret_cast<double2*>(gacc + (size_t)i * 2 * I);
+        for (int j = threadIdx.x; j < I; j += blockDim.x) g[j] = make_double2(0.0, 0.0);
+        double2* y = reinterpret_cast<double2*>(yacc + (size_t)i * H);
+        for (int j = threadIdx.x; j < H / 2; j += blockDim.x) y[j] = make_double2(0.0, 0.0);
     }
 }
 
@@ -185,12 +218,24 @@ cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_swiglu_hquant(const double* gacc, const float* sx, const int32_t* perm, int P,
-                                 int k, int I, int8_t* hq, float* sh, int32_t* hinit,
-                                 int8_t* dbg_hq, float* dbg_sh, cudaStream_t st) {
+cudaError_t launch_hquant(const double* gacc, const float* hbuf, const uint32_t* amax,
+                          const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
+                          const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
+                          int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
-    k_swiglu_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, sx, perm, k, I, hq, sh,
-                                                                      hinit, dbg_hq, dbg_sh);
+    k_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, hbuf, amax, expert_tc, topk_idx, sx,
+                                                               perm, P, k, E, I, hq, sh, hinit, dbg_hq,
+                                                               dbg_sh, flag);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
+                                int P, int E, int I, int H, uint32_t* amax, double* gacc, double* yacc,
+                                int32_t* flag, cudaStream_t st) {
+    if (P == 0) return cudaSuccess;
+    k_prepare_rows<<<std::min(P, 148 * 8), 256, 0, st>>>(expert_tc, topk_idx, perm, P, E, I, H, amax,
+                                                          gacc, yacc, flag);
     count_launches(1);
     return cudaGetLastError();
 }

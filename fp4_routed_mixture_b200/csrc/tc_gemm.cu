@@ -26,9 +26,11 @@
 //               6-stage ring (mbarrier transaction counts);
 //   warp 1      MMA issuer: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs per
 //               stage, tcgen05.commit frees the stage / publishes the tile;
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld) -> fp64 accumulators
-//               in global memory, one thread per weight row; two accumulator
-//               buffers in TMEM let the epilogue overlap the next tile's MMAs.
+//   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld), one thread per
+//               weight row and half of the columns; W1 applies the token scale and SwiGLU (gate and up
+//               rows share a warp) and writes h plus the row maxima of |h|, W2
+//               writes the final fp32 Y; two accumulator buffers in TMEM let
+//               the epilogue overlap the next tile's MMAs.
 // Every wait is bounded in time; a wait that gives up raises FLAG_TIMEOUT and
 // the roles wind down (copies in flight are waited for, TMEM is freed).
 #include "kernels.cuh"
@@ -42,7 +44,8 @@ constexpr int TC_STAGES = 6;
 constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
 constexpr int TC_B_PLANE_BYTES = TC_BN * 64;   // 128 rows x 128 inputs, 4 bits each
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + 3 * TC_B_PLANE_BYTES;
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 8;                // two per TMEM lane quadrant
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SFA_COL = 2 * TC_BN;          // 4 columns per stage
 constexpr int TC_SFB_COL = TC_SFA_COL + 4 * TC_STAGES;  // 4 columns per plane
@@ -50,6 +53,7 @@ constexpr int TC_SFB_COL = TC_SFA_COL + 4 * TC_STAGES;  // 4 columns per plane
 struct TcShared {
     uint8_t stage[TC_STAGES][TC_STAGE_BYTES];
     uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once
+    float col_scale[TC_EPI_WARPS][TC_BN];  // per epilogue warp: activation scale of each tile column
     uint64_t full[TC_STAGES], empty[TC_STAGES], acc_full[2], acc_empty[2];
     uint32_t tmem_base;
     int32_t abort;
@@ -64,11 +68,17 @@ struct TcArgs {
     const uint8_t* planes;     // 3 digit planes, [K/32][P_pad][16] each
     size_t plane_stride;       // bytes per plane
     int P_pad;
+    int P;                     // sorted rows (pairs)
     const int32_t* offsets;    // [E+1]
     const int32_t* tile_off;   // [E+1] exclusive scan of tiles per expert
     int E;
-    double* out;               // [P, N] fp64 accumulators
     int32_t* flag;
+    // epilogue
+    const float* row_scale;    // activation scale per source row (W1: sx per token, W2: sh per sorted row)
+    const int32_t* perm;       // sorted row -> pair id (W1: source row = perm[i] / k_div)
+    int k_div;                 // W1: k; W2: 0 (source row = sorted row)
+    float* out;                // W1: h [P, I]; W2: Y [P, H]  (fp32, final values)
+    uint32_t* amax;            // W1: per sorted row, bits of max |h| (atomicMax); W2: unused
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -209,12 +219,6 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     return tt;
 }
 
-__device__ __forceinline__ int canonical_row_tc(int d, int gate_up_half) {
-    if (gate_up_half <= 0) return d;
-    const int rb = d >> 7, r = d & 127;
-    return (r < 64) ? rb * 64 + r : gate_up_half + rb * 64 + (r - 64);
-}
-
 __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sh.acc_full[b]), 1);
-            mbar_init(smem_u32(&sh.acc_empty[b]), 4);
+            mbar_init(smem_u32(&sh.acc_empty[b]), TC_EPI_WARPS);
         }
         sh.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -358,26 +362,71 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
+        // Two warps per TMEM lane quadrant; warp half h takes the 32-column
+        // chunks h, h+2, ... of the tile.  Each warp first stages the
+        // activation scale of every tile column in its own shared-memory slice
+        // (no cross-warp waits).  Scaling: the accumulator is an fp32 value,
+        // so fp32(fp64(s) * fp64(acc)) -- the definition -- equals the single
+        // correctly rounded fp32 product s * acc (the exact product of two
+        // 24-bit significands fits in fp64).
+        // W1: lanes 0-15 of a warp hold the gate rows and lanes 16-31 the up
+        // rows of the same 16 outputs (row interleave of pack.cu).  Columns go
+        // in pairs: lanes 0-15 form h for column j (up value shuffled down),
+        // lanes 16-31 for column j+1 (gate value shuffled up), h = SwiGLU(g, u);
+        // h is stored and |h| folded into the row maximum (max over 16 lanes,
+        // then one atomicMax per half-warp and column; max is order-independent).
+        // W2: Y = s * acc straight out.
+        const int ew = warp - 2;
         const int q = warp & 3;            // TMEM lane quadrant this warp may access
+        const int half = ew >> 2;          // which alternate 32-column chunks
         const int m = q * 32 + lane;       // weight row within the tile
+        const bool w1 = a.amax != nullptr;
+        float* csc = sh.col_scale[ew];
         int buf = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
             const TcTile tt = tile_at(a, t);
+            for (int n = lane; n < tt.n_mma; n += 32) {
+                const int i = min(tt.i0 + n, tt.i0 + tt.n_valid - 1);
+                const int src = a.k_div > 0 ? checked_index(__ldg(a.perm + i), a.P, a.flag) / a.k_div : i;
+                csc[n] = __ldg(a.row_scale + src);
+            }
+            __syncwarp();
             if (!mbar_wait(smem_u32(&sh.acc_full[buf]), acc_phase, abort)) {
                 give_up();
                 break;
             }
             tc_fence_after();
-            const int crow = canonical_row_tc(tt.rb * TC_BM + m, a.gate_up_half);
-            double* out = a.out + (size_t)tt.i0 * a.N + crow;
-            for (int n0 = 0; n0 < tt.n_mma; n0 += 32) {
+            for (int n0 = 32 * half; n0 < tt.n_mma; n0 += 64) {
                 uint32_t r[32];
                 tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * TC_BN + n0, r);
+                if (!w1) {
+                    float* out = a.out + (size_t)(tt.i0 + n0) * a.N + tt.rb * TC_BM + m;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (n0 + j < tt.n_valid) out[(size_t)(n0 + j) * a.N] = (double)__uint_as_float(r[j]);
+                    for (int j = 0; j < 32; ++j)
+                        if (n0 + j < tt.n_valid) out[(size_t)j * a.N] = __fmul_rn(csc[n0 + j], __uint_as_float(r[j]));
+                } else {
+                    const int I = a.gate_up_half;
+                    const bool lo = lane < 16;
+                    float* out = a.out + (size_t)(tt.i0 + n0) * I + (tt.rb * 4 + q) * 16 + (lane & 15);
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const float v0 = __fmul_rn(csc[n0 + j], __uint_as_float(r[j]));
+                        const float v1 = __fmul_rn(csc[n0 + j + 1], __uint_as_float(r[j + 1]));
+                        const float from_hi = __shfl_down_sync(0xffffffffu, v0, 16);  // up value, column j
+                        const float from_lo = __shfl_up_sync(0xffffffffu, v1, 16);    // gate value, column j+1
+                        const float hv = lo ? swiglu(v0, from_hi) : swiglu(from_lo, v1);
+                        const int col = n0 + j + (lo ? 0 : 1);
+                        float am = fabsf(hv);
+#pragma unroll
+                        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+                        if (col < tt.n_valid) {
+                            out[(size_t)(j + (lo ? 0 : 1)) * I] = hv;
+                            if ((lane & 15) == 0) atomicMax(a.amax + tt.i0 + col, __float_as_uint(am));
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -405,12 +454,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
 // consecutive 16-byte pieces of a plane.
 __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm,
                          int k_div, int rows, int P_pad, uint8_t* __restrict__ planes,
-                         size_t plane_stride) {
+                         size_t plane_stride, int32_t* flag) {
     const int nc = K / 32;
     const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (id >= (long long)rows * nc) return;
     const int i = (int)(id % rows), c = (int)(id / rows);
-    const int srow = k_div > 0 ? __ldg(perm + i) / k_div : i;
+    const int srow = k_div > 0 ? checked_index(__ldg(perm + i), rows, flag) / k_div : i;
     const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
     const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -453,20 +502,22 @@ static int tc_grid() {
 size_t tc_smem_bytes() { return sizeof(TcShared); }
 
 cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
-                          int P_pad, uint8_t* planes, size_t plane_stride, cudaStream_t st) {
+                          int P_pad, uint8_t* planes, size_t plane_stride, int32_t* flag, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
     const long long n = (long long)rows * (K / 32);
     k_planes<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, K, perm, k_div, rows, P_pad, planes,
-                                                          plane_stride);
+                                                          plane_stride, flag);
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, size_t plane_stride, int P_pad,
-                           const int32_t* offsets, const int32_t* tile_off, int E, double* out,
-                           int32_t* flag, cudaStream_t st) {
-    TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_stride, P_pad, offsets, tile_off, E, out, flag};
+                           const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
+                           const float* row_scale, const int32_t* perm, int k_div, float* out,
+                           uint32_t* amax, cudaStream_t st) {
+    TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_stride, P_pad, P_pad - 128, offsets, tile_off,
+             E, flag, row_scale, perm, k_div, out, amax};
     k_tc_gemm<<<tc_grid(), TC_THREADS, sizeof(TcShared), st>>>(a);
     count_launches(1);
     return cudaGetLastError();

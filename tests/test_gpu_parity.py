@@ -395,3 +395,24 @@ def test_tc_option_validation(moe):
     with pytest.raises(moe.MoeError):
         moe.moe_set_option(99, 1)
     assert moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS) >= 1
+
+
+def test_forward_with_garbage_tables_raises_bounds_flag(moe):
+    # perm/pos/topk_idx that did not come from moe_sort: every index is checked
+    # inside the kernels, so the call completes and reports FLAG_BOUNDS
+    w = synth.custom("g", 6, 128, 4, 2, 128, 61)
+    d = synth.make(w)
+    packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]),
+                                  cu(d["w2_scales"]))
+    idx, gates = moe.moe_route(cu(d["logits"]), 2)
+    perm, pos, offsets = moe.moe_sort(idx, 4)
+    bad = torch.full_like(perm, 1 << 20)
+    ws = torch.empty(moe.moe_workspace_bytes(6, 128, 128, 4, 2), dtype=torch.uint8, device="cuda")
+    moe.moe_forward(cu(d["x"]).view(torch.bfloat16), idx, gates, bad, bad, offsets, packed, 128, 128, 4,
+                    ws=ws)
+    assert moe.moe_check_device_flag(ws) & moe.FLAG_BOUNDS
+    bad_off = offsets.clone()
+    bad_off[2] = 10 ** 6
+    moe.moe_forward(cu(d["x"]).view(torch.bfloat16), idx, gates, perm, pos, bad_off, packed, 128, 128, 4,
+                    ws=ws)
+    assert moe.moe_check_device_flag(ws) & moe.FLAG_BOUNDS
