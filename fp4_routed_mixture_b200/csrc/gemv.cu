@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
 }
 
 // Work split per expert: experts with at least tc_min rows go to the
-// tensor-core GEMM (tiles of 128 weight rows x 128 token rows), the others to
+// tensor-core GEMM (tiles of kTcWeightTile weight rows x kTcTokenTile token rows), the others to
 // the streaming GEMM (units of 32 weight rows x kGroup tokens).  Writes the
 // exclusive scans over experts of the streaming units of W1/W2 and of the
 // tensor-core tiles of W1/W2, and expert_tc[e] = 1 for tensor-core experts.
@@ -351,11 +351,11 @@ __global__ void k_plan(const int32_t* __restrict__ offsets, int E, int P, int n1
         const int m = any_bad ? 0 : offsets[e + 1] - offsets[e];
         const bool tc = m >= tc_min;
         const int g = tc ? 0 : (m + kGroup - 1) / kGroup;
-        const int nb = tc ? (m + 127) / 128 : 0;
+        const int nb = tc ? (m + kTcTokenTile - 1) / kTcTokenTile : 0;
         u1 = g * (n1 / 32);
         u2 = g * (n2 / 32);
-        t1 = nb * (n1 / 128);
-        t2 = nb * (n2 / 128);
+        t1 = nb * (n1 / kTcWeightTile);
+        t2 = nb * (n2 / kTcWeightTile);
     };
     int s[4] = {0, 0, 0, 0};
     for (int e = e0; e < e1; ++e) {

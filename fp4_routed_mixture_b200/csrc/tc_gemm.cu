@@ -21,16 +21,24 @@
 //       the same exact sum the CUDA-core kernel forms (every product is an
 //       integer multiple of the row's smallest weight scale).
 //
-// One persistent CTA per SM, warp-specialised:
+// Two persistent CTAs per SM, each warp-specialised:
 //   warp 0      producer: bulk copies of A and the three B planes into a
-//               6-stage ring (mbarrier transaction counts);
+//               3-stage ring (mbarrier transaction counts);
 //   warp 1      MMA issuer: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs per
 //               stage, tcgen05.commit frees the stage / publishes the tile;
 //   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld), one thread per
-//               weight row and half of the columns; W1 applies the token scale and SwiGLU (gate and up
-//               rows share a warp) and writes h plus the row maxima of |h|, W2
-//               writes the final fp32 Y; two accumulator buffers in TMEM let
-//               the epilogue overlap the next tile's MMAs.
+//               weight row and half of the columns; W1 applies the token scale
+//               and SwiGLU (gate and up rows share a warp) and writes h plus the
+//               row maxima of |h|, W2 writes the final fp32 Y; two accumulator
+//               buffers in TMEM let the epilogue overlap the next tile's MMAs.
+// Why two CTAs: the tensor core queues only a few MMAs, and an issuing thread
+// that waits on an mbarrier (a shared-memory operation, ordered behind its
+// queued MMAs) stalls for about as long as that queue lasts at N <= 128, so
+// one issuer leaves the pipe idle about half the time.  Two independent
+// issuers per SM fill each other's gaps (measured: 62-65 clocks per
+// 128 x 112..128 x 64 MMA per SM against 56-64 ideal, versus ~125 with one).
+// Each CTA owns half of the SM's TMEM (256 columns): two 112-column
+// accumulators plus the scale factors.
 // Every wait is bounded in time; a wait that gives up raises FLAG_TIMEOUT and
 // the roles wind down (copies in flight are waited for, TMEM is freed).
 #include "kernels.cuh"
@@ -38,17 +46,21 @@
 
 namespace moe {
 
-constexpr int TC_BM = 128;                     // weight rows per tile (MMA M)
-constexpr int TC_BN = 128;                     // token rows per tile (largest MMA N used)
-constexpr int TC_STAGES = 6;
+constexpr int TC_BM = kTcWeightTile;           // weight rows per tile (MMA M)
+constexpr int TC_BN = kTcTokenTile;            // token rows per tile (largest MMA N used)
+constexpr int TC_STAGES = 3;
 constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
-constexpr int TC_B_PLANE_BYTES = TC_BN * 64;   // 128 rows x 128 inputs, 4 bits each
+constexpr int TC_B_PLANE_BYTES = TC_BN * 64;   // TC_BN rows x 128 inputs, 4 bits each
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + 3 * TC_B_PLANE_BYTES;
 constexpr int TC_EPI_WARPS = 8;                // two per TMEM lane quadrant
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
-constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_SFA_COL = 2 * TC_BN;          // 4 columns per stage
+constexpr int TC_CTAS_PER_SM = 2;
+constexpr int TC_TMEM_COLS = 512 / TC_CTAS_PER_SM;   // the two CTAs of an SM split its TMEM
+constexpr int TC_SFA_COL = 2 * TC_BN;          // after two accumulator buffers; 4 columns per stage
 constexpr int TC_SFB_COL = TC_SFA_COL + 4 * TC_STAGES;  // 4 columns per plane
+static_assert(TC_SFB_COL + 12 <= TC_TMEM_COLS, "accumulators and scale factors exceed the TMEM share");
+static_assert(TC_SFA_COL % 4 == 0 && TC_SFB_COL % 4 == 0, "scale-factor columns hold 4 bytes per lane");
+static_assert(TC_BN % 16 == 0 && TC_BN <= 256, "MMA N");
 
 struct TcShared {
     uint8_t stage[TC_STAGES][TC_STAGE_BYTES];
@@ -219,7 +231,7 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     return tt;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a) {
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -494,7 +506,7 @@ static int tc_grid() {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaFuncSetAttribute(k_tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
-        grid = sms;
+        grid = sms * TC_CTAS_PER_SM;
     }
     return grid;
 }
