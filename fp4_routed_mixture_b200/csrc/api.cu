@@ -57,9 +57,9 @@ int check_dims(const moe_dims* d, bool need_T) {
 int g_tc_min_rows = 32;
 
 struct WsLayout {
-    size_t flag, uoff1, uoff2, toff1, toff2, etc, amax, sx, xq, xinit, hq, sh, hinit, px, ph, hbuf, yf,
-        gacc, yacc, total;
-    int P_pad;
+    size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xinit, hq, sh, hinit, px, ph,
+        hbuf, yf, gacc, yacc, total;
+    int plane_rows;
 };
 
 WsLayout ws_layout(const moe_dims& d, long long T) {
@@ -72,19 +72,20 @@ WsLayout ws_layout(const moe_dims& d, long long T) {
     L.uoff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.toff1 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.toff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.poff = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.etc = o; o += align_up(4 * (size_t)d.E, 256);
-    L.amax = o; o += align_up(4 * P, 256);
+    L.prow = o; o += align_up(4 * P, 256);
     L.sx = o; o += align_up(4 * (size_t)T, 256);
     L.xq = o; o += align_up((size_t)T * d.H, 256);
     L.xinit = o; o += align_up(4 * (size_t)T * (d.H / 32), 256);
     L.hq = o; o += align_up(P * d.I, 256);
     L.sh = o; o += align_up(4 * P, 256);
     L.hinit = o; o += align_up(4 * P * (d.I / 32), 256);
-    // digit planes of the tensor-core GEMM: 3 x [K/32][P_pad][16 bytes]; the
-    // last tile of an expert may read up to 128 rows past the end
-    L.P_pad = (int)P + 128;
-    L.px = o; o += align_up(3 * (size_t)(d.H / 32) * L.P_pad * 16, 256);
-    L.ph = o; o += align_up(3 * (size_t)(d.I / 32) * L.P_pad * 16, 256);
+    // digit planes of the tensor-core GEMM (stage-major, see kernels.cuh):
+    // each tensor-core expert's rows are padded to a multiple of 16
+    L.plane_rows = (int)align_up(P + 16 * (size_t)d.E + 16, 16);
+    L.px = o; o += align_up(moe::plane_bytes(d.H, L.plane_rows), 256);
+    L.ph = o; o += align_up(moe::plane_bytes(d.I, L.plane_rows), 256);
     L.hbuf = o; o += align_up(4 * P * d.I, 256);        // h of tensor-core rows
     L.yf = o; o += align_up(4 * P * d.H, 256);          // Y of tensor-core rows
     L.gacc = o; o += align_up(8 * P * 2 * d.I, 256);   // fp64 sums of streaming-GEMM rows
@@ -246,40 +247,41 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     int32_t* toff2 = (int32_t*)(w + L.toff2);
     uint8_t* px = (uint8_t*)(w + L.px);
     uint8_t* ph = (uint8_t*)(w + L.ph);
-    const size_t px_stride = (size_t)(H / 32) * L.P_pad * 16, ph_stride = (size_t)(I / 32) * L.P_pad * 16;
+    int32_t* poff = (int32_t*)(w + L.poff);
+    int32_t* prow = (int32_t*)(w + L.prow);
     // an expert has at most T rows, so the tensor-core path is skipped without
     // reading any count when T < tc_min
     const bool use_tc = T >= g_tc_min_rows;
     int32_t* etc = (int32_t*)(w + L.etc);
-    uint32_t* amax = (uint32_t*)(w + L.amax);
     float* hbuf = (float*)(w + L.hbuf);
     float* yf = (float*)(w + L.yf);
     MOE_TRY(moe::launch_plan(offsets, E, P, 2 * I, H, use_tc ? g_tc_min_rows : 0x7fffffff, uoff1, uoff2,
-                             toff1, toff2, etc, flag, stream), "plan");
-    MOE_TRY(moe::launch_prepare_rows(etc, topk_idx, perm, P, E, I, H, amax, gacc, yacc, flag, stream),
+                             toff1, toff2, poff, etc, flag, stream), "plan");
+    MOE_TRY(moe::launch_prepare_rows(etc, topk_idx, perm, offsets, poff, P, E, I, H, prow, gacc, yacc,
+                                     flag, stream),
             "row state");
     if (use_tc)
-        MOE_TRY(moe::launch_planes(xq, H, perm, k, P, L.P_pad, px, px_stride, flag, stream), "x planes");
+        MOE_TRY(moe::launch_planes(xq, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
                              uoff1, E, gacc, flag, I, P, stream), "W1");
     if (use_tc)
-        MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, px_stride, L.P_pad,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, amax, stream),
+        MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
-    MOE_TRY(moe::launch_hquant(gacc, hbuf, amax, etc, topk_idx, sx, perm, P, k, E, I, hq, sh, hinit,
+    MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, P, k, E, I, hq, sh, hinit,
                                dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
             "SwiGLU + h quant");
     if (use_tc)
-        MOE_TRY(moe::launch_planes(hq, I, perm, 0, P, L.P_pad, ph, ph_stride, flag, stream), "h planes");
+        MOE_TRY(moe::launch_planes(hq, I, perm, 0, P, prow, L.plane_rows, ph, flag, stream), "h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
                              uoff2, E, yacc, flag, 0, P, stream), "W2");
     if (use_tc)
-        MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, ph_stride, L.P_pad, offsets,
-                                    toff2, E, flag, sh, perm, 0, yf, nullptr, stream),
+        MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, yf, etc, topk_idx, sh, gates, pos, T, k, E, H, y_bf16, flag, stream),

@@ -42,12 +42,13 @@ cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
                           int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
-cudaError_t launch_hquant(const double* gacc, const float* hbuf, const uint32_t* amax,
+cudaError_t launch_hquant(const double* gacc, const float* hbuf,
                           const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
                           const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
                           int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st);
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                int P, int E, int I, int H, uint32_t* amax, double* gacc, double* yacc,
+                                const int32_t* offsets, const int32_t* plane_off, int P, int E, int I,
+                                int H, int32_t* plane_row, double* gacc, double* yacc,
                                 int32_t* flag, cudaStream_t st);
 cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
@@ -56,20 +57,28 @@ cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, flo
 
 cudaError_t launch_plan(const int32_t* offsets, int E, int P, int n1, int n2, int tc_min,
                         int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2,
-                        int32_t* expert_tc, int32_t* flag, cudaStream_t st);
+                        int32_t* plane_off, int32_t* expert_tc, int32_t* flag, cudaStream_t st);
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
                         const int32_t* flag, int gate_up_half, int P, cudaStream_t st);
 
 size_t tc_smem_bytes();
+// Digit planes, per 128-input stage g and group of 8 plane rows, hold
+// [plane 0..2][32-input chunk 0..3][8 rows][16 bytes] (1536 bytes); plane rows
+// are the sorted rows of tensor-core experts, each expert padded to 16 rows.
+constexpr int kPlaneGroupBytes = 1536;
+__host__ __device__ inline size_t plane_bytes(int K, int plane_rows) {
+    return (size_t)(K / 128) * (plane_rows / 8) * kPlaneGroupBytes;
+}
 cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
-                          int P_pad, uint8_t* planes, size_t plane_stride, int32_t* flag, cudaStream_t st);
+                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int32_t* flag,
+                          cudaStream_t st);
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
-                           const uint8_t* planes, size_t plane_stride, int P_pad,
+                           const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out,
-                           uint32_t* amax, cudaStream_t st);
+                           cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
                            const int32_t* topk_idx, const float* sh, const float* gates,

@@ -90,30 +90,32 @@ __global__ void __launch_bounds__(kQThreads)
 // One CTA per sorted row i: the row's h values and |h| maximum, then its INT8
 // codes.  Rows of experts on the streaming GEMM arrive as exact fp64 sums of
 // the W1 product (gate and up): G = fp32(fp64(sx[t]) * sum), h = SwiGLU(g, u)
-// here.  Rows of experts on the tensor-core GEMM arrive as h itself plus the
-// bits of max |h| (formed in that GEMM's epilogue).
+// here.  Rows of experts on the tensor-core GEMM arrive as h itself (formed in
+// that GEMM's epilogue).
 __global__ void __launch_bounds__(kQThreads)
     k_hquant(const double* __restrict__ gacc, const float* __restrict__ hbuf,
-             const uint32_t* __restrict__ amax_bits, const int32_t* __restrict__ expert_tc,
+             const int32_t* __restrict__ expert_tc,
              const int32_t* __restrict__ topk_idx, const float* __restrict__ sx,
              const int32_t* __restrict__ perm, int P, int k, int E, int I, int8_t* __restrict__ hq,
              float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
              float* __restrict__ dbg_sh, int32_t* flag) {
-    extern __shared__ float h[];  // [I]
+    extern __shared__ __align__(16) float h[];  // [I]
     __shared__ float red[33];
     const int i = blockIdx.x;
     const int p = checked_index(perm[i], P, flag);
     const bool tc = expert_tc[checked_index(topk_idx[p], E, flag)] != 0;
-    float a;
+    float a = 0.0f;
     if (tc) {
-        const float* hr = hbuf + (size_t)i * I;
-        for (int j = threadIdx.x; j < I; j += blockDim.x) h[j] = hr[j];
-        a = __uint_as_float(amax_bits[i]);
-        __syncthreads();
+        const float4* hr = reinterpret_cast<const float4*>(hbuf + (size_t)i * I);
+        for (int j = threadIdx.x; j < I / 4; j += blockDim.x) {
+            const float4 v = hr[j];
+            reinterpret_cast<float4*>(h)[j] = v;
+            a = fmaxf(fmaxf(a, fabsf(v.x)), fmaxf(fmaxf(fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
+        }
+        a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
     } else {
         const double s = (double)sx[p / k];
         const double* g = gacc + (size_t)i * 2 * I;
-        a = 0.0f;
         for (int j = threadIdx.x; j < I; j += blockDim.x) {
             const float gv = (float)__dmul_rn(s, g[j]);
             const float uv = (float)__dmul_rn(s, g[I + j]);
@@ -150,16 +152,33 @@ __global__ void __launch_bounds__(kQThreads)
     }
 }
 
-// Per sorted row: clears the row's |h| maximum and, for rows of experts on
-// the streaming GEMM, its fp64 accumulators (that GEMM adds partial sums into
-// them).  Rows of tensor-core experts are written whole by that GEMM.
+// Per sorted row: for rows of tensor-core experts writes the row's place in the digit-plane buffers
+// (plane_off[e] + rank inside the expert), for the others -1 and clears the
+// fp64 accumulators (the streaming GEMM adds partial sums into them).  Rows of
+// tensor-core experts are written whole by that GEMM.  A row whose expert's
+// offsets do not contain it (tables that did not come from one sort) raises
+// FLAG_BOUNDS and gets no plane row.
 __global__ void __launch_bounds__(256)
     k_prepare_rows(const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
-                   const int32_t* __restrict__ perm, int P, int E, int I, int H, uint32_t* __restrict__ amax,
+                   const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ plane_off, int P, int E, int I, int H,
+                   int32_t* __restrict__ plane_row,
                    double* __restrict__ gacc, double* __restrict__ yacc, int32_t* flag) {
     for (int i = blockIdx.x; i < P; i += gridDim.x) {
-        if (threadIdx.x == 0) amax[i] = 0u;
-        if (expert_tc[checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag)]) continue;
+        const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
+        const bool tc = expert_tc[e] != 0;
+        if (threadIdx.x == 0) {
+            int pr = -1;
+            if (tc) {
+                const int r0 = offsets[e], r1 = offsets[e + 1];
+                if (i >= r0 && i < r1)
+                    pr = plane_off[e] + (i - r0);
+                else
+                    raise_flag(flag, FLAG_BOUNDS);
+            }
+            plane_row[i] = pr;
+        }
+        if (tc) continue;
         double2* g = reinterpret_cast<double2*>(gacc + (size_t)i * 2 * I);
         for (int j = threadIdx.x; j < I; j += blockDim.x) g[j] = make_double2(0.0, 0.0);
         double2* y = reinterpret_cast<double2*>(yacc + (size_t)i * H);
@@ -218,12 +237,12 @@ cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_hquant(const double* gacc, const float* hbuf, const uint32_t* amax,
+cudaError_t launch_hquant(const double* gacc, const float* hbuf,
                           const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
                           const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
                           int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
-    k_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, hbuf, amax, expert_tc, topk_idx, sx,
+    k_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, hbuf, expert_tc, topk_idx, sx,
                                                                perm, P, k, E, I, hq, sh, hinit, dbg_hq,
                                                                dbg_sh, flag);
     count_launches(1);
@@ -231,11 +250,12 @@ cudaError_t launch_hquant(const double* gacc, const float* hbuf, const uint32_t*
 }
 
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                int P, int E, int I, int H, uint32_t* amax, double* gacc, double* yacc,
+                                const int32_t* offsets, const int32_t* plane_off, int P, int E, int I,
+                                int H, int32_t* plane_row, double* gacc, double* yacc,
                                 int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
-    k_prepare_rows<<<std::min(P, 148 * 8), 256, 0, st>>>(expert_tc, topk_idx, perm, P, E, I, H, amax,
-                                                          gacc, yacc, flag);
+    k_prepare_rows<<<std::min(P, 148 * 8), 256, 0, st>>>(expert_tc, topk_idx, perm, offsets, plane_off, P, E,
+                                                          I, H, plane_row, gacc, yacc, flag);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -15,22 +15,26 @@
 //   B = the INT8 activations of the expert's sorted rows, written exactly as
 //       three E2M1 digit planes: q = 64*a + 8*b + c with a, b, c in [-4, 3]
 //       (balanced base-8 digits; every digit is an E2M1 value).  Plane p has
-//       the constant scale 2^(6 - 3p).  Each plane is stored chunk-major
-//       ([K/32][rows][16 bytes]) so that the N rows of a tile are contiguous.
+//       the constant scale 2^(6 - 3p).  The planes are stored stage-major:
+//       for every 128-input stage and group of 8 rows, [plane][32-input
+//       chunk][8 rows][16 bytes] (1536 bytes), and every expert's rows start
+//       on a 16-row boundary, so the whole B operand of a tile and stage is
+//       one contiguous block: one bulk copy (the copy engine moves about one
+//       copy per 80 clocks per CTA, so many small copies cannot feed the MMAs).
 //   D (TMEM, fp32) = sum over planes of A * SFA * B_p * SFB_p = sum_k w * q:
 //       the same exact sum the CUDA-core kernel forms (every product is an
 //       integer multiple of the row's smallest weight scale).
 //
 // Two persistent CTAs per SM, each warp-specialised:
-//   warp 0      producer: bulk copies of A and the three B planes into a
-//               3-stage ring (mbarrier transaction counts);
+//   warp 0      producer: two bulk copies per stage (A chunk, B planes) into
+//               a 3-stage ring (mbarrier transaction counts);
 //   warp 1      MMA issuer: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs per
 //               stage, tcgen05.commit frees the stage / publishes the tile;
 //   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld), one thread per
 //               weight row and half of the columns; W1 applies the token scale
-//               and SwiGLU (gate and up rows share a warp) and writes h plus the
-//               row maxima of |h|, W2 writes the final fp32 Y; two accumulator
-//               buffers in TMEM let the epilogue overlap the next tile's MMAs.
+//               and SwiGLU (gate and up rows share a warp) and writes h, W2
+//               writes the final fp32 Y; two accumulator buffers in TMEM let
+//               the epilogue overlap the next tile's MMAs.
 // Why two CTAs: the tensor core queues only a few MMAs, and an issuing thread
 // that waits on an mbarrier (a shared-memory operation, ordered behind its
 // queued MMAs) stalls for about as long as that queue lasts at N <= 128, so
@@ -50,8 +54,8 @@ constexpr int TC_BM = kTcWeightTile;           // weight rows per tile (MMA M)
 constexpr int TC_BN = kTcTokenTile;            // token rows per tile (largest MMA N used)
 constexpr int TC_STAGES = 3;
 constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
-constexpr int TC_B_PLANE_BYTES = TC_BN * 64;   // TC_BN rows x 128 inputs, 4 bits each
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + 3 * TC_B_PLANE_BYTES;
+constexpr int TC_B_BYTES = TC_BN / 8 * kPlaneGroupBytes;  // 3 planes x TC_BN rows x 128 inputs
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_EPI_WARPS = 8;                // two per TMEM lane quadrant
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr int TC_CTAS_PER_SM = 2;
@@ -77,9 +81,9 @@ struct TcArgs {
     int K;                     // inputs per weight row
     int N;                     // weight rows per expert
     int gate_up_half;          // W1: I (gate/up interleave), W2: 0
-    const uint8_t* planes;     // 3 digit planes, [K/32][P_pad][16] each
-    size_t plane_stride;       // bytes per plane
-    int P_pad;
+    const uint8_t* planes;     // digit planes, stage-major (see above)
+    int plane_rows;            // rows of the plane buffer (multiple of 16)
+    const int32_t* plane_off;  // [E+1] first plane row of each expert (multiple of 16)
     int P;                     // sorted rows (pairs)
     const int32_t* offsets;    // [E+1]
     const int32_t* tile_off;   // [E+1] exclusive scan of tiles per expert
@@ -90,7 +94,6 @@ struct TcArgs {
     const int32_t* perm;       // sorted row -> pair id (W1: source row = perm[i] / k_div)
     int k_div;                 // W1: k; W2: 0 (source row = sorted row)
     float* out;                // W1: h [P, I]; W2: Y [P, H]  (fp32, final values)
-    uint32_t* amax;            // W1: per sorted row, bits of max |h| (atomicMax); W2: unused
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -209,7 +212,7 @@ __device__ __forceinline__ uint32_t make_idesc(int n, int a_sf_id, int b_sf_id) 
 }
 
 struct TcTile {
-    int e, rb, i0, n_valid, n_mma;
+    int e, rb, i0, pr0, n_valid, n_mma;   // i0: first sorted row, pr0: its plane row
 };
 
 __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
@@ -226,6 +229,7 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     tt.rb = local % RB;
     const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
     tt.i0 = r0 + nb * TC_BN;
+    tt.pr0 = __ldg(a.plane_off + lo) + nb * TC_BN;
     tt.n_valid = min(TC_BN, r1 - tt.i0);
     tt.n_mma = (tt.n_valid + 15) & ~15;
     return tt;
@@ -282,7 +286,11 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
         for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
             const TcTile tt = tile_at(a, t);
             const uint8_t* wsrc = a.w + (size_t)tt.e * a.expert_bytes + (size_t)tt.rb * KG * TC_A_BYTES;
-            const uint32_t bbytes = 16u * (uint32_t)tt.n_mma;  // one 32-input chunk of one plane
+            const uint32_t bbytes = (uint32_t)(tt.n_mma / 8) * kPlaneGroupBytes;  // B of one stage
+            // the tile's rows must lie inside the plane buffer (a plane_off
+            // table that did not come from the planner is refused here)
+            const bool rows_ok = tt.pr0 >= 0 && (tt.pr0 & 15) == 0 && tt.pr0 + tt.n_mma <= a.plane_rows;
+            if (!rows_ok && lane == 0) raise_flag(a.flag, FLAG_BOUNDS);
             for (int g = 0; g < KG; ++g) {
                 const uint32_t fb = smem_u32(&sh.full[stage]), eb = smem_u32(&sh.empty[stage]);
                 if (!mbar_wait(eb, phase ^ 1u, abort)) {
@@ -290,15 +298,16 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
                     break;
                 }
                 const uint32_t sbase = smem_u32(sh.stage[stage]);
-                if (lane == 0) mbar_expect_tx(fb, TC_A_BYTES + 12u * bbytes);
-                __syncwarp();
                 if (lane == 0) {
-                    bulk_g2s(sbase, wsrc + (size_t)g * TC_A_BYTES, TC_A_BYTES, fb);
-                } else if (lane <= 12) {
-                    const int p = (lane - 1) >> 2, cc = (lane - 1) & 3;
-                    const uint8_t* src = a.planes + (size_t)p * a.plane_stride +
-                                         ((size_t)(4 * g + cc) * a.P_pad + tt.i0) * 16;
-                    bulk_g2s(sbase + TC_A_BYTES + p * TC_B_PLANE_BYTES + cc * bbytes, src, bbytes, fb);
+                    if (rows_ok) {
+                        mbar_expect_tx(fb, TC_A_BYTES + bbytes);
+                        bulk_g2s(sbase, wsrc + (size_t)g * TC_A_BYTES, TC_A_BYTES, fb);
+                        const uint8_t* src =
+                            a.planes + ((size_t)g * (a.plane_rows / 8) + tt.pr0 / 8) * kPlaneGroupBytes;
+                        bulk_g2s(sbase + TC_A_BYTES, src, bbytes, fb);
+                    } else {
+                        mbar_arrive(fb);  // keep the ring moving; the tile's result is not used
+                    }
                 }
                 __syncwarp();
                 filled[stage] = true;
@@ -332,7 +341,6 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
             }
             tc_fence_after();
             const uint32_t dcol = tmem + buf * TC_BN;
-            const uint32_t bbytes = 16u * (uint32_t)tt.n_mma;
             bool ok = true;
             for (int g = 0; g < KG; ++g) {
                 if (!mbar_wait(smem_u32(&sh.full[stage]), phase, abort)) {
@@ -350,8 +358,10 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
                         const uint64_t adesc = make_sdesc(sbase + 512 + ks * 2 * 2048, 2048, 128);
 #pragma unroll
                         for (int p = 0; p < 3; ++p) {
-                            const uint64_t bdesc = make_sdesc(
-                                sbase + TC_A_BYTES + p * TC_B_PLANE_BYTES + ks * 2 * bbytes, bbytes, 128);
+                            // plane p, chunks 2ks and 2ks+1: K-adjacent core
+                            // matrices 128 bytes apart, 8-row groups 1536 apart
+                            const uint64_t bdesc = make_sdesc(sbase + TC_A_BYTES + p * 512 + ks * 256, 128,
+                                                              kPlaneGroupBytes);
                             const uint32_t idesc = make_idesc(tt.n_mma, 2 * ks, 0);
                             tc_mma_mxf4(dcol, adesc, bdesc, idesc, sfa,
                                         tmem + TC_SFB_COL + 4 * p, (g | ks | p) != 0);
@@ -385,15 +395,14 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
         // W1: lanes 0-15 of a warp hold the gate rows and lanes 16-31 the up
         // rows of the same 16 outputs (row interleave of pack.cu).  Columns go
         // in pairs: lanes 0-15 form h for column j (up value shuffled down),
-        // lanes 16-31 for column j+1 (gate value shuffled up), h = SwiGLU(g, u);
-        // h is stored and |h| folded into the row maximum (max over 16 lanes,
-        // then one atomicMax per half-warp and column; max is order-independent).
-        // W2: Y = s * acc straight out.
+        // lanes 16-31 for column j+1 (gate value shuffled up), h = SwiGLU(g, u),
+        // stored in fp32 (the row maximum of |h| is taken when h is
+        // requantised).  W2: Y = s * acc straight out.
         const int ew = warp - 2;
         const int q = warp & 3;            // TMEM lane quadrant this warp may access
         const int half = ew >> 2;          // which alternate 32-column chunks
         const int m = q * 32 + lane;       // weight row within the tile
-        const bool w1 = a.amax != nullptr;
+        const bool w1 = a.gate_up_half > 0;
         float* csc = sh.col_scale[ew];
         int buf = 0;
         uint32_t acc_phase = 0;
@@ -429,14 +438,7 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
                         const float from_hi = __shfl_down_sync(0xffffffffu, v0, 16);  // up value, column j
                         const float from_lo = __shfl_up_sync(0xffffffffu, v1, 16);    // gate value, column j+1
                         const float hv = lo ? swiglu(v0, from_hi) : swiglu(from_lo, v1);
-                        const int col = n0 + j + (lo ? 0 : 1);
-                        float am = fabsf(hv);
-#pragma unroll
-                        for (int o = 8; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-                        if (col < tt.n_valid) {
-                            out[(size_t)(j + (lo ? 0 : 1)) * I] = hv;
-                            if ((lane & 15) == 0) atomicMax(a.amax + tt.i0 + col, __float_as_uint(am));
-                        }
+                        if (n0 + j + (lo ? 0 : 1) < tt.n_valid) out[(size_t)(j + (lo ? 0 : 1)) * I] = hv;
                     }
                 }
             }
@@ -458,19 +460,26 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
                      : "memory");
 }
 
-// Writes the three E2M1 digit planes of INT8 rows in chunk-major order:
-// plane p, input chunk c (32 inputs), row i -> 16 bytes at
-// planes + p*plane_stride + (c*P_pad + i)*16; element 2j of the chunk in the
-// low nibble of byte j.  Source row of sorted row i: perm[i] / k_div (k_div > 0)
-// or i.  One thread per (row, chunk), rows fastest: consecutive threads write
-// consecutive 16-byte pieces of a plane.
+// Writes the three E2M1 digit planes of INT8 rows in the stage-major layout:
+// plane p, 32-input chunk c = 4*g + cc of plane row pr -> 16 bytes at
+// planes + (g*(plane_rows/8) + pr/8)*1536 + p*512 + cc*128 + (pr%8)*16, element
+// 2j of the chunk in the low nibble of byte j.  Source row of sorted row i:
+// perm[i] / k_div (k_div > 0) or i; its plane row is plane_row[i] (-1: a row of
+// a streaming-GEMM expert, not written).  One thread per (row, chunk), rows
+// fastest: 8 consecutive rows fill 128 contiguous bytes of each plane.
 __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm,
-                         int k_div, int rows, int P_pad, uint8_t* __restrict__ planes,
-                         size_t plane_stride, int32_t* flag) {
+                         int k_div, int rows, const int32_t* __restrict__ plane_row, int plane_rows,
+                         uint8_t* __restrict__ planes, int32_t* flag) {
     const int nc = K / 32;
     const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (id >= (long long)rows * nc) return;
     const int i = (int)(id % rows), c = (int)(id / rows);
+    const int pr = __ldg(plane_row + i);
+    if (pr < 0) return;
+    if (pr >= plane_rows) {
+        raise_flag(flag, FLAG_BOUNDS);
+        return;
+    }
     const int srow = k_div > 0 ? checked_index(__ldg(perm + i), rows, flag) / k_div : i;
     const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
     const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
@@ -493,10 +502,12 @@ __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* _
         out[1][e >> 3] |= code(b0) << (4 * (e & 7));
         out[2][e >> 3] |= code(c0) << (4 * (e & 7));
     }
+    const int g = c >> 2, cc = c & 3;
+    uint8_t* dst = planes + ((size_t)g * (plane_rows / 8) + (pr >> 3)) * kPlaneGroupBytes + cc * 128 +
+                   (pr & 7) * 16;
 #pragma unroll
     for (int p = 0; p < 3; ++p)
-        *reinterpret_cast<uint4*>(planes + (size_t)p * plane_stride + ((size_t)c * P_pad + i) * 16) =
-            make_uint4(out[p][0], out[p][1], out[p][2], out[p][3]);
+        *reinterpret_cast<uint4*>(dst + p * 512) = make_uint4(out[p][0], out[p][1], out[p][2], out[p][3]);
 }
 
 static int tc_grid() {
@@ -514,22 +525,23 @@ static int tc_grid() {
 size_t tc_smem_bytes() { return sizeof(TcShared); }
 
 cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
-                          int P_pad, uint8_t* planes, size_t plane_stride, int32_t* flag, cudaStream_t st) {
+                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int32_t* flag,
+                          cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
     const long long n = (long long)rows * (K / 32);
-    k_planes<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, K, perm, k_div, rows, P_pad, planes,
-                                                          plane_stride, flag);
+    k_planes<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, K, perm, k_div, rows, plane_row, plane_rows,
+                                                          planes, flag);
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
-                           const uint8_t* planes, size_t plane_stride, int P_pad,
+                           const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out,
-                           uint32_t* amax, cudaStream_t st) {
-    TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_stride, P_pad, P_pad - 128, offsets, tile_off,
-             E, flag, row_scale, perm, k_div, out, amax};
+                           cudaStream_t st) {
+    TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
+             E, flag, row_scale, perm, k_div, out};
     k_tc_gemm<<<tc_grid(), TC_THREADS, sizeof(TcShared), st>>>(a);
     count_launches(1);
     return cudaGetLastError();
