@@ -271,11 +271,9 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
                                     offsets, toff1, E, flag, sx, perm, k, hbuf, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
-    MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, P, k, E, I, hq, sh, hinit,
-                               dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
-            "SwiGLU + h quant");
-    if (use_tc)
-        MOE_TRY(moe::launch_planes(hq, I, perm, 0, P, prow, L.plane_rows, ph, flag, stream), "h planes");
+    MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, prow, L.plane_rows, ph, P, k, E, I, hq,
+                               sh, hinit, dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
+            "SwiGLU + h quant + h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
                              uoff2, E, yacc, flag, 0, P, stream), "W2");

@@ -11,35 +11,44 @@
 
 namespace moe {
 
+// One thread per 4 consecutive columns of one token (16-byte loads of Y).
 __global__ void __launch_bounds__(256)
     k_combine(const double* __restrict__ yacc, const float* __restrict__ yf,
               const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
               const float* __restrict__ sh, const float* __restrict__ gates,
-              const int32_t* __restrict__ pos, int P, int k, int E, int H, __nv_bfloat162* __restrict__ y,
+              const int32_t* __restrict__ pos, int P, int k, int E, int H, uint2* __restrict__ y,
               int32_t* flag) {
     const int t = blockIdx.y;
-    const int n2 = blockIdx.x * blockDim.x + threadIdx.x;  // pair of columns
-    if (2 * n2 >= H) return;
-    float acc0 = 0.0f, acc1 = 0.0f;
+    const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
+    if (4 * n4 >= H) return;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     for (int j = 0; j < k; ++j) {
         const int p = t * k + j;
         const int i = checked_index(__ldg(pos + p), P, flag);
         const float g = __ldg(gates + p);
-        float y0, y1;
+        float v[4];
         if (__ldg(expert_tc + checked_index(__ldg(topk_idx + p), E, flag))) {
-            const float2 v = __ldg(reinterpret_cast<const float2*>(yf + (size_t)i * H) + n2);
-            y0 = v.x;
-            y1 = v.y;
+            const float4 f = __ldg(reinterpret_cast<const float4*>(yf + (size_t)i * H) + n4);
+            v[0] = f.x;
+            v[1] = f.y;
+            v[2] = f.z;
+            v[3] = f.w;
         } else {
             const double s = (double)__ldg(sh + i);
-            const double2 v = __ldg(reinterpret_cast<const double2*>(yacc + (size_t)i * H) + n2);
-            y0 = (float)__dmul_rn(s, v.x);
-            y1 = (float)__dmul_rn(s, v.y);
+            const double2* r = reinterpret_cast<const double2*>(yacc + (size_t)i * H) + 2 * n4;
+            const double2 d0 = __ldg(r), d1 = __ldg(r + 1);
+            v[0] = (float)__dmul_rn(s, d0.x);
+            v[1] = (float)__dmul_rn(s, d0.y);
+            v[2] = (float)__dmul_rn(s, d1.x);
+            v[3] = (float)__dmul_rn(s, d1.y);
         }
-        acc0 = __fmaf_rn(g, y0, acc0);
-        acc1 = __fmaf_rn(g, y1, acc1);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(g, v[c], acc[c]);
     }
-    y[(size_t)t * (H / 2) + n2] = __floats2bfloat162_rn(acc0, acc1);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+    y[(size_t)t * (H / 4) + n4] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                             *reinterpret_cast<const uint32_t*>(&hi));
 }
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
@@ -47,9 +56,9 @@ cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* e
                            const int32_t* pos, int T, int k, int E, int H, void* y, int32_t* flag,
                            cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    dim3 grid((H / 2 + 255) / 256, T);
+    dim3 grid((H / 4 + 255) / 256, T);
     k_combine<<<grid, 256, 0, st>>>(yacc, yf, expert_tc, topk_idx, sh, gates, pos, T * k, k, E, H,
-                                    (__nv_bfloat162*)y, flag);
+                                    (uint2*)y, flag);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -42,10 +42,11 @@ cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
                           int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
-cudaError_t launch_hquant(const double* gacc, const float* hbuf,
-                          const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
-                          const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
-                          int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st);
+cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
+                          const int32_t* topk_idx, const float* sx, const int32_t* perm,
+                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
+                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
+                          int32_t* flag, cudaStream_t st);
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
                                 const int32_t* offsets, const int32_t* plane_off, int P, int E, int I,
                                 int H, int32_t* plane_row, double* gacc, double* yacc,

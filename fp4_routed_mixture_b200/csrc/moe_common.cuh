@@ -82,6 +82,23 @@ __device__ __forceinline__ int quant_code(float v, float amax, float s) {
     return (int)r;
 }
 
+// E2M1 codes of the three balanced base-8 digits of an INT8 code q =
+// 64*a + 8*b + c (a in [-2, 2], b and c in [-4, 3]): a | b << 4 | c << 8.  A
+// digit d has code 0, 2, 4, 5, 6 for |d| = 0..4 (nibbles packed in 0x65420)
+// with the sign in bit 3.  Both digit-plane writers build a 256-entry table
+// from it.
+__device__ __forceinline__ uint32_t digit_codes(int q) {
+    const int c0 = ((q + 4) & 7) - 4;
+    const int q1 = (q - c0) >> 3;
+    const int b0 = ((q1 + 4) & 7) - 4;
+    const int a0 = (q1 - b0) >> 3;
+    auto code = [](int d) -> uint32_t {
+        const uint32_t mag = (0x65420u >> (4 * (d < 0 ? -d : d))) & 0xFu;
+        return d < 0 ? (8u | mag) : mag;
+    };
+    return code(a0) | code(b0) << 4 | code(c0) << 8;
+}
+
 // 2^(S-128) as a double (S is a UE8M0 byte in [0, 254]); used as the weight
 // scale of codes that are decoded to 2*e2m1 integers.
 __device__ __forceinline__ double pow2_scale_minus128(uint32_t S) {

@@ -87,68 +87,118 @@ __global__ void __launch_bounds__(kQThreads)
     }
 }
 
-// One CTA per sorted row i: the row's h values and |h| maximum, then its INT8
-// codes.  Rows of experts on the streaming GEMM arrive as exact fp64 sums of
-// the W1 product (gate and up): G = fp32(fp64(sx[t]) * sum), h = SwiGLU(g, u)
-// here.  Rows of experts on the tensor-core GEMM arrive as h itself (formed in
-// that GEMM's epilogue).
+// R threads per sorted row (R = 32: a warp per row, for many rows; R = 256:
+// a CTA per row, for few), grid-stride over rows: the row's h values and |h|
+// maximum, then its INT8 codes.  Rows of experts on the streaming GEMM arrive
+// as exact fp64 sums of the W1 product (gate and up):
+// G = fp32(fp64(sx[t]) * sum), h = SwiGLU(g, u) is formed here and parked in
+// hbuf; rows of experts on the tensor-core GEMM arrive as h itself in hbuf
+// (formed in that GEMM's epilogue).  Pass 1 reads the row and reduces the
+// maximum, pass 2 reads it again (each thread its own elements, from cache)
+// and quantises: streaming rows get hq and the block sums hinit their GEMM
+// needs, tensor-core rows get the digit planes of the W2 tensor-core GEMM
+// written directly (plane row plane_row[i]).  Thread l of a row holds the
+// elements 4*(l + R*g) .. +3 in step g; 8 consecutive threads cover one
+// 32-input chunk.
+template <int R>
 __global__ void __launch_bounds__(kQThreads)
-    k_hquant(const double* __restrict__ gacc, const float* __restrict__ hbuf,
-             const int32_t* __restrict__ expert_tc,
-             const int32_t* __restrict__ topk_idx, const float* __restrict__ sx,
-             const int32_t* __restrict__ perm, int P, int k, int E, int I, int8_t* __restrict__ hq,
-             float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
-             float* __restrict__ dbg_sh, int32_t* flag) {
-    extern __shared__ __align__(16) float h[];  // [I]
+    k_hquant(const double* __restrict__ gacc, float* __restrict__ hbuf,
+             const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
+             const float* __restrict__ sx, const int32_t* __restrict__ perm,
+             const int32_t* __restrict__ plane_row, int plane_rows, uint8_t* __restrict__ planes,
+             int P, int k, int E, int I, int8_t* __restrict__ hq, float* __restrict__ sh,
+             int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh,
+             int32_t* flag) {
+    static_assert(R == 32 || R == kQThreads, "a warp or a CTA per row");
+    __shared__ uint16_t lut[256];
     __shared__ float red[33];
-    const int i = blockIdx.x;
-    const int p = checked_index(perm[i], P, flag);
-    const bool tc = expert_tc[checked_index(topk_idx[p], E, flag)] != 0;
-    float a = 0.0f;
-    if (tc) {
-        const float4* hr = reinterpret_cast<const float4*>(hbuf + (size_t)i * I);
-        for (int j = threadIdx.x; j < I / 4; j += blockDim.x) {
-            const float4 v = hr[j];
-            reinterpret_cast<float4*>(h)[j] = v;
-            a = fmaxf(fmaxf(a, fabsf(v.x)), fmaxf(fmaxf(fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
+    for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
+    __syncthreads();
+    const int l = threadIdx.x % R;
+    const int rows_per_cta = kQThreads / R;
+    const int steps = I / (4 * R);          // I % 128 == 0; for R = 256 also I % 1024 == 0 (checked by the launcher)
+    for (int i0 = blockIdx.x * rows_per_cta; i0 < P; i0 += gridDim.x * rows_per_cta) {
+        const int i = i0 + (int)threadIdx.x / R;
+        const bool row_ok = i < P;           // (R = 256: always)
+        float a = 0.0f;
+        bool tc = false;
+        int p = 0;
+        if (row_ok) {
+            p = checked_index(perm[i], P, flag);
+            tc = expert_tc[checked_index(topk_idx[p], E, flag)] != 0;
         }
-        a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
-    } else {
-        const double s = (double)sx[p / k];
-        const double* g = gacc + (size_t)i * 2 * I;
-        for (int j = threadIdx.x; j < I; j += blockDim.x) {
-            const float gv = (float)__dmul_rn(s, g[j]);
-            const float uv = (float)__dmul_rn(s, g[I + j]);
-            const float hv = swiglu(gv, uv);
-            h[j] = hv;
-            a = fmaxf(a, fabsf(hv));
-        }
-        a = block_max(a, red);  // contains __syncthreads: h[] is complete afterwards
-    }
-    const float sc = quant_scale(a);
-    if (threadIdx.x == 0) {
-        sh[i] = sc;
-        if (dbg_sh) dbg_sh[i] = sc;
-    }
-    // 4 codes per thread-step; 8 consecutive lanes cover one 32-element block
-    for (int j0 = 0; j0 < I; j0 += 4 * blockDim.x) {
-        const int j = j0 + 4 * threadIdx.x;
-        int bsum = 0;
-        if (j < I) {
-            uint32_t packed = 0;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int q = quant_code(h[j + u], a, sc);
-                bsum += q;
-                packed |= (uint32_t)(q & 0xff) << (8 * u);
+        float4* hr = reinterpret_cast<float4*>(hbuf + (size_t)(row_ok ? i : 0) * I);
+        if (row_ok && tc) {
+            for (int g = 0; g < steps; ++g) {
+                const float4 v = hr[g * R + l];
+                a = fmaxf(fmaxf(a, fabsf(v.x)), fmaxf(fmaxf(fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
             }
-            *reinterpret_cast<uint32_t*>(hq + (size_t)i * I + j) = packed;
-            if (dbg_hq) *reinterpret_cast<uint32_t*>(dbg_hq + (size_t)i * I + j) = packed;
+        } else if (row_ok) {
+            const double s = (double)sx[p / k];
+            const double* gr = gacc + (size_t)i * 2 * I;
+            for (int g = 0; g < steps; ++g) {
+                const int e0 = 4 * (g * R + l);
+                float hv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float gv = (float)__dmul_rn(s, gr[e0 + u]);
+                    const float uv = (float)__dmul_rn(s, gr[I + e0 + u]);
+                    hv[u] = swiglu(gv, uv);
+                    a = fmaxf(a, fabsf(hv[u]));
+                }
+                hr[g * R + l] = make_float4(hv[0], hv[1], hv[2], hv[3]);  // read back by this thread
+            }
         }
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 4);
-        if (j < I && (j & 31) == 0) hinit[(size_t)i * (I / 32) + (j >> 5)] = -12 * bsum;
+        if (R == 32)
+            a = warp_max(a);
+        else
+            a = block_max(a, red);
+        if (!row_ok) continue;  // (R = 32 only: whole warps skip together)
+        const float sc = quant_scale(a);
+        if (l == 0) {
+            sh[i] = sc;
+            if (dbg_sh) dbg_sh[i] = sc;
+        }
+        int pr = -1;
+        if (tc) {
+            pr = plane_row[i];
+            if (pr >= plane_rows || pr < 0) {
+                if (l == 0) raise_flag(flag, FLAG_BOUNDS);
+                pr = -1;
+            }
+        }
+        for (int g = 0; g < steps; ++g) {
+            const int e0 = 4 * (g * R + l);
+            const float4 v = hr[g * R + l];
+            const int q[4] = {quant_code(v.x, a, sc), quant_code(v.y, a, sc), quant_code(v.z, a, sc),
+                              quant_code(v.w, a, sc)};
+            const uint32_t packed = (uint32_t)(q[0] & 0xff) | (uint32_t)(q[1] & 0xff) << 8 |
+                                    (uint32_t)(q[2] & 0xff) << 16 | (uint32_t)(q[3] & 0xff) << 24;
+            if (dbg_hq) *reinterpret_cast<uint32_t*>(dbg_hq + (size_t)i * I + e0) = packed;
+            if (!tc) {
+                *reinterpret_cast<uint32_t*>(hq + (size_t)i * I + e0) = packed;
+                int bsum = q[0] + q[1] + q[2] + q[3];
+                bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
+                bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
+                bsum += __shfl_xor_sync(0xffffffffu, bsum, 4);
+                if ((l & 7) == 0) hinit[(size_t)i * (I / 32) + (e0 >> 5)] = -12 * bsum;
+            } else if (pr >= 0) {
+                // 4 codes = 16 bits of each plane's 16-byte piece of chunk e0/32
+                uint32_t d[3] = {0u, 0u, 0u};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t t = lut[q[u] & 0xff];
+                    d[0] |= (t & 0xFu) << (4 * u);
+                    d[1] |= ((t >> 4) & 0xFu) << (4 * u);
+                    d[2] |= (t >> 8) << (4 * u);
+                }
+                const int st = e0 >> 7, cc = (e0 >> 5) & 3;
+                uint8_t* dst = planes + ((size_t)st * (plane_rows / 8) + (pr >> 3)) * kPlaneGroupBytes +
+                               cc * 128 + (pr & 7) * 16 + ((e0 & 31) >> 2) * 2;
+#pragma unroll
+                for (int pl = 0; pl < 3; ++pl) *reinterpret_cast<uint16_t*>(dst + pl * 512) = (uint16_t)d[pl];
+            }
+        }
     }
 }
 
@@ -237,14 +287,25 @@ cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_hquant(const double* gacc, const float* hbuf,
-                          const int32_t* expert_tc, const int32_t* topk_idx, const float* sx,
-                          const int32_t* perm, int P, int k, int E, int I, int8_t* hq, float* sh,
-                          int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag, cudaStream_t st) {
+cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
+                          const int32_t* topk_idx, const float* sx, const int32_t* perm,
+                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
+                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
+                          int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
-    k_hquant<<<P, kQThreads, (size_t)I * sizeof(float), st>>>(gacc, hbuf, expert_tc, topk_idx, sx,
-                                                               perm, P, k, E, I, hq, sh, hinit, dbg_hq,
-                                                               dbg_sh, flag);
+    // few rows (decode): a CTA per row keeps every row's chain short; many
+    // rows (prefill): a warp per row needs no block barriers
+    if (P < 4096 && I % (4 * kQThreads) == 0) {
+        k_hquant<kQThreads><<<std::min(P, 148 * 8), kQThreads, 0, st>>>(
+            gacc, hbuf, expert_tc, topk_idx, sx, perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh,
+            hinit, dbg_hq, dbg_sh, flag);
+    } else {
+        const int warps = kQThreads / 32;
+        const int grid = std::min((P + warps - 1) / warps, 148 * 8);
+        k_hquant<32><<<grid, kQThreads, 0, st>>>(gacc, hbuf, expert_tc, topk_idx, sx, perm, plane_row,
+                                                 plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq,
+                                                 dbg_sh, flag);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

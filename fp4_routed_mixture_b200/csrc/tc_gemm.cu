@@ -467,9 +467,13 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
 // perm[i] / k_div (k_div > 0) or i; its plane row is plane_row[i] (-1: a row of
 // a streaming-GEMM expert, not written).  One thread per (row, chunk), rows
 // fastest: 8 consecutive rows fill 128 contiguous bytes of each plane.
-__global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm,
-                         int k_div, int rows, const int32_t* __restrict__ plane_row, int plane_rows,
-                         uint8_t* __restrict__ planes, int32_t* flag) {
+__global__ void __launch_bounds__(256)
+    k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm, int k_div, int rows,
+             const int32_t* __restrict__ plane_row, int plane_rows, uint8_t* __restrict__ planes,
+             int32_t* flag) {
+    __shared__ uint16_t lut[256];  // byte of q -> digit_codes(q)
+    for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
+    __syncthreads();
     const int nc = K / 32;
     const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (id >= (long long)rows * nc) return;
@@ -484,23 +488,14 @@ __global__ void k_planes(const int8_t* __restrict__ src, int K, const int32_t* _
     const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
     const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    // E2M1 code of a digit d in [-4, 3]: magnitudes 0, 1, 2, 3, 4 are the codes
-    // 0, 2, 4, 5, 6 (nibbles packed in 0x65420), the sign is bit 3
-    auto code = [](int d) -> uint32_t {
-        const uint32_t mag = (0x65420u >> (4 * (d < 0 ? -d : d))) & 0xFu;
-        return d < 0 ? (8u | mag) : mag;
-    };
     uint32_t out[3][4] = {};
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
-        const int qv = (int)(int8_t)(w[e >> 2] >> (8 * (e & 3)));
-        const int c0 = ((qv + 4) & 7) - 4;          // least significant digit
-        const int q1 = (qv - c0) >> 3;
-        const int b0 = ((q1 + 4) & 7) - 4;
-        const int a0 = (q1 - b0) >> 3;              // in [-2, 2]
-        out[0][e >> 3] |= code(a0) << (4 * (e & 7));
-        out[1][e >> 3] |= code(b0) << (4 * (e & 7));
-        out[2][e >> 3] |= code(c0) << (4 * (e & 7));
+        const uint32_t t = lut[(w[e >> 2] >> (8 * (e & 3))) & 0xFFu];
+        const int sh = 4 * (e & 7);
+        out[0][e >> 3] |= (t & 0xFu) << sh;
+        out[1][e >> 3] |= ((t >> 4) & 0xFu) << sh;
+        out[2][e >> 3] |= (t >> 8) << sh;
     }
     const int g = c >> 2, cc = c & 3;
     uint8_t* dst = planes + ((size_t)g * (plane_rows / 8) + (pr >> 3)) * kPlaneGroupBytes + cc * 128 +
