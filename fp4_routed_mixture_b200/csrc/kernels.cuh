@@ -9,9 +9,9 @@
 namespace moe {
 
 // Tile of the tensor-core grouped GEMM: 128 weight rows (the MMA's M) by up to
-// 112 sorted token rows (its N); shared by the planner and the kernel.
+// 128 sorted token rows (its N); shared by the planner and the kernel.
 constexpr int kTcWeightTile = 128;
-constexpr int kTcTokenTile = 112;
+constexpr int kTcTokenTile = 128;
 
 // Number of kernels this library has launched in the process (diagnostics).
 void count_launches(int n);

@@ -25,24 +25,28 @@
 //       the same exact sum the CUDA-core kernel forms (every product is an
 //       integer multiple of the row's smallest weight scale).
 //
-// Two persistent CTAs per SM, each warp-specialised:
-//   warp 0      producer: two bulk copies per stage (A chunk, B planes) into
-//               a 3-stage ring (mbarrier transaction counts);
-//   warp 1      MMA issuer: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs per
-//               stage, tcgen05.commit frees the stage / publishes the tile;
-//   warps 2..9  epilogue: TMEM -> registers (tcgen05.ld), one thread per
-//               weight row and half of the columns; W1 applies the token scale
-//               and SwiGLU (gate and up rows share a warp) and writes h, W2
-//               writes the final fp32 Y; two accumulator buffers in TMEM let
-//               the epilogue overlap the next tile's MMAs.
-// Why two CTAs: the tensor core queues only a few MMAs, and an issuing thread
-// that waits on an mbarrier (a shared-memory operation, ordered behind its
-// queued MMAs) stalls for about as long as that queue lasts at N <= 128, so
-// one issuer leaves the pipe idle about half the time.  Two independent
-// issuers per SM fill each other's gaps (measured: 62-65 clocks per
-// 128 x 112..128 x 64 MMA per SM against 56-64 ideal, versus ~125 with one).
-// Each CTA owns half of the SM's TMEM (256 columns): two 112-column
-// accumulators plus the scale factors.
+// One persistent CTA per SM, warp-specialised, with two independent pipes
+// that take alternate tiles of the CTA's share:
+//   warps 0, 1   producers: two bulk copies per stage (A chunk, B planes)
+//                into the pipe's own 3-stage ring (mbarrier transaction
+//                counts);
+//   warps 2, 3   MMA issuers: scale factors to TMEM (tcgen05.cp), 2 x 3 MMAs
+//                per stage, tcgen05.commit frees the stage / publishes the
+//                tile;
+//   warps 4..19  epilogue, one per (TMEM lane quadrant, 32-column chunk),
+//                tiles in order: TMEM -> registers (tcgen05.ld), one thread
+//                per weight row; W1 applies the token scale and SwiGLU (gate
+//                and up rows share a warp) and writes h, W2 writes the final
+//                fp32 Y.
+// Three 128-column accumulators in TMEM, tile j in buffer j % 3: two tiles
+// take MMAs while the epilogue drains the third.  Why two issuers: the tensor
+// core queues only a few MMAs, and a thread that waits on an mbarrier (a
+// shared-memory operation, ordered behind its own queued MMAs) stalls for
+// about as long as that queue lasts at N <= 128, so one issuer leaves the pipe
+// idle about half the time; two fill each other's gaps (measured 62-65 clocks
+// per 128 x 112..128 x 64 MMA per SM against 56-64 ideal, ~125 with one).  Why
+// 128-row token tiles: an MMA with N below 128 costs about as much as one
+// with N = 128, so fewer, fuller tiles win.
 // Every wait is bounded in time; a wait that gives up raises FLAG_TIMEOUT and
 // the roles wind down (copies in flight are waited for, TMEM is freed).
 #include "kernels.cuh"
@@ -52,25 +56,31 @@ namespace moe {
 
 constexpr int TC_BM = kTcWeightTile;           // weight rows per tile (MMA M)
 constexpr int TC_BN = kTcTokenTile;            // token rows per tile (largest MMA N used)
-constexpr int TC_STAGES = 3;
+constexpr int TC_PIPES = 2;                    // producer + MMA-issuer pairs, alternating tiles
+constexpr int TC_STAGES = 3;                   // ring stages per pipe
+constexpr int TC_ACC = 3;                      // accumulator buffers shared by the pipes
 constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
 constexpr int TC_B_BYTES = TC_BN / 8 * kPlaneGroupBytes;  // 3 planes x TC_BN rows x 128 inputs
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
-constexpr int TC_EPI_WARPS = 8;                // two per TMEM lane quadrant
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
-constexpr int TC_CTAS_PER_SM = 2;
-constexpr int TC_TMEM_COLS = 512 / TC_CTAS_PER_SM;   // the two CTAs of an SM split its TMEM
-constexpr int TC_SFA_COL = 2 * TC_BN;          // after two accumulator buffers; 4 columns per stage
-constexpr int TC_SFB_COL = TC_SFA_COL + 4 * TC_STAGES;  // 4 columns per plane
-static_assert(TC_SFB_COL + 12 <= TC_TMEM_COLS, "accumulators and scale factors exceed the TMEM share");
-static_assert(TC_SFA_COL % 4 == 0 && TC_SFB_COL % 4 == 0, "scale-factor columns hold 4 bytes per lane");
-static_assert(TC_BN % 16 == 0 && TC_BN <= 256, "MMA N");
+constexpr int TC_CHUNKS = TC_BN / 32;          // 32-column chunks of a tile
+constexpr int TC_EPI_WARPS = 4 * TC_CHUNKS;    // one per (TMEM lane quadrant, column chunk)
+constexpr int TC_EPI_WARP0 = 2 * TC_PIPES;     // warps 0..: producers, then MMA issuers
+constexpr int TC_THREADS = 32 * (TC_EPI_WARP0 + TC_EPI_WARPS);
+constexpr int TC_TMEM_COLS = 512;
+// TMEM columns: accumulator b at b * TC_BN; then per pipe r, at TC_SF_COL + 24r,
+// the A scale factors (4 columns per stage) and the three constant B plane
+// scales (4 columns each).
+constexpr int TC_SF_COL = TC_ACC * TC_BN;
+constexpr int TC_SF_PIPE_COLS = 4 * TC_STAGES + 12;
+static_assert(TC_SF_COL + TC_PIPES * TC_SF_PIPE_COLS <= TC_TMEM_COLS, "accumulators and scale factors exceed TMEM");
+static_assert(TC_SF_COL % 4 == 0 && TC_SF_PIPE_COLS % 4 == 0, "scale-factor columns hold 4 bytes per lane");
+static_assert(TC_BN % 32 == 0 && TC_BN <= 256, "MMA N, whole column chunks");
 
 struct TcShared {
-    uint8_t stage[TC_STAGES][TC_STAGE_BYTES];
-    uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once
-    float col_scale[TC_EPI_WARPS][TC_BN];  // per epilogue warp: activation scale of each tile column
-    uint64_t full[TC_STAGES], empty[TC_STAGES], acc_full[2], acc_empty[2];
+    uint8_t stage[TC_PIPES][TC_STAGES][TC_STAGE_BYTES];
+    uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once per pipe
+    float col_scale[TC_EPI_WARPS][32];  // per epilogue warp: activation scale of its 32 columns
+    uint64_t full[TC_PIPES][TC_STAGES], empty[TC_PIPES][TC_STAGES], acc_full[TC_ACC], acc_empty[TC_ACC];
     uint32_t tmem_base;
     int32_t abort;
 };
@@ -235,7 +245,7 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     return tt;
 }
 
-__global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -243,14 +253,18 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
     const int total = __ldg(a.tile_off + a.E);
     if (*(volatile int32_t*)a.flag & FLAG_LAYOUT) return;
     if (total == 0) return;
+    // this CTA's tiles: t_j = blockIdx.x + j * gridDim.x, j < ntiles; tile j
+    // belongs to pipe j % TC_PIPES and accumulator j % TC_ACC
+    const int ntiles = (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
     // ---- set-up: barriers, constant plane scales, TMEM ----
     if (threadIdx.x == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
-            mbar_init(smem_u32(&sh.full[s]), 1);
-            mbar_init(smem_u32(&sh.empty[s]), 1);
-        }
-        for (int b = 0; b < 2; ++b) {
+        for (int r = 0; r < TC_PIPES; ++r)
+            for (int s = 0; s < TC_STAGES; ++s) {
+                mbar_init(smem_u32(&sh.full[r][s]), 1);
+                mbar_init(smem_u32(&sh.empty[r][s]), 1);
+            }
+        for (int b = 0; b < TC_ACC; ++b) {
             mbar_init(smem_u32(&sh.acc_full[b]), 1);
             mbar_init(smem_u32(&sh.acc_empty[b]), TC_EPI_WARPS);
         }
@@ -277,14 +291,15 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
         raise_flag(a.flag, FLAG_TIMEOUT);
     };
 
-    if (warp == 0) {
-        // ---------------- producer ----------------
+    if (warp < TC_PIPES) {
+        // ---------------- producer of pipe r ----------------
+        const int r = warp;
         int stage = 0;
         uint32_t phase = 0;
         bool filled[TC_STAGES] = {};
         uint32_t fill_parity[TC_STAGES] = {};
-        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-            const TcTile tt = tile_at(a, t);
+        for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
+            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
             const uint8_t* wsrc = a.w + (size_t)tt.e * a.expert_bytes + (size_t)tt.rb * KG * TC_A_BYTES;
             const uint32_t bbytes = (uint32_t)(tt.n_mma / 8) * kPlaneGroupBytes;  // B of one stage
             // the tile's rows must lie inside the plane buffer (a plane_off
@@ -292,12 +307,12 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
             const bool rows_ok = tt.pr0 >= 0 && (tt.pr0 & 15) == 0 && tt.pr0 + tt.n_mma <= a.plane_rows;
             if (!rows_ok && lane == 0) raise_flag(a.flag, FLAG_BOUNDS);
             for (int g = 0; g < KG; ++g) {
-                const uint32_t fb = smem_u32(&sh.full[stage]), eb = smem_u32(&sh.empty[stage]);
+                const uint32_t fb = smem_u32(&sh.full[r][stage]), eb = smem_u32(&sh.empty[r][stage]);
                 if (!mbar_wait(eb, phase ^ 1u, abort)) {
                     give_up();
                     break;
                 }
-                const uint32_t sbase = smem_u32(sh.stage[stage]);
+                const uint32_t sbase = smem_u32(sh.stage[r][stage]);
                 if (lane == 0) {
                     if (rows_ok) {
                         mbar_expect_tx(fb, TC_A_BYTES + bbytes);
@@ -321,21 +336,24 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
         // let every copy this warp issued land before the CTA can exit (on the
         // normal path the MMA warp has already waited for all of them)
         for (int s = 0; s < TC_STAGES; ++s)
-            if (filled[s]) mbar_wait_bounded(smem_u32(&sh.full[s]), fill_parity[s]);
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+            if (filled[s]) mbar_wait_bounded(smem_u32(&sh.full[r][s]), fill_parity[s]);
+    } else if (warp < TC_EPI_WARP0) {
+        // ---------------- MMA issuer of pipe r ----------------
+        const int r = warp - TC_PIPES;
+        const uint32_t sfa_col = tmem + TC_SF_COL + TC_SF_PIPE_COLS * r;
+        const uint32_t sfb_col = sfa_col + 4 * TC_STAGES;
         if (lane == 0) {
             for (int p = 0; p < 3; ++p)
-                tc_cp_sf(tmem + TC_SFB_COL + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
+                tc_cp_sf(sfb_col + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
         }
         __syncwarp();
         int stage = 0;
         uint32_t phase = 0;
-        int buf = 0;
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-            const TcTile tt = tile_at(a, t);
-            if (!mbar_wait(smem_u32(&sh.acc_empty[buf]), acc_phase ^ 1u, abort)) {
+        for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
+            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
+            const int buf = j % TC_ACC;
+            const uint32_t use = (uint32_t)(j / TC_ACC);
+            if (!mbar_wait(smem_u32(&sh.acc_empty[buf]), (use & 1u) ^ 1u, abort)) {
                 give_up();
                 break;
             }
@@ -343,15 +361,15 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
             const uint32_t dcol = tmem + buf * TC_BN;
             bool ok = true;
             for (int g = 0; g < KG; ++g) {
-                if (!mbar_wait(smem_u32(&sh.full[stage]), phase, abort)) {
+                if (!mbar_wait(smem_u32(&sh.full[r][stage]), phase, abort)) {
                     give_up();
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t sbase = smem_u32(sh.stage[stage]);
-                    const uint32_t sfa = tmem + TC_SFA_COL + 4 * stage;
+                    const uint32_t sbase = smem_u32(sh.stage[r][stage]);
+                    const uint32_t sfa = sfa_col + 4 * stage;
                     tc_cp_sf(sfa, make_sdesc(sbase, 0, 128));
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
@@ -363,11 +381,10 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
                             const uint64_t bdesc = make_sdesc(sbase + TC_A_BYTES + p * 512 + ks * 256, 128,
                                                               kPlaneGroupBytes);
                             const uint32_t idesc = make_idesc(tt.n_mma, 2 * ks, 0);
-                            tc_mma_mxf4(dcol, adesc, bdesc, idesc, sfa,
-                                        tmem + TC_SFB_COL + 4 * p, (g | ks | p) != 0);
+                            tc_mma_mxf4(dcol, adesc, bdesc, idesc, sfa, sfb_col + 4 * p, (g | ks | p) != 0);
                         }
                     }
-                    tc_commit(smem_u32(&sh.empty[stage]));
+                    tc_commit(smem_u32(&sh.empty[r][stage]));
                 }
                 __syncwarp();
                 if (++stage == TC_STAGES) {
@@ -378,77 +395,70 @@ __global__ void __launch_bounds__(TC_THREADS, TC_CTAS_PER_SM) k_tc_gemm(TcArgs a
             if (!ok) break;
             if (lane == 0) tc_commit(smem_u32(&sh.acc_full[buf]));
             __syncwarp();
-            if (++buf == 2) {
-                buf = 0;
-                acc_phase ^= 1u;
-            }
         }
     } else {
-        // ---------------- epilogue (warps 2..9) ----------------
-        // Two warps per TMEM lane quadrant; warp half h takes the 32-column
-        // chunks h, h+2, ... of the tile.  Each warp first stages the
-        // activation scale of every tile column in its own shared-memory slice
-        // (no cross-warp waits).  Scaling: the accumulator is an fp32 value,
-        // so fp32(fp64(s) * fp64(acc)) -- the definition -- equals the single
-        // correctly rounded fp32 product s * acc (the exact product of two
-        // 24-bit significands fits in fp64).
+        // ---------------- epilogue (warps TC_EPI_WARP0 ..) ----------------
+        // Warp (q, c) owns the 32 weight rows of TMEM lane quadrant q and the
+        // 32-column chunk c of every tile, tiles in this CTA's order.  It first
+        // stages the activation scale of its columns in its own shared-memory
+        // slice (no cross-warp waits).  Scaling: the accumulator is an fp32
+        // value, so fp32(fp64(s) * fp64(acc)) -- the definition -- equals the
+        // single correctly rounded fp32 product s * acc (the exact product of
+        // two 24-bit significands fits in fp64).
         // W1: lanes 0-15 of a warp hold the gate rows and lanes 16-31 the up
         // rows of the same 16 outputs (row interleave of pack.cu).  Columns go
         // in pairs: lanes 0-15 form h for column j (up value shuffled down),
         // lanes 16-31 for column j+1 (gate value shuffled up), h = SwiGLU(g, u),
         // stored in fp32 (the row maximum of |h| is taken when h is
         // requantised).  W2: Y = s * acc straight out.
-        const int ew = warp - 2;
+        const int ew = warp - TC_EPI_WARP0;
         const int q = warp & 3;            // TMEM lane quadrant this warp may access
-        const int half = ew >> 2;          // which alternate 32-column chunks
+        const int n0 = 32 * (ew >> 2);     // this warp's column chunk
         const int m = q * 32 + lane;       // weight row within the tile
         const bool w1 = a.gate_up_half > 0;
         float* csc = sh.col_scale[ew];
-        int buf = 0;
-        uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-            const TcTile tt = tile_at(a, t);
-            for (int n = lane; n < tt.n_mma; n += 32) {
-                const int i = min(tt.i0 + n, tt.i0 + tt.n_valid - 1);
+        for (int j = 0; j < ntiles && !*abort; ++j) {
+            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
+            const int buf = j % TC_ACC;
+            const uint32_t use = (uint32_t)(j / TC_ACC);
+            const bool mine = n0 < tt.n_mma;
+            if (mine) {
+                const int i = min(tt.i0 + n0 + lane, tt.i0 + tt.n_valid - 1);
                 const int src = a.k_div > 0 ? checked_index(__ldg(a.perm + i), a.P, a.flag) / a.k_div : i;
-                csc[n] = __ldg(a.row_scale + src);
+                csc[lane] = __ldg(a.row_scale + src);
             }
             __syncwarp();
-            if (!mbar_wait(smem_u32(&sh.acc_full[buf]), acc_phase, abort)) {
+            if (!mbar_wait(smem_u32(&sh.acc_full[buf]), use & 1u, abort)) {
                 give_up();
                 break;
             }
             tc_fence_after();
-            for (int n0 = 32 * half; n0 < tt.n_mma; n0 += 64) {
-                uint32_t r[32];
-                tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * TC_BN + n0, r);
+            if (mine) {
+                uint32_t v[32];
+                tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * TC_BN + n0, v);
                 if (!w1) {
                     float* out = a.out + (size_t)(tt.i0 + n0) * a.N + tt.rb * TC_BM + m;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (n0 + j < tt.n_valid) out[(size_t)j * a.N] = __fmul_rn(csc[n0 + j], __uint_as_float(r[j]));
+                    for (int c = 0; c < 32; ++c)
+                        if (n0 + c < tt.n_valid) out[(size_t)c * a.N] = __fmul_rn(csc[c], __uint_as_float(v[c]));
                 } else {
                     const int I = a.gate_up_half;
                     const bool lo = lane < 16;
                     float* out = a.out + (size_t)(tt.i0 + n0) * I + (tt.rb * 4 + q) * 16 + (lane & 15);
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const float v0 = __fmul_rn(csc[n0 + j], __uint_as_float(r[j]));
-                        const float v1 = __fmul_rn(csc[n0 + j + 1], __uint_as_float(r[j + 1]));
-                        const float from_hi = __shfl_down_sync(0xffffffffu, v0, 16);  // up value, column j
-                        const float from_lo = __shfl_up_sync(0xffffffffu, v1, 16);    // gate value, column j+1
+                    for (int c = 0; c < 32; c += 2) {
+                        const float v0 = __fmul_rn(csc[c], __uint_as_float(v[c]));
+                        const float v1 = __fmul_rn(csc[c + 1], __uint_as_float(v[c + 1]));
+                        const float from_hi = __shfl_down_sync(0xffffffffu, v0, 16);  // up value, column c
+                        const float from_lo = __shfl_up_sync(0xffffffffu, v1, 16);    // gate value, column c+1
                         const float hv = lo ? swiglu(v0, from_hi) : swiglu(from_lo, v1);
-                        if (n0 + j + (lo ? 0 : 1) < tt.n_valid) out[(size_t)(j + (lo ? 0 : 1)) * I] = hv;
+                        if (n0 + c + (lo ? 0 : 1) < tt.n_valid) out[(size_t)(c + (lo ? 0 : 1)) * I] = hv;
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[buf]));
-            if (++buf == 2) {
-                buf = 0;
-                acc_phase ^= 1u;
-            }
         }
     }
 
@@ -512,7 +522,7 @@ static int tc_grid() {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaFuncSetAttribute(k_tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
-        grid = sms * TC_CTAS_PER_SM;
+        grid = sms;  // one CTA per SM: it allocates all of the SM's TMEM
     }
     return grid;
 }
