@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import subprocess
@@ -152,18 +153,23 @@ def measured_peaks() -> dict:
             "source": "fallback"}
 
 
-def profiled_traffic(kernel_file: str, workload: str):
-    """DRAM bytes per launch of the streaming GEMM from a committed ncu summary,
-    valid only while the kernel source is unchanged since the capture."""
-    p = os.path.join(ROOT, "profiles", f"gemv_{workload}_traffic.json")
-    src = os.path.join(ROOT, "fp4_routed_mixture_b200", "csrc", kernel_file)
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch (read + write) of a GEMM kernel, from a committed ncu
+    summary under profiles/; None unless the kernel source is unchanged since the
+    capture (the summary records the source file and its SHA-256)."""
+    p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    if d.get("kernel_sha256") != h:
+    text = open(p).read()
+    src = re.search(r"^\s*kernel_source:\s*(\S+)", text, re.M)
+    sha = re.search(r"^\s*kernel_source_sha256:\s*([0-9a-f]{64})", text, re.M)
+    val = re.search(r"^\s*dram_bytes_per_launch:\s*(\d+)", text, re.M)
+    if not (src and sha and val):
         return None
-    return d.get("dram_bytes_per_launch")
+    path = os.path.join(ROOT, src.group(1))
+    if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest() != sha.group(1):
+        return None
+    return int(val.group(1))
 
 
 # ---------------------------------------------------------------------------------------
@@ -349,7 +355,7 @@ def main():
                    "touched_experts": r["touched"],
                    "l2": "inputs larger than L2: %.2f GB of expert weights streamed per step "
                          "vs 126 MB L2" % (r["alg_bytes_step"] / 1e9)},
-        "roofline": roofline_hbm(r, peaks, profiled_traffic("gemv.cu", w.name)),
+        "roofline": roofline_hbm(r, peaks, profiled_traffic(f"k_gemv_{w.name}.md")),
         "e2e": {"value": round(N * w.T * steps / (r["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
@@ -376,7 +382,8 @@ def main():
                          "mma_issued_tflops": round(3 * ptf, 2),
                          "mma_peak_fp4": 4.0 * peaks["bf16_tflops"],
                          "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
-                         "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1)},
+                         "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
+                         "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
         }
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)
