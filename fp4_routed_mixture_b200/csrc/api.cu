@@ -217,9 +217,10 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws_bytes %zu < %zu", ws_bytes, L.total);
     char* w = (char*)ws;
     int32_t* flag = (int32_t*)(w + L.flag);
-    cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int32_t), stream);
-    if (e != cudaSuccess) return cuda_fail(e, "moe_forward memset");
-    if (d->T == 0) return MOE_OK;
+    if (d->T == 0) {  // no kernel runs; otherwise the first kernel clears the word
+        cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int32_t), stream);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_forward memset");
+    }
 
     const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k, P = T * k;
     const moe::PackedLayout PL = moe::packed_layout(H, I, E);

@@ -18,6 +18,7 @@ __global__ void __launch_bounds__(256)
               const float* __restrict__ sh, const float* __restrict__ gates,
               const int32_t* __restrict__ pos, int P, int k, int E, int H, uint2* __restrict__ y,
               int32_t* flag) {
+    pdl_begin();
     const int t = blockIdx.y;
     const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
     if (4 * n4 >= H) return;
@@ -57,10 +58,10 @@ cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* e
                            cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     dim3 grid((H / 4 + 255) / 256, T);
-    k_combine<<<grid, 256, 0, st>>>(yacc, yf, expert_tc, topk_idx, sh, gates, pos, T * k, k, E, H,
-                                    (uint2*)y, flag);
+    const cudaError_t e = launch_pdl(k_combine, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates,
+                                     pos, T * k, k, E, H, (uint2*)y, flag);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

@@ -195,6 +195,7 @@ __device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, 
 }
 
 __global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
+    pdl_begin();
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // packed weights built for other dims may be smaller than the offsets used here
@@ -347,9 +348,9 @@ cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, con
                         const int32_t* flag, int gate_up_half, int P, cudaStream_t st) {
     GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
                gate_up_half, P, 0u};
-    k_gemv<<<gemv_grid(), kGemvWarps * 32, kSmemBytes, st>>>(a);
+    const cudaError_t e = launch_pdl(k_gemv, dim3(gemv_grid()), dim3(kGemvWarps * 32), kSmemBytes, st, a);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

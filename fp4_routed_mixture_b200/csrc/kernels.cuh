@@ -18,6 +18,27 @@ constexpr int kTcTokenTile = 128;
 // Number of kernels this library has launched in the process (diagnostics).
 void count_launches(int n);
 
+// Launch with programmatic dependent launch allowed: the kernel may be
+// scheduled before the preceding kernel in the stream completes.  Every kernel
+// launched this way starts with pdl_begin() (moe_common.cuh), which waits for
+// that kernel (and so, transitively, for every earlier one) before touching
+// memory.  This hides the launch gap between the layer's short kernels.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct PackedLayout {
     size_t header, w1, w1_expert_bytes, w2, w2_expert_bytes, total;
 };

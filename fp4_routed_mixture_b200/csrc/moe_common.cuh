@@ -82,6 +82,16 @@ __device__ __forceinline__ int quant_code(float v, float amax, float s) {
     return (int)r;
 }
 
+// First statement of every kernel launched with launch_pdl: wait until the
+// preceding kernel in the stream has completed and its writes are visible,
+// then allow the next kernel to be scheduled (it waits in turn, so at most two
+// grids overlap and the later one only waits).  Both are no-ops for a launch
+// without the attribute.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // E2M1 codes of the three balanced base-8 digits of an INT8 code q =
 // 64*a + 8*b + c (a in [-2, 2], b and c in [-4, 3]): a | b << 4 | c << 8.  A
 // digit d has code 0, 2, 4, 5, 6 for |d| = 0..4 (nibbles packed in 0x65420)

@@ -105,11 +105,13 @@ __global__ void k_write_header(PackHeader* h, int H, int I, int E, uint64_t w1_o
     h->flag = 0;
 }
 
-// Raises FLAG_LAYOUT when the packed buffer was built for other dims.
+// First kernel of moe_forward (one thread): clears the call's device error word
+// and sets FLAG_LAYOUT when the packed buffer was built for other dims.
 __global__ void k_check_header(const PackHeader* h, int H, int I, int E, int32_t* flag) {
-    if (h->magic != kPackMagic || h->version != kPackVersion || (int)h->H != H ||
-        (int)h->I != I || (int)h->E != E)
-        raise_flag(flag, FLAG_LAYOUT);
+    pdl_begin();
+    const bool bad = h->magic != kPackMagic || h->version != kPackVersion || (int)h->H != H ||
+                     (int)h->I != I || (int)h->E != E;
+    *flag = bad ? FLAG_LAYOUT : 0;
 }
 
 PackedLayout packed_layout(int H, int I, int E) {
@@ -163,9 +165,10 @@ const int32_t* packed_flag_ptr(const void* packed) {
 
 cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t* flag,
                                 cudaStream_t st) {
-    k_check_header<<<1, 1, 0, st>>>((const PackHeader*)packed, H, I, E, flag);
+    const cudaError_t e = launch_pdl(k_check_header, dim3(1), dim3(1), 0, st, (const PackHeader*)packed, H, I, E,
+                                     flag);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

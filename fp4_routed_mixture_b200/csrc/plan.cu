@@ -22,6 +22,7 @@ __global__ void k_plan(const int32_t* __restrict__ offsets, int E, int P, int n1
                        int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                        int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                        int32_t* __restrict__ plane_off, int32_t* __restrict__ expert_tc, int32_t* flag) {
+    pdl_begin();
     constexpr int NS = 5;
     const int lane = threadIdx.x;
     const int per = (E + 31) / 32;
@@ -78,10 +79,10 @@ __global__ void k_plan(const int32_t* __restrict__ offsets, int E, int P, int n1
 cudaError_t launch_plan(const int32_t* offsets, int E, int P, int n1, int n2, int tc_min,
                         int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2,
                         int32_t* plane_off, int32_t* expert_tc, int32_t* flag, cudaStream_t st) {
-    k_plan<<<1, 32, 0, st>>>(offsets, E, P, n1, n2, tc_min, unit_off1, unit_off2, tile_off1, tile_off2,
-                             plane_off, expert_tc, flag);
+    const cudaError_t e = launch_pdl(k_plan, dim3(1), dim3(32), 0, st, offsets, E, P, n1, n2, tc_min, unit_off1,
+                                     unit_off2, tile_off1, tile_off2, plane_off, expert_tc, flag);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

@@ -40,6 +40,7 @@ __global__ void __launch_bounds__(kQThreads)
     k_xquant(const __nv_bfloat16* __restrict__ x, int T, int H, int8_t* __restrict__ xq,
              float* __restrict__ sx, int32_t* __restrict__ xinit, int8_t* __restrict__ dbg_xq,
              float* __restrict__ dbg_sx) {
+    pdl_begin();
     __shared__ float red[33];
     const int t = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kQThreads)
              int P, int k, int E, int I, int8_t* __restrict__ hq, float* __restrict__ sh,
              int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh,
              int32_t* flag) {
+    pdl_begin();
     static_assert(R == 32 || R == kQThreads, "a warp or a CTA per row");
     __shared__ uint16_t lut[256];
     __shared__ float red[33];
@@ -214,6 +216,7 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ plane_off, int P, int E, int I, int H,
                    int32_t* __restrict__ plane_row,
                    double* __restrict__ gacc, double* __restrict__ yacc, int32_t* flag) {
+    pdl_begin();
     for (int i = blockIdx.x; i < P; i += gridDim.x) {
         const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
         const bool tc = expert_tc[e] != 0;
@@ -282,9 +285,10 @@ cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, c
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
                           int8_t* dbg_xq, float* dbg_sx, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    k_xquant<<<T, kQThreads, 0, st>>>((const __nv_bfloat16*)x, T, H, xq, sx, xinit, dbg_xq, dbg_sx);
+    const cudaError_t e = launch_pdl(k_xquant, dim3(T), dim3(kQThreads), 0, st, (const __nv_bfloat16*)x, T, H,
+                                     xq, sx, xinit, dbg_xq, dbg_sx);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
@@ -295,19 +299,19 @@ cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert
     if (P == 0) return cudaSuccess;
     // few rows (decode): a CTA per row keeps every row's chain short; many
     // rows (prefill): a warp per row needs no block barriers
+    cudaError_t e;
     if (P < 4096 && I % (4 * kQThreads) == 0) {
-        k_hquant<kQThreads><<<std::min(P, 148 * 8), kQThreads, 0, st>>>(
-            gacc, hbuf, expert_tc, topk_idx, sx, perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh,
-            hinit, dbg_hq, dbg_sh, flag);
+        e = launch_pdl(k_hquant<kQThreads>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf,
+                       expert_tc, topk_idx, sx, perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit,
+                       dbg_hq, dbg_sh, flag);
     } else {
         const int warps = kQThreads / 32;
         const int grid = std::min((P + warps - 1) / warps, 148 * 8);
-        k_hquant<32><<<grid, kQThreads, 0, st>>>(gacc, hbuf, expert_tc, topk_idx, sx, perm, plane_row,
-                                                 plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq,
-                                                 dbg_sh, flag);
+        e = launch_pdl(k_hquant<32>, dim3(grid), dim3(kQThreads), 0, st, gacc, hbuf, expert_tc, topk_idx, sx, perm,
+                       plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq, dbg_sh, flag);
     }
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
@@ -315,10 +319,10 @@ cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_id
                                 int H, int32_t* plane_row, double* gacc, double* yacc,
                                 int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
-    k_prepare_rows<<<std::min(P, 148 * 8), 256, 0, st>>>(expert_tc, topk_idx, perm, offsets, plane_off, P, E,
-                                                          I, H, plane_row, gacc, yacc, flag);
+    const cudaError_t e = launch_pdl(k_prepare_rows, dim3(std::min(P, 148 * 8)), dim3(256), 0, st, expert_tc,
+                                     topk_idx, perm, offsets, plane_off, P, E, I, H, plane_row, gacc, yacc, flag);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,

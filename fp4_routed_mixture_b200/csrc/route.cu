@@ -23,6 +23,7 @@ template <int KMAX>
 __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits, int T, int E, int k,
                                                int32_t* __restrict__ topk_idx,
                                                float* __restrict__ gates) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -88,12 +89,11 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
     if (T == 0) return cudaSuccess;
     const int warps = 8;
     dim3 grid((T + warps - 1) / warps);
-    if (k <= 8)
-        k_route<8><<<grid, warps * 32, 0, st>>>(logits, T, E, k, topk_idx, gates);
-    else
-        k_route<16><<<grid, warps * 32, 0, st>>>(logits, T, E, k, topk_idx, gates);
+    const cudaError_t e =
+        k <= 8 ? launch_pdl(k_route<8>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates)
+               : launch_pdl(k_route<16>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

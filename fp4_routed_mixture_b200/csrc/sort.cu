@@ -89,6 +89,7 @@ __device__ void warp_stable_scatter(const int32_t* __restrict__ topk_idx, int p0
 __global__ void __launch_bounds__(kSortThreads)
     k_sort_count(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ chunk_hist,
                  int32_t* flag) {
+    pdl_begin();
     extern __shared__ int hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(kSortThreads)
     k_sort_scatter(const int32_t* __restrict__ topk_idx, int P, int E,
                    const int32_t* __restrict__ chunk_hist, int32_t* __restrict__ perm,
                    int32_t* __restrict__ pos, int32_t* __restrict__ offsets) {
+    pdl_begin();
     extern __shared__ int sm[];
     int* total = sm;           // [E] -> exclusive offsets
     int* cursor = sm + E;      // [E]
@@ -143,9 +145,11 @@ __global__ void __launch_bounds__(kSortThreads)
 __global__ void __launch_bounds__(kSortThreads)
     k_sort_single(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ perm,
                   int32_t* __restrict__ pos, int32_t* __restrict__ offsets, int32_t* flag) {
+    pdl_begin();
     extern __shared__ int sm[];
     int* hist = sm;
     int* tmp = sm + E;
+    if (threadIdx.x == 0) *flag = 0;  // this single CTA is the whole sort: it owns the error word
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
     __syncthreads();
     bool bad = false;
@@ -176,25 +180,25 @@ cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* p
     int32_t* flag = (int32_t*)ws;
     int32_t* chunk_hist = (int32_t*)((char*)ws + 256);
     const int P = T * k;
+    if (P <= kSortChunk) {  // k_sort_single clears the error word itself
+        const size_t smem = (size_t)(E + kSortThreads + 1) * sizeof(int);
+        const cudaError_t e = launch_pdl(k_sort_single, dim3(1), dim3(kSortThreads), smem, st, topk_idx, P, E,
+                                         perm, pos, offsets, flag);
+        count_launches(1);
+        return e;
+    }
     cudaError_t err = cudaMemsetAsync(flag, 0, sizeof(int32_t), st);
     if (err != cudaSuccess) return err;
-    if (P <= kSortChunk) {
-        const size_t smem = (size_t)(E + kSortThreads + 1) * sizeof(int);
-        k_sort_single<<<1, kSortThreads, smem, st>>>(topk_idx, P, E, perm, pos, offsets, flag);
-        count_launches(1);
-        return cudaGetLastError();
-    }
     const int chunks = (P + kSortChunk - 1) / kSortChunk;
-    k_sort_count<<<chunks, kSortThreads, (size_t)E * sizeof(int), st>>>(topk_idx, P, E, chunk_hist,
-                                                                        flag);
+    err = launch_pdl(k_sort_count, dim3(chunks), dim3(kSortThreads), (size_t)E * sizeof(int), st, topk_idx, P, E,
+                     chunk_hist, flag);
     count_launches(1);
-    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const size_t smem = (size_t)(2 * E + kSortThreads + 1) * sizeof(int);
-    k_sort_scatter<<<chunks, kSortThreads, smem, st>>>(topk_idx, P, E, chunk_hist, perm, pos,
-                                                       offsets);
+    err = launch_pdl(k_sort_scatter, dim3(chunks), dim3(kSortThreads), smem, st, topk_idx, P, E,
+                     (const int32_t*)chunk_hist, perm, pos, offsets);
     count_launches(1);
-    return cudaGetLastError();
+    return err;
 }
 
 // ---- the same sort with library-owned scratch (moe_sort_static) -------------

@@ -246,6 +246,7 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
+    pdl_begin();
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -481,6 +482,7 @@ __global__ void __launch_bounds__(256)
     k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm, int k_div, int rows,
              const int32_t* __restrict__ plane_row, int plane_rows, uint8_t* __restrict__ planes,
              int32_t* flag) {
+    pdl_begin();
     __shared__ uint16_t lut[256];  // byte of q -> digit_codes(q)
     for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
     __syncthreads();
@@ -534,10 +536,10 @@ cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_d
                           cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
     const long long n = (long long)rows * (K / 32);
-    k_planes<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, K, perm, k_div, rows, plane_row, plane_rows,
-                                                          planes, flag);
+    const cudaError_t e = launch_pdl(k_planes, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, src, K, perm,
+                                     k_div, rows, plane_row, plane_rows, planes, flag);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
@@ -547,9 +549,9 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            cudaStream_t st) {
     TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
              E, flag, row_scale, perm, k_div, out};
-    k_tc_gemm<<<tc_grid(), TC_THREADS, sizeof(TcShared), st>>>(a);
+    const cudaError_t e = launch_pdl(k_tc_gemm, dim3(tc_grid()), dim3(TC_THREADS), sizeof(TcShared), st, a);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe
