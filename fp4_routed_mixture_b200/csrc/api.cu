@@ -57,7 +57,7 @@ int check_dims(const moe_dims* d, bool need_T) {
 int g_tc_min_rows = 32;
 
 struct WsLayout {
-    size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xinit, hq, sh, hinit, px, ph,
+    size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xtp, xinit, hq, sh, hinit, px, ph,
         hbuf, yf, gacc, yacc, total;
     int plane_rows;
 };
@@ -77,6 +77,7 @@ WsLayout ws_layout(const moe_dims& d, long long T) {
     L.prow = o; o += align_up(4 * P, 256);
     L.sx = o; o += align_up(4 * (size_t)T, 256);
     L.xq = o; o += align_up((size_t)T * d.H, 256);
+    L.xtp = o; o += align_up((size_t)T * (d.H / 32) * 48, 256);   // x digit planes, token order
     L.xinit = o; o += align_up(4 * (size_t)T * (d.H / 32), 256);
     L.hq = o; o += align_up(P * d.I, 256);
     L.sh = o; o += align_up(4 * P, 256);
@@ -242,7 +243,11 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
         if (_e != cudaSuccess) return cuda_fail(_e, what); \
     } while (0)
     MOE_TRY(moe::launch_check_header(packed, H, I, E, flag, stream), "header check");
-    MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, dbg ? dbg->xq : nullptr,
+    // an expert has at most T rows, so the tensor-core path is skipped without
+    // reading any count when T < tc_min
+    const bool use_tc = T >= g_tc_min_rows;
+    uint8_t* xtp = (uint8_t*)(w + L.xtp);
+    MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
                                dbg ? dbg->sx : nullptr, stream), "x quant");
     int32_t* toff1 = (int32_t*)(w + L.toff1);
     int32_t* toff2 = (int32_t*)(w + L.toff2);
@@ -250,19 +255,16 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     uint8_t* ph = (uint8_t*)(w + L.ph);
     int32_t* poff = (int32_t*)(w + L.poff);
     int32_t* prow = (int32_t*)(w + L.prow);
-    // an expert has at most T rows, so the tensor-core path is skipped without
-    // reading any count when T < tc_min
-    const bool use_tc = T >= g_tc_min_rows;
     int32_t* etc = (int32_t*)(w + L.etc);
     float* hbuf = (float*)(w + L.hbuf);
     float* yf = (float*)(w + L.yf);
     MOE_TRY(moe::launch_plan(offsets, E, P, 2 * I, H, use_tc ? g_tc_min_rows : 0x7fffffff, uoff1, uoff2,
                              toff1, toff2, poff, etc, flag, stream), "plan");
-    MOE_TRY(moe::launch_prepare_rows(etc, topk_idx, perm, offsets, poff, P, E, I, H, prow, gacc, yacc,
+    MOE_TRY(moe::launch_prepare_rows(etc, topk_idx, perm, offsets, poff, uoff1, P, E, I, H, prow, gacc, yacc,
                                      flag, stream),
             "row state");
     if (use_tc)
-        MOE_TRY(moe::launch_planes(xq, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
+        MOE_TRY(moe::launch_planes(xtp, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,

@@ -11,7 +11,10 @@
 
 namespace moe {
 
-// One thread per 4 consecutive columns of one token (16-byte loads of Y).
+// One thread per 4 consecutive columns of one token (16-byte loads of Y).  The
+// k slots' row indices, gates and kernel choices are read first and all k rows
+// are then loaded before the sum, so the loads overlap.
+template <int KMAX>
 __global__ void __launch_bounds__(256)
     k_combine(const double* __restrict__ yacc, const float* __restrict__ yf,
               const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
@@ -22,29 +25,42 @@ __global__ void __launch_bounds__(256)
     const int t = blockIdx.y;
     const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
     if (4 * n4 >= H) return;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int j = 0; j < k; ++j) {
-        const int p = t * k + j;
-        const int i = checked_index(__ldg(pos + p), P, flag);
-        const float g = __ldg(gates + p);
-        float v[4];
-        if (__ldg(expert_tc + checked_index(__ldg(topk_idx + p), E, flag))) {
-            const float4 f = __ldg(reinterpret_cast<const float4*>(yf + (size_t)i * H) + n4);
-            v[0] = f.x;
-            v[1] = f.y;
-            v[2] = f.z;
-            v[3] = f.w;
-        } else {
-            const double s = (double)__ldg(sh + i);
-            const double2* r = reinterpret_cast<const double2*>(yacc + (size_t)i * H) + 2 * n4;
-            const double2 d0 = __ldg(r), d1 = __ldg(r + 1);
-            v[0] = (float)__dmul_rn(s, d0.x);
-            v[1] = (float)__dmul_rn(s, d0.y);
-            v[2] = (float)__dmul_rn(s, d1.x);
-            v[3] = (float)__dmul_rn(s, d1.y);
-        }
+    int row[KMAX];
+    float g[KMAX];
+    bool tc[KMAX];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(g, v[c], acc[c]);
+    for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+            const int p = t * k + j;
+            row[j] = checked_index(__ldg(pos + p), P, flag);
+            g[j] = __ldg(gates + p);
+            tc[j] = __ldg(expert_tc + checked_index(__ldg(topk_idx + p), E, flag)) != 0;
+        }
+    }
+    float4 v[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+            if (tc[j]) {
+                v[j] = __ldg(reinterpret_cast<const float4*>(yf + (size_t)row[j] * H) + n4);
+            } else {
+                const double s = (double)__ldg(sh + row[j]);
+                const double2* r = reinterpret_cast<const double2*>(yacc + (size_t)row[j] * H) + 2 * n4;
+                const double2 d0 = __ldg(r), d1 = __ldg(r + 1);
+                v[j] = make_float4((float)__dmul_rn(s, d0.x), (float)__dmul_rn(s, d0.y), (float)__dmul_rn(s, d1.x),
+                                   (float)__dmul_rn(s, d1.y));
+            }
+        }
+    }
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {  // slot order
+            acc[0] = __fmaf_rn(g[j], v[j].x, acc[0]);
+            acc[1] = __fmaf_rn(g[j], v[j].y, acc[1]);
+            acc[2] = __fmaf_rn(g[j], v[j].z, acc[2]);
+            acc[3] = __fmaf_rn(g[j], v[j].w, acc[3]);
+        }
     }
     const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
     const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
@@ -58,8 +74,11 @@ cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* e
                            cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     dim3 grid((H / 4 + 255) / 256, T);
-    const cudaError_t e = launch_pdl(k_combine, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates,
-                                     pos, T * k, k, E, H, (uint2*)y, flag);
+    const cudaError_t e =
+        k <= 8 ? launch_pdl(k_combine<8>, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates, pos, T * k,
+                            k, E, H, (uint2*)y, flag)
+               : launch_pdl(k_combine<16>, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates, pos,
+                            T * k, k, E, H, (uint2*)y, flag);
     count_launches(1);
     return e;
 }

@@ -64,15 +64,15 @@ cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t
                                 cudaStream_t st);
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
-                          int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
+                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
 cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
                           const int32_t* topk_idx, const float* sx, const int32_t* perm,
                           const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
                           int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
                           int32_t* flag, cudaStream_t st);
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                const int32_t* offsets, const int32_t* plane_off, int P, int E, int I,
-                                int H, int32_t* plane_row, double* gacc, double* yacc,
+                                const int32_t* offsets, const int32_t* plane_off, const int32_t* unit_off,
+                                int P, int E, int I, int H, int32_t* plane_row, double* gacc, double* yacc,
                                 int32_t* flag, cudaStream_t st);
 cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
@@ -95,7 +95,7 @@ constexpr int kPlaneGroupBytes = 1536;
 __host__ __device__ inline size_t plane_bytes(int K, int plane_rows) {
     return (size_t)(K / 128) * (plane_rows / 8) * kPlaneGroupBytes;
 }
-cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
+cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, int k_div, int rows,
                           const int32_t* plane_row, int plane_rows, uint8_t* planes, int32_t* flag,
                           cudaStream_t st);
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,

@@ -36,12 +36,20 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // One CTA per token; each thread handles chunks of 8 consecutive elements.
+// With tplanes != NULL the token's codes are also written once as E2M1 digit
+// planes in token order: per 32-input block b, 48 bytes at
+// tplanes + (t*(H/32) + b)*48: plane p's 16 bytes at +16p (element 2j of the
+// block in the low nibble of byte j).  The tensor-core GEMM's plane writer
+// copies these pieces into sorted-row order.
 __global__ void __launch_bounds__(kQThreads)
     k_xquant(const __nv_bfloat16* __restrict__ x, int T, int H, int8_t* __restrict__ xq,
-             float* __restrict__ sx, int32_t* __restrict__ xinit, int8_t* __restrict__ dbg_xq,
-             float* __restrict__ dbg_sx) {
+             float* __restrict__ sx, int32_t* __restrict__ xinit, uint8_t* __restrict__ tplanes,
+             int8_t* __restrict__ dbg_xq, float* __restrict__ dbg_sx) {
     pdl_begin();
     __shared__ float red[33];
+    __shared__ uint16_t lut[256];
+    if (tplanes)
+        for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
     const int t = blockIdx.x;
     const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * H);
     const int nchunk = H / 8;
@@ -81,6 +89,21 @@ __global__ void __launch_bounds__(kQThreads)
             const uint2 pv = make_uint2(packed[0], packed[1]);
             reinterpret_cast<uint2*>(xq + (size_t)t * H)[c] = pv;
             if (dbg_xq) reinterpret_cast<uint2*>(dbg_xq + (size_t)t * H)[c] = pv;
+            if (tplanes) {
+                // 8 codes -> one 32-bit word of each plane (word c % 4 of block c / 4)
+                uint32_t d[3] = {0u, 0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint32_t tc = lut[(packed[e >> 2] >> (8 * (e & 3))) & 0xffu];
+                    d[0] |= (tc & 0xFu) << (4 * e);
+                    d[1] |= ((tc >> 4) & 0xFu) << (4 * e);
+                    d[2] |= (tc >> 8) << (4 * e);
+                }
+                uint32_t* dst = reinterpret_cast<uint32_t*>(tplanes + ((size_t)t * (H / 32) + (c >> 2)) * 48) + (c & 3);
+                dst[0] = d[0];
+                dst[4] = d[1];
+                dst[8] = d[2];
+            }
         }
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
         bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
@@ -100,8 +123,9 @@ __global__ void __launch_bounds__(kQThreads)
 // needs, tensor-core rows get the digit planes of the W2 tensor-core GEMM
 // written directly (plane row plane_row[i]).  Thread l of a row holds the
 // elements 4*(l + R*g) .. +3 in step g; 8 consecutive threads cover one
-// 32-input chunk.
-template <int R>
+// 32-input chunk.  KEEP > 0 (rows of at most 4*R*KEEP elements): pass 1 keeps
+// the values in registers for pass 2 instead of reading them again.
+template <int R, int KEEP>
 __global__ void __launch_bounds__(kQThreads)
     k_hquant(const double* __restrict__ gacc, float* __restrict__ hbuf,
              const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
@@ -112,6 +136,7 @@ __global__ void __launch_bounds__(kQThreads)
              int32_t* flag) {
     pdl_begin();
     static_assert(R == 32 || R == kQThreads, "a warp or a CTA per row");
+    float4 keep[KEEP > 0 ? KEEP : 1];
     __shared__ uint16_t lut[256];
     __shared__ float red[33];
     for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
@@ -131,9 +156,20 @@ __global__ void __launch_bounds__(kQThreads)
         }
         float4* hr = reinterpret_cast<float4*>(hbuf + (size_t)(row_ok ? i : 0) * I);
         if (row_ok && tc) {
-            for (int g = 0; g < steps; ++g) {
-                const float4 v = hr[g * R + l];
-                a = fmaxf(fmaxf(a, fabsf(v.x)), fmaxf(fmaxf(fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
+            if (KEEP > 0) {
+#pragma unroll
+                for (int g = 0; g < (KEEP > 0 ? KEEP : 1); ++g)
+                    if (g < steps) {
+                        keep[g] = hr[g * R + l];
+                        a = fmaxf(fmaxf(a, fabsf(keep[g].x)), fmaxf(fmaxf(fabsf(keep[g].y), fabsf(keep[g].z)),
+                                                                   fabsf(keep[g].w)));
+                    }
+            } else {
+#pragma unroll 4
+                for (int g = 0; g < steps; ++g) {
+                    const float4 v = hr[g * R + l];
+                    a = fmaxf(fmaxf(a, fabsf(v.x)), fmaxf(fmaxf(fabsf(v.y), fabsf(v.z)), fabsf(v.w)));
+                }
             }
         } else if (row_ok) {
             const double s = (double)sx[p / k];
@@ -169,9 +205,18 @@ __global__ void __launch_bounds__(kQThreads)
                 pr = -1;
             }
         }
+#pragma unroll(KEEP > 0 ? KEEP : 4)
         for (int g = 0; g < steps; ++g) {
             const int e0 = 4 * (g * R + l);
-            const float4 v = hr[g * R + l];
+            float4 v;
+            if (KEEP > 0 && tc) {
+                // (the loop is unrolled KEEP times, so the index is a constant)
+#pragma unroll
+                for (int u = 0; u < (KEEP > 0 ? KEEP : 1); ++u)
+                    if (u == g) v = keep[u];
+            } else {
+                v = hr[g * R + l];
+            }
             const int q[4] = {quant_code(v.x, a, sc), quant_code(v.y, a, sc), quant_code(v.z, a, sc),
                               quant_code(v.w, a, sc)};
             const uint32_t packed = (uint32_t)(q[0] & 0xff) | (uint32_t)(q[1] & 0xff) << 8 |
@@ -213,25 +258,29 @@ __global__ void __launch_bounds__(kQThreads)
 __global__ void __launch_bounds__(256)
     k_prepare_rows(const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
                    const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
-                   const int32_t* __restrict__ plane_off, int P, int E, int I, int H,
-                   int32_t* __restrict__ plane_row,
-                   double* __restrict__ gacc, double* __restrict__ yacc, int32_t* flag) {
+                   const int32_t* __restrict__ plane_off, const int32_t* __restrict__ unit_off, int P,
+                   int E, int I, int H, int32_t* __restrict__ plane_row, double* __restrict__ gacc,
+                   double* __restrict__ yacc, int32_t* flag) {
     pdl_begin();
+    // phase 1, a thread per row: plane rows
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += gridDim.x * blockDim.x) {
+        const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
+        int pr = -1;
+        if (expert_tc[e]) {
+            const int r0 = offsets[e], r1 = offsets[e + 1];
+            if (i >= r0 && i < r1)
+                pr = plane_off[e] + (i - r0);
+            else
+                raise_flag(flag, FLAG_BOUNDS);
+        }
+        plane_row[i] = pr;
+    }
+    // phase 2, a CTA per row: clear the accumulators of streaming rows (none
+    // when the planner gave the streaming GEMM no units)
+    if (__ldg(unit_off + E) == 0) return;
     for (int i = blockIdx.x; i < P; i += gridDim.x) {
         const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
-        const bool tc = expert_tc[e] != 0;
-        if (threadIdx.x == 0) {
-            int pr = -1;
-            if (tc) {
-                const int r0 = offsets[e], r1 = offsets[e + 1];
-                if (i >= r0 && i < r1)
-                    pr = plane_off[e] + (i - r0);
-                else
-                    raise_flag(flag, FLAG_BOUNDS);
-            }
-            plane_row[i] = pr;
-        }
-        if (tc) continue;
+        if (expert_tc[e]) continue;
         double2* g = reinterpret_cast<double2*>(gacc + (size_t)i * 2 * I);
         for (int j = threadIdx.x; j < I; j += blockDim.x) g[j] = make_double2(0.0, 0.0);
         double2* y = reinterpret_cast<double2*>(yacc + (size_t)i * H);
@@ -283,10 +332,10 @@ cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, c
 }
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
-                          int8_t* dbg_xq, float* dbg_sx, cudaStream_t st) {
+                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const cudaError_t e = launch_pdl(k_xquant, dim3(T), dim3(kQThreads), 0, st, (const __nv_bfloat16*)x, T, H,
-                                     xq, sx, xinit, dbg_xq, dbg_sx);
+                                     xq, sx, xinit, tplanes, dbg_xq, dbg_sx);
     count_launches(1);
     return e;
 }
@@ -301,26 +350,29 @@ cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert
     // rows (prefill): a warp per row needs no block barriers
     cudaError_t e;
     if (P < 4096 && I % (4 * kQThreads) == 0) {
-        e = launch_pdl(k_hquant<kQThreads>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf,
+        e = launch_pdl(k_hquant<kQThreads, 0>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf,
                        expert_tc, topk_idx, sx, perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit,
                        dbg_hq, dbg_sh, flag);
     } else {
         const int warps = kQThreads / 32;
         const int grid = std::min((P + warps - 1) / warps, 148 * 8);
-        e = launch_pdl(k_hquant<32>, dim3(grid), dim3(kQThreads), 0, st, gacc, hbuf, expert_tc, topk_idx, sx, perm,
-                       plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq, dbg_sh, flag);
+        // (keeping a row in registers between the passes, k_hquant<32, 16>,
+        // measured slower: 112 registers halve the rows in flight)
+        e = launch_pdl(k_hquant<32, 0>, dim3(grid), dim3(kQThreads), 0, st, gacc, hbuf, expert_tc, topk_idx, sx,
+                       perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq, dbg_sh, flag);
     }
     count_launches(1);
     return e;
 }
 
 cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                const int32_t* offsets, const int32_t* plane_off, int P, int E, int I,
-                                int H, int32_t* plane_row, double* gacc, double* yacc,
+                                const int32_t* offsets, const int32_t* plane_off, const int32_t* unit_off,
+                                int P, int E, int I, int H, int32_t* plane_row, double* gacc, double* yacc,
                                 int32_t* flag, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
     const cudaError_t e = launch_pdl(k_prepare_rows, dim3(std::min(P, 148 * 8)), dim3(256), 0, st, expert_tc,
-                                     topk_idx, perm, offsets, plane_off, P, E, I, H, plane_row, gacc, yacc, flag);
+                                     topk_idx, perm, offsets, plane_off, unit_off, P, E, I, H, plane_row, gacc,
+                                     yacc, flag);
     count_launches(1);
     return e;
 }

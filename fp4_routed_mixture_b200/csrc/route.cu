@@ -19,7 +19,7 @@ __device__ __forceinline__ bool ranks_above(float a, int ia, float b, int ib) {
     return ia < ib;
 }
 
-template <int KMAX>
+template <int KMAX, int S>
 __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits, int T, int E, int k,
                                                int32_t* __restrict__ topk_idx,
                                                float* __restrict__ gates) {
@@ -28,11 +28,15 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     const float* row = logits + (size_t)t * E;
-    const int per_lane = (E + 31) >> 5;  // <= 32 because E <= 1024
-    uint32_t avail = per_lane >= 32 ? 0xffffffffu : ((1u << per_lane) - 1u);
-    // drop slots past E
-    for (int s = 0; s < per_lane; ++s)
-        if (lane + 32 * s >= E) avail &= ~(1u << s);
+    // lane l holds logits l, l+32, ... (S slots, E <= 32*S) in registers
+    float val[S];
+    uint32_t avail = 0u;
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        const int id = lane + 32 * s;
+        val[s] = id < E ? __ldg(row + id) : 0.0f;
+        if (id < E) avail |= 1u << s;
+    }
 
     float sel_val[KMAX];
     int sel_id[KMAX];
@@ -42,12 +46,11 @@ __global__ void __launch_bounds__(256) k_route(const float* __restrict__ logits,
         // lane-local best among still-available slots
         float bv = 0.0f;
         int bi = -1;
-        for (uint32_t m = avail; m; m &= m - 1) {
-            const int s = __ffs(m) - 1;
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
             const int id = lane + 32 * s;
-            const float v = __ldg(row + id);
-            if (bi < 0 || ranks_above(v, id, bv, bi)) {
-                bv = v;
+            if (((avail >> s) & 1u) && (bi < 0 || ranks_above(val[s], id, bv, bi))) {
+                bv = val[s];
                 bi = id;
             }
         }
@@ -89,9 +92,13 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
     if (T == 0) return cudaSuccess;
     const int warps = 8;
     dim3 grid((T + warps - 1) / warps);
-    const cudaError_t e =
-        k <= 8 ? launch_pdl(k_route<8>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates)
-               : launch_pdl(k_route<16>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates);
+    cudaError_t e;
+    if (E <= 256)
+        e = k <= 8 ? launch_pdl(k_route<8, 8>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates)
+                   : launch_pdl(k_route<16, 8>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates);
+    else
+        e = k <= 8 ? launch_pdl(k_route<8, 32>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates)
+                   : launch_pdl(k_route<16, 32>, grid, dim3(warps * 32), 0, st, logits, T, E, k, topk_idx, gates);
     count_launches(1);
     return e;
 }

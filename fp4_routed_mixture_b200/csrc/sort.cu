@@ -59,17 +59,27 @@ __device__ int block_exclusive_scan(int* vals, int E, int* tmp) {
     return total;
 }
 
-// Stable scatter of pairs [p0, p1) by one warp; cursor[e] is the next free
-// sorted slot of expert e and is advanced in place.
+// Stable scatter of pairs [p0, p1) (at most 32 x 32 of them) by one warp;
+// cursor[e] is the next free sorted slot of expert e and is advanced in place.
+// The warp first loads all of its expert ids (lane l holds pairs p0 + 32s + l)
+// so the serial steps wait on no global load.
 __device__ void warp_stable_scatter(const int32_t* __restrict__ topk_idx, int p0, int p1, int E,
                                     int* cursor, int32_t* __restrict__ perm,
                                     int32_t* __restrict__ pos) {
     const int lane = threadIdx.x & 31;
-    for (int base = p0; base < p1; base += 32) {
+    int ids[32];
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+        const int p = p0 + 32 * s + lane;
+        ids[s] = p < p1 ? __ldg(topk_idx + p) : -1;
+    }
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+        const int base = p0 + 32 * s;
+        if (base >= p1) break;
         const int p = base + lane;
-        const bool in = p < p1;
-        int e = in ? __ldg(topk_idx + p) : -1;
-        if (!valid_expert(e, E)) e = -1 - lane;  // unique key: never grouped, never written
+        int e = ids[s];
+        if (p >= p1 || !valid_expert(e, E)) e = -1 - lane;  // unique key: never grouped, never written
         const uint32_t same = __match_any_sync(0xffffffffu, e);
         const int rank = __popc(same & ((1u << lane) - 1u));
         const int leader = __ffs(same) - 1;
@@ -119,6 +129,7 @@ __global__ void __launch_bounds__(kSortThreads)
     const int nchunks = gridDim.x, c = blockIdx.x;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int tot = 0, before = 0;
+#pragma unroll 8
         for (int j = 0; j < nchunks; ++j) {
             const int v = chunk_hist[(size_t)j * E + e];
             tot += v;
@@ -216,6 +227,7 @@ constexpr size_t kSortStaticBytes =
 static __device__ __align__(256) uint8_t g_sort_scratch[kSortStaticBytes];
 
 static_assert(kSortStaticMaxPairs % kSortChunk == 0, "whole chunks");
+static_assert(kSortChunk <= 32 * 32, "warp_stable_scatter holds 32 ids per lane");
 
 // Device address of g_sort_scratch on the current device, looked up once per
 // device (the host-side name is only a stand-in for it).

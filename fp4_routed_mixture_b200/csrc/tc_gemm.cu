@@ -471,50 +471,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                      : "memory");
 }
 
-// Writes the three E2M1 digit planes of INT8 rows in the stage-major layout:
-// plane p, 32-input chunk c = 4*g + cc of plane row pr -> 16 bytes at
-// planes + (g*(plane_rows/8) + pr/8)*1536 + p*512 + cc*128 + (pr%8)*16, element
-// 2j of the chunk in the low nibble of byte j.  Source row of sorted row i:
-// perm[i] / k_div (k_div > 0) or i; its plane row is plane_row[i] (-1: a row of
-// a streaming-GEMM expert, not written).  One thread per (row, chunk), rows
-// fastest: 8 consecutive rows fill 128 contiguous bytes of each plane.
+// Copies the x digit planes of every sorted row of a tensor-core expert from
+// token order (k_xquant: per token and 32-input block c, 48 bytes = plane p's
+// 16 bytes at +16p) into the stage-major layout: plane p, block c = 4*g + cc of
+// plane row pr -> 16 bytes at planes + (g*(plane_rows/8) + pr/8)*1536 + p*512
+// + cc*128 + (pr%8)*16.  Source token of sorted row i: perm[i] / k_div; its
+// plane row is plane_row[i] (-1: a row of a streaming-GEMM expert, skipped).
+// One thread per (row, block), rows fastest: 8 consecutive rows fill 128
+// contiguous bytes of each plane.  Grid: (rows / 256, K / 128); a thread
+// copies the 4 blocks of one stage of its row.
 __global__ void __launch_bounds__(256)
-    k_planes(const int8_t* __restrict__ src, int K, const int32_t* __restrict__ perm, int k_div, int rows,
+    k_planes(const uint8_t* __restrict__ tplanes, int K, const int32_t* __restrict__ perm, int k_div, int rows,
              const int32_t* __restrict__ plane_row, int plane_rows, uint8_t* __restrict__ planes,
              int32_t* flag) {
     pdl_begin();
-    __shared__ uint16_t lut[256];  // byte of q -> digit_codes(q)
-    for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
-    __syncthreads();
     const int nc = K / 32;
-    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (id >= (long long)rows * nc) return;
-    const int i = (int)(id % rows), c = (int)(id / rows);
+    const int i = blockIdx.x * blockDim.x + threadIdx.x, g = blockIdx.y;
+    if (i >= rows) return;
     const int pr = __ldg(plane_row + i);
     if (pr < 0) return;
     if (pr >= plane_rows) {
         raise_flag(flag, FLAG_BOUNDS);
         return;
     }
-    const int srow = k_div > 0 ? checked_index(__ldg(perm + i), rows, flag) / k_div : i;
-    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)srow * K + c * 32);
-    const uint4 v0 = __ldg(s), v1 = __ldg(s + 1);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t out[3][4] = {};
+    const int t = checked_index(__ldg(perm + i), rows, flag) / k_div;
+    const uint4* s = reinterpret_cast<const uint4*>(tplanes + ((size_t)t * nc + 4 * g) * 48);
+    uint4 v[12];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const uint32_t t = lut[(w[e >> 2] >> (8 * (e & 3))) & 0xFFu];
-        const int sh = 4 * (e & 7);
-        out[0][e >> 3] |= (t & 0xFu) << sh;
-        out[1][e >> 3] |= ((t >> 4) & 0xFu) << sh;
-        out[2][e >> 3] |= (t >> 8) << sh;
-    }
-    const int g = c >> 2, cc = c & 3;
-    uint8_t* dst = planes + ((size_t)g * (plane_rows / 8) + (pr >> 3)) * kPlaneGroupBytes + cc * 128 +
-                   (pr & 7) * 16;
+    for (int u = 0; u < 12; ++u) v[u] = __ldg(s + u);   // blocks 4g..4g+3, planes 0..2
+    uint8_t* dst = planes + ((size_t)g * (plane_rows / 8) + (pr >> 3)) * kPlaneGroupBytes + (pr & 7) * 16;
 #pragma unroll
-    for (int p = 0; p < 3; ++p)
-        *reinterpret_cast<uint4*>(dst + p * 512) = make_uint4(out[p][0], out[p][1], out[p][2], out[p][3]);
+    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+        for (int p = 0; p < 3; ++p) *reinterpret_cast<uint4*>(dst + p * 512 + cc * 128) = v[3 * cc + p];
 }
 
 static int tc_grid() {
@@ -531,13 +520,13 @@ static int tc_grid() {
 
 size_t tc_smem_bytes() { return sizeof(TcShared); }
 
-cudaError_t launch_planes(const int8_t* src, int K, const int32_t* perm, int k_div, int rows,
+cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, int k_div, int rows,
                           const int32_t* plane_row, int plane_rows, uint8_t* planes, int32_t* flag,
                           cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
-    const long long n = (long long)rows * (K / 32);
-    const cudaError_t e = launch_pdl(k_planes, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, src, K, perm,
-                                     k_div, rows, plane_row, plane_rows, planes, flag);
+    const cudaError_t e = launch_pdl(k_planes, dim3((unsigned)((rows + 255) / 256), (unsigned)(K / 128)),
+                                     dim3(256), 0, st, tplanes, K, perm, k_div, rows, plane_row, plane_rows, planes,
+                                     flag);
     count_launches(1);
     return e;
 }
