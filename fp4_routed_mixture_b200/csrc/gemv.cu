@@ -35,13 +35,17 @@
 
 namespace moe {
 
-// Tuning (measured on B200, decode T=8 and T=64): a 2-deep ring per warp and
-// 8 warps per CTA (5 CTAs per SM) stream at ~96% of the measured copy
-// bandwidth.  Giving a warp two 32-row tiles per item (two weight streams 69 KB
-// apart) or deeper rings with fewer warps, and TMA bulk copies in place of the
-// per-lane 16-byte copies, were all slower.
+// Tuning (measured on B200, decode T=8 and T=64): a 2-deep ring per warp,
+// 32 warps per SM.  Giving a warp two 32-row tiles per item (two weight
+// streams 69 KB apart), deeper rings with fewer warps, more warps with fewer
+// registers, and TMA bulk copies in place of the per-lane 16-byte copies were
+// all slower.  The kernel is bound by integer issue (the nibble decode), at
+// about 0.6 of the measured copy bandwidth.
 constexpr int kGroup = kGemvGroup;  // token rows per unit
-constexpr int kGemvWarps = 8;      // warps per CTA; every warp runs its own pipeline
+// One warp per CTA, 32 CTAs per SM: every warp runs its own pipeline anyway,
+// and single-warp CTAs measured ~10% faster than 8-warp CTAs at the same 32
+// warps per SM (decode_T8: 3.58 -> 3.96 TB/s; 4 warps/CTA: 3.70).
+constexpr int kGemvWarps = 1;
 constexpr int kStages = 2;         // shared-memory ring depth per warp
 constexpr int kGroupBytes = 2176;  // 4 scale blocks of 32 rows: 128 B scales + 4 x 512 B codes
 constexpr int kChunkBytes = 8704;  // packed chunk: 4 scale blocks of 128 rows (see pack.cu)
@@ -194,7 +198,7 @@ __device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, 
     return d0 + d1;
 }
 
-__global__ void __launch_bounds__(kGemvWarps * 32, 4) k_gemv(GemvArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
     pdl_begin();
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
