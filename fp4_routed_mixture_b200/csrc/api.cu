@@ -242,13 +242,13 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
         cudaError_t _e = (call);                     \
         if (_e != cudaSuccess) return cuda_fail(_e, what); \
     } while (0)
-    MOE_TRY(moe::launch_check_header(packed, H, I, E, flag, stream), "header check");
     // an expert has at most T rows, so the tensor-core path is skipped without
     // reading any count when T < tc_min
     const bool use_tc = T >= g_tc_min_rows;
     uint8_t* xtp = (uint8_t*)(w + L.xtp);
     MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
-                               dbg ? dbg->sx : nullptr, stream), "x quant");
+                               dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
+            "x quant + header check");
     int32_t* toff1 = (int32_t*)(w + L.toff1);
     int32_t* toff2 = (int32_t*)(w + L.toff2);
     uint8_t* px = (uint8_t*)(w + L.px);
@@ -258,11 +258,9 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     int32_t* etc = (int32_t*)(w + L.etc);
     float* hbuf = (float*)(w + L.hbuf);
     float* yf = (float*)(w + L.yf);
-    MOE_TRY(moe::launch_plan(offsets, E, P, 2 * I, H, use_tc ? g_tc_min_rows : 0x7fffffff, uoff1, uoff2,
-                             toff1, toff2, poff, etc, flag, stream), "plan");
-    MOE_TRY(moe::launch_prepare_rows(etc, topk_idx, perm, offsets, poff, uoff1, P, E, I, H, prow, gacc, yacc,
-                                     flag, stream),
-            "row state");
+    MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? g_tc_min_rows : 0x7fffffff,
+                                  uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
+            "plan + row state");
     if (use_tc)
         MOE_TRY(moe::launch_planes(xtp, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;

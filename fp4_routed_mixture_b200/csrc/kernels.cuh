@@ -12,11 +12,17 @@ namespace moe {
 // 128 sorted token rows (its N); shared by the planner and the kernel.
 // Token rows per unit of the streaming GEMM (shared by it and the planner).
 constexpr int kGemvGroup = 4;
+constexpr int kMaxExperts = 1024;   // the API's limit on E
 constexpr int kTcWeightTile = 128;
 constexpr int kTcTokenTile = 128;
 
 // Number of kernels this library has launched in the process (diagnostics).
 void count_launches(int n);
+
+cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
+                             int I, int H, int tc_min, int32_t* unit_off1, int32_t* unit_off2,
+                             int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc,
+                             int32_t* plane_row, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may be
 // scheduled before the preceding kernel in the stream completes.  Every kernel
@@ -60,28 +66,23 @@ cudaError_t launch_pack(int H, int I, int E, const uint8_t* w1c, const uint8_t* 
                         uint8_t* out_w1c, uint8_t* out_w1s, uint8_t* out_w2c, uint8_t* out_w2s,
                         cudaStream_t st);
 const int32_t* packed_flag_ptr(const void* packed);
-cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t* flag,
-                                cudaStream_t st);
+
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
-                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, cudaStream_t st);
+                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, const void* packed, int I, int E,
+                          int32_t* flag, cudaStream_t st);
 cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
                           const int32_t* topk_idx, const float* sx, const int32_t* perm,
                           const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
                           int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
                           int32_t* flag, cudaStream_t st);
-cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                const int32_t* offsets, const int32_t* plane_off, const int32_t* unit_off,
-                                int P, int E, int I, int H, int32_t* plane_row, double* gacc, double* yacc,
-                                int32_t* flag, cudaStream_t st);
+
 cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
 cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
                               cudaStream_t st);
 
-cudaError_t launch_plan(const int32_t* offsets, int E, int P, int n1, int n2, int tc_min,
-                        int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2,
-                        int32_t* plane_off, int32_t* expert_tc, int32_t* flag, cudaStream_t st);
+
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,

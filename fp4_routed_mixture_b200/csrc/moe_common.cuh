@@ -82,6 +82,23 @@ __device__ __forceinline__ int quant_code(float v, float amax, float s) {
     return (int)r;
 }
 
+// Header at the start of a packed weight buffer (written by moe_pack_weights).
+struct PackHeader {
+    uint32_t magic, version, H, I, E, reserved0;
+    uint64_t w1_off, w2_off;
+    int32_t flag;  // device error word of moe_pack_weights
+};
+constexpr uint32_t kPackMagic = 0x34454F4Du;  // "MOE4"
+constexpr uint32_t kPackVersion = 3;
+
+// True when the packed buffer was built for these dims (a mismatch raises
+// FLAG_LAYOUT and keeps the GEMMs out of the buffer).
+__device__ __forceinline__ bool packed_header_ok(const void* packed, int H, int I, int E) {
+    const PackHeader* h = reinterpret_cast<const PackHeader*>(packed);
+    return h->magic == kPackMagic && h->version == kPackVersion && (int)h->H == H && (int)h->I == I &&
+           (int)h->E == E;
+}
+
 // First statement of every kernel launched with launch_pdl: wait until the
 // preceding kernel in the stream has completed and its writes are visible,
 // then allow the next kernel to be scheduled (it waits in turn, so at most two

@@ -30,14 +30,6 @@
 
 namespace moe {
 
-struct PackHeader {
-    uint32_t magic, version, H, I, E, reserved0;
-    uint64_t w1_off, w2_off;
-    int32_t flag;  // device error word of moe_pack_weights
-};
-
-constexpr uint32_t kPackMagic = 0x34454F4Du;  // "MOE4"
-constexpr uint32_t kPackVersion = 3;
 
 __host__ __device__ inline size_t matrix_bytes(int N, int K) { return (size_t)N * K * 17 / 32; }
 
@@ -105,14 +97,6 @@ __global__ void k_write_header(PackHeader* h, int H, int I, int E, uint64_t w1_o
     h->flag = 0;
 }
 
-// First kernel of moe_forward (one thread): clears the call's device error word
-// and sets FLAG_LAYOUT when the packed buffer was built for other dims.
-__global__ void k_check_header(const PackHeader* h, int H, int I, int E, int32_t* flag) {
-    pdl_begin();
-    const bool bad = h->magic != kPackMagic || h->version != kPackVersion || (int)h->H != H ||
-                     (int)h->I != I || (int)h->E != E;
-    *flag = bad ? FLAG_LAYOUT : 0;
-}
 
 PackedLayout packed_layout(int H, int I, int E) {
     PackedLayout L;
@@ -163,12 +147,5 @@ const int32_t* packed_flag_ptr(const void* packed) {
     return &((const PackHeader*)packed)->flag;
 }
 
-cudaError_t launch_check_header(const void* packed, int H, int I, int E, int32_t* flag,
-                                cudaStream_t st) {
-    const cudaError_t e = launch_pdl(k_check_header, dim3(1), dim3(1), 0, st, (const PackHeader*)packed, H, I, E,
-                                     flag);
-    count_launches(1);
-    return e;
-}
 
 }  // namespace moe

@@ -1,10 +1,12 @@
 // INT8 activation quantisation ("DeepSeek-V4-Flash on AMD gfx90a", abstract:
 // INT8 activations feeding the packed-FP4 expert GEMMs).
 //
-//   k_xquant        x [T,H] bf16 -> xq [T,H] int8, sx [T], xinit [T,H/32]
+//   k_xquant        x [T,H] bf16 -> xq [T,H] int8, sx [T], xinit [T,H/32], and
+//                   (tensor-core path) the x digit planes in token order; also
+//                   checks the packed header and clears the call's error word
 //   k_hquant        h of every sorted row (SwiGLU of the streaming GEMM's fp64
-//                   sums, or h from the tensor-core epilogue) -> hq, sh, hinit
-//   k_prepare_rows  clears per-row state before the W1/W2 GEMMs
+//                   sums, or h from the tensor-core epilogue) -> hq, sh, hinit,
+//                   or the W2 digit planes for tensor-core rows
 //   k_quant_rows    fp32 rows -> int8 + scale (stage entry point)
 //
 // Rule for every row: a = max|v| (exact), s = fp32(a/127) by IEEE division,
@@ -41,11 +43,16 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // tplanes + (t*(H/32) + b)*48: plane p's 16 bytes at +16p (element 2j of the
 // block in the low nibble of byte j).  The tensor-core GEMM's plane writer
 // copies these pieces into sorted-row order.
+// It is also the first kernel of moe_forward: thread 0 of CTA 0 clears the
+// call's device error word and sets FLAG_LAYOUT when the packed buffer was
+// built for other dims (no other CTA of this kernel touches the word).
 __global__ void __launch_bounds__(kQThreads)
     k_xquant(const __nv_bfloat16* __restrict__ x, int T, int H, int8_t* __restrict__ xq,
              float* __restrict__ sx, int32_t* __restrict__ xinit, uint8_t* __restrict__ tplanes,
-             int8_t* __restrict__ dbg_xq, float* __restrict__ dbg_sx) {
+             int8_t* __restrict__ dbg_xq, float* __restrict__ dbg_sx, const void* __restrict__ packed, int I,
+             int E, int32_t* flag) {
     pdl_begin();
+    if (blockIdx.x == 0 && threadIdx.x == 0) *flag = packed_header_ok(packed, H, I, E) ? 0 : FLAG_LAYOUT;
     __shared__ float red[33];
     __shared__ uint16_t lut[256];
     if (tplanes)
@@ -249,44 +256,6 @@ __global__ void __launch_bounds__(kQThreads)
     }
 }
 
-// Per sorted row: for rows of tensor-core experts writes the row's place in the digit-plane buffers
-// (plane_off[e] + rank inside the expert), for the others -1 and clears the
-// fp64 accumulators (the streaming GEMM adds partial sums into them).  Rows of
-// tensor-core experts are written whole by that GEMM.  A row whose expert's
-// offsets do not contain it (tables that did not come from one sort) raises
-// FLAG_BOUNDS and gets no plane row.
-__global__ void __launch_bounds__(256)
-    k_prepare_rows(const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
-                   const int32_t* __restrict__ perm, const int32_t* __restrict__ offsets,
-                   const int32_t* __restrict__ plane_off, const int32_t* __restrict__ unit_off, int P,
-                   int E, int I, int H, int32_t* __restrict__ plane_row, double* __restrict__ gacc,
-                   double* __restrict__ yacc, int32_t* flag) {
-    pdl_begin();
-    // phase 1, a thread per row: plane rows
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += gridDim.x * blockDim.x) {
-        const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
-        int pr = -1;
-        if (expert_tc[e]) {
-            const int r0 = offsets[e], r1 = offsets[e + 1];
-            if (i >= r0 && i < r1)
-                pr = plane_off[e] + (i - r0);
-            else
-                raise_flag(flag, FLAG_BOUNDS);
-        }
-        plane_row[i] = pr;
-    }
-    // phase 2, a CTA per row: clear the accumulators of streaming rows (none
-    // when the planner gave the streaming GEMM no units)
-    if (__ldg(unit_off + E) == 0) return;
-    for (int i = blockIdx.x; i < P; i += gridDim.x) {
-        const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
-        if (expert_tc[e]) continue;
-        double2* g = reinterpret_cast<double2*>(gacc + (size_t)i * 2 * I);
-        for (int j = threadIdx.x; j < I; j += blockDim.x) g[j] = make_double2(0.0, 0.0);
-        double2* y = reinterpret_cast<double2*>(yacc + (size_t)i * H);
-        for (int j = threadIdx.x; j < H / 2; j += blockDim.x) y[j] = make_double2(0.0, 0.0);
-    }
-}
 
 __global__ void __launch_bounds__(kQThreads)
     k_quant_rows(const float* __restrict__ v, int cols, int8_t* __restrict__ q, float* __restrict__ s) {
@@ -332,10 +301,11 @@ cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, c
 }
 
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
-                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, cudaStream_t st) {
+                          uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, const void* packed, int I, int E,
+                          int32_t* flag, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const cudaError_t e = launch_pdl(k_xquant, dim3(T), dim3(kQThreads), 0, st, (const __nv_bfloat16*)x, T, H,
-                                     xq, sx, xinit, tplanes, dbg_xq, dbg_sx);
+                                     xq, sx, xinit, tplanes, dbg_xq, dbg_sx, packed, I, E, flag);
     count_launches(1);
     return e;
 }
@@ -365,17 +335,6 @@ cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert
     return e;
 }
 
-cudaError_t launch_prepare_rows(const int32_t* expert_tc, const int32_t* topk_idx, const int32_t* perm,
-                                const int32_t* offsets, const int32_t* plane_off, const int32_t* unit_off,
-                                int P, int E, int I, int H, int32_t* plane_row, double* gacc, double* yacc,
-                                int32_t* flag, cudaStream_t st) {
-    if (P == 0) return cudaSuccess;
-    const cudaError_t e = launch_pdl(k_prepare_rows, dim3(std::min(P, 148 * 8)), dim3(256), 0, st, expert_tc,
-                                     topk_idx, perm, offsets, plane_off, unit_off, P, E, I, H, plane_row, gacc,
-                                     yacc, flag);
-    count_launches(1);
-    return e;
-}
 
 cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, float* s,
                               cudaStream_t st) {
