@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--workload", default="decode_T8")
     ap.add_argument("--prefill-workload", default="prefill_T4604")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-skew", action="store_true", help="skip the skewed prefill line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
@@ -363,28 +364,34 @@ def main():
         "kernel_ms_per_step": {"w1": round(r["w1_ms"] / steps, 5), "w2": round(r["w2_ms"] / steps, 5)},
     }
     if not a.no_prefill:
-        pw = synth.WORKLOADS[a.prefill_workload]
-        psteps = max(3, min(20, steps // 100))
-        rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=False)
-        ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
+        # prefill lines (tensor-core path): the prefill chunk, and the skewed
+        # prefill (one expert takes almost every row) as an informational line
         fp8_peak = 2.0 * peaks["bf16_tflops"]
-        out["prefill"] = {
-            "workload": pw.name, "T": pw.T, "steps": psteps,
-            "value": round(N * pw.T * psteps / (rp["ms"] * 1e-3), 1), "unit": "tokens/s",
-            "ms_per_step": round(rp["ms"] / psteps, 4),
-            "roofline": {"bound": "tensor",
-                         "kernel": "k_tc_gemm (tcgen05 kind::mxf4 block-scaled, W1 and W2 launches)",
-                         "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
-                         "frac": round(ptf / fp8_peak, 5),
-                         "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
-                         # the INT8 operand enters the FP4 MMA as three exact digit planes,
-                         # so the tensor pipe issues 3x the algorithmic work at the FP4 rate
-                         "mma_issued_tflops": round(3 * ptf, 2),
-                         "mma_peak_fp4": 4.0 * peaks["bf16_tflops"],
-                         "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
-                         "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
-                         "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
-        }
+        for key, pname, cap in (("prefill", a.prefill_workload, 20), ("prefill_skew", "prefill_skew_T16384", 5)):
+            if key == "prefill_skew" and a.no_skew:
+                continue
+            pw = synth.WORKLOADS[pname]
+            psteps = max(3, min(cap, steps // 100))
+            rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=False)
+            ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
+            out[key] = {
+                "workload": pw.name, "T": pw.T, "steps": psteps,
+                "value": round(N * pw.T * psteps / (rp["ms"] * 1e-3), 1), "unit": "tokens/s",
+                "ms_per_step": round(rp["ms"] / psteps, 4),
+                "gemm_ms_per_step": round(rp["gemm_ms"] / psteps, 4),
+                "roofline": {"bound": "tensor",
+                             "kernel": "k_tc_gemm (tcgen05 kind::mxf4 block-scaled, W1 and W2 launches)",
+                             "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
+                             "frac": round(ptf / fp8_peak, 5),
+                             "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
+                             # the INT8 operand enters the FP4 MMA as three exact digit planes,
+                             # so the tensor pipe issues 3x the algorithmic work at the FP4 rate
+                             "mma_issued_tflops": round(3 * ptf, 2),
+                             "mma_peak_fp4": 4.0 * peaks["bf16_tflops"],
+                             "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
+                             "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
+                             "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
+            }
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)
     if rank0:
