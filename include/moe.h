@@ -18,8 +18,12 @@
  *     says otherwise.  The library never allocates or frees device memory.
  *   - Calls are asynchronous on `stream` and never synchronise the host, except
  *     moe_pack_weights and moe_check_device_flag (load-time / test calls that
- *     say so).  moe_route, moe_sort and moe_forward can be captured in a CUDA
- *     graph.
+ *     say so).  moe_route, moe_sort, moe_forward and moe_layer_forward can be
+ *     captured in a CUDA graph.
+ *   - Kernels are launched with programmatic dependent launch: a kernel may be
+ *     scheduled while the previous kernel on `stream` finishes, but it waits for
+ *     that kernel to complete before it touches memory, so stream order holds
+ *     for the caller's own work before and after every call.
  *   - Return value: MOE_OK, or a negative moe_status.  Host-side argument
  *     checks fail before anything is launched; moe_last_error() returns the
  *     message of the calling thread's last failure.
