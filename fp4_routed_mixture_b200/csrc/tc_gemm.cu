@@ -81,6 +81,7 @@ struct TcShared {
     uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once per pipe
     float col_scale[TC_EPI_WARPS][32];  // per epilogue warp: activation scale of its 32 columns
     uint64_t full[TC_PIPES][TC_STAGES], empty[TC_PIPES][TC_STAGES], acc_full[TC_ACC], acc_empty[TC_ACC];
+    uint64_t drain[TC_PIPES];   // each issuer's last commit: all of its MMAs are done
     uint32_t tmem_base;
     int32_t abort;
 };
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             mbar_init(smem_u32(&sh.acc_full[b]), 1);
             mbar_init(smem_u32(&sh.acc_empty[b]), TC_EPI_WARPS);
         }
+        for (int r = 0; r < TC_PIPES; ++r) mbar_init(smem_u32(&sh.drain[r]), 1);
         sh.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -397,6 +399,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             if (lane == 0) tc_commit(smem_u32(&sh.acc_full[buf]));
             __syncwarp();
         }
+        // before the CTA frees TMEM, every MMA this warp issued must be done
+        // (on the normal path the epilogue has already seen them finish; after a
+        // timeout some may still be in flight)
+        if (lane == 0) {
+            tc_commit(smem_u32(&sh.drain[r]));
+            mbar_wait_bounded(smem_u32(&sh.drain[r]), 0);
+        }
+        __syncwarp();
     } else {
         // ---------------- epilogue (warps TC_EPI_WARP0 ..) ----------------
         // Warp (q, c) owns the 32 weight rows of TMEM lane quadrant q and the
