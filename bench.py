@@ -63,19 +63,23 @@ def parse():
 # distributed plumbing (replicas: barrier + max-over-ranks only, no data-path collective)
 
 class Dist:
-    def __init__(self, n_expected: int):
+    """One process per GPU (torchrun env vars): barrier and max over ranks.
+    backend/device default to NCCL on the rank's GPU; the CPU tests use gloo."""
+
+    def __init__(self, n_expected: int, backend: str | None = None, device: str | None = None):
         import torch
         import torch.distributed as dist
         self.torch, self.dist = torch, dist
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend or "nccl"
+        self.device = device or "cuda"
+        if self.device == "cuda":
+            torch.cuda.set_device(self.local if self.world > 1 else 0)
         if self.world > 1:
             import datetime
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-        else:
-            torch.cuda.set_device(0)
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=300))
         if n_expected != self.world:
             print(f"warning: --gpus {n_expected} but WORLD_SIZE {self.world}", file=sys.stderr)
 
@@ -86,13 +90,19 @@ class Dist:
     def max(self, v: float) -> float:
         if self.world == 1:
             return v
-        t = self.torch.tensor([v], dtype=self.torch.float64, device="cuda")
+        t = self.torch.tensor([v], dtype=self.torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.world > 1:
             self.dist.destroy_process_group()
+
+
+def whole_job_value(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Tokens/s of the whole job: every replica processes tokens_per_step tokens per
+    step (weak scaling); the slowest rank's time bounds the job."""
+    return world * tokens_per_step * steps / (max_ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------------------
@@ -344,7 +354,7 @@ def main():
     r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
     w = r["workload"]
     N = dist.world
-    value = N * w.T * steps / (r["ms"] * 1e-3)
+    value = whole_job_value(N, w.T, steps, r["ms"])
     out = {
         "metric": "routed-MoE layer tokens/s (T=8 decode, T=4604 prefill); % HBM / TC roofline",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": N, "steps": steps,
@@ -357,7 +367,7 @@ def main():
                    "l2": "inputs larger than L2: %.2f GB of expert weights streamed per step "
                          "vs 126 MB L2" % (r["alg_bytes_step"] / 1e9)},
         "roofline": roofline_hbm(r, peaks, profiled_traffic(f"k_gemv_{w.name}.md")),
-        "e2e": {"value": round(N * w.T * steps / (r["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_value(N, w.T, steps, r["e2e_ms"]), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
@@ -376,7 +386,7 @@ def main():
             ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
             out[key] = {
                 "workload": pw.name, "T": pw.T, "steps": psteps,
-                "value": round(N * pw.T * psteps / (rp["ms"] * 1e-3), 1), "unit": "tokens/s",
+                "value": round(whole_job_value(N, pw.T, psteps, rp["ms"]), 1), "unit": "tokens/s",
                 "ms_per_step": round(rp["ms"] / psteps, 4),
                 "gemm_ms_per_step": round(rp["gemm_ms"] / psteps, 4),
                 "roofline": {"bound": "tensor",
