@@ -34,6 +34,8 @@ __device__ __forceinline__ int checked_index(int v, int n, int32_t* flag) {
 }
 
 // ---- The layer's fp32 exp ---------------------------------------------------
+// Cody-Waite argument reduction (ln 2 split into a short exact high part and a
+// low part) followed by a Taylor polynomial; written from the mathematics.
 // Specification (the CPU reference implements the same one separately):
 //   NaN -> NaN; x > 88.8 -> +inf; x < -104 -> 0;
 //   n = rint(fp32(x * log2e)); r = fma(-n, ln2_hi, x); r = fma(-n, ln2_lo, r);
@@ -124,12 +126,6 @@ __device__ __forceinline__ uint32_t digit_codes(int q) {
         return d < 0 ? (8u | mag) : mag;
     };
     return code(a0) | code(b0) << 4 | code(c0) << 8;
-}
-
-// 2^(S-128) as a double (S is a UE8M0 byte in [0, 254]); used as the weight
-// scale of codes that are decoded to 2*e2m1 integers.
-__device__ __forceinline__ double pow2_scale_minus128(uint32_t S) {
-    return __hiloint2double((int)((S + 895u) << 20), 0);
 }
 
 template <class T>
