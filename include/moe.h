@@ -176,7 +176,10 @@ int moe_sort_static(const int32_t *topk_idx, int T, int k, int E, int32_t *perm,
  *   Y[i, n] = fp32( fp64(sh[i]) * sum_j hq[i,j] * w2[e, n, j] ),  n < H
  *   y[t, n] = bf16( sum_{j<k} gates[t,j] * Y[pos[t*k+j], n] )   (fp32 sum, slot order)
  * for every sorted row i = pos[t*k+j] with e = topk_idx[t*k+j].  The sums over
- * k and j are exact (integer-valued products in units of the smallest scale).
+ * k and j are exact (integer-valued products in units of half the row's
+ * smallest weight scale): in the streaming GEMM (fp64 block sums) while a row's
+ * scale bytes span less than about 28 binades, in the tensor-core GEMM (fp32
+ * accumulators) while every partial sum stays below 2^24 of those units.
  * x [T, H] bf16, y [T, H] bf16; the other pointers as produced by moe_route /
  * moe_sort; packed from moe_pack_weights with the same H, I, E.
  * ws: moe_workspace_bytes(d, T_max) bytes, 256-byte aligned, T <= T_max; its
@@ -219,7 +222,8 @@ int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStre
  *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
  *   run on the tensor-core grouped GEMM (tcgen05, tiles of 128 weight rows x
  *   128 token rows); experts with fewer rows run on the CUDA-core streaming
- *   GEMM.  Default 32; must be >= 1.  Both paths give the same results.
+ *   GEMM.  Default 32; must be >= 1.  Both paths give the same results inside
+ *   the exactness domains stated at moe_forward.
  * moe_set_option returns MOE_OK or MOE_ERR_INVALID_ARG; moe_get_option returns
  * the current value (-1 for an unknown option). */
 #define MOE_OPT_TC_MIN_ROWS 1
