@@ -24,7 +24,8 @@ FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_LAYOUT, FLAG_TIMEOUT, FLAG_BOUNDS = 1, 2, 
 # Exported symbols of include/moe.h, in declaration order.
 SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack_weights",
            "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_sort_static", "moe_workspace_bytes",
-           "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
+           "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_tables",
+           "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
            "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
 
 
@@ -63,6 +64,7 @@ def _load():
         "moe_forward": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
         "moe_layer_workspace_bytes": ([D, i32], sz),
         "moe_layer_forward": ([D, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
+        "moe_layer_tables": ([D, vp] + [ctypes.POINTER(vp)] * 5, i32),
         "moe_quant_rows_f32": ([vp, i32, i32, vp, vp, vp], i32),
         "moe_exp_f32": ([vp, vp, ctypes.c_int64, vp], i32),
         "moe_swiglu_f32": ([vp, vp, vp, ctypes.c_int64, vp], i32),
@@ -258,6 +260,26 @@ def moe_layer_forward(logits, x, packed, H: int, I: int, E: int, k: int, ws=None
                                  _ptr(ws), ws.numel(), ctypes.byref(dbg) if dbg is not None else None,
                                  _stream(stream)))
     return y
+
+
+def moe_layer_tables(ws, T: int, H: int, I: int, E: int, k: int):
+    """Views of the routing tables moe_layer_forward left in `ws` (a uint8 CUDA
+    tensor): topk_idx [T,k] int32, gates [T,k] fp32, perm [T*k], pos [T*k] and
+    offsets [E+1] int32."""
+    d = _dims(T, H, I, E, k)
+    ptrs = [ctypes.c_void_p() for _ in range(5)]
+    _check(lib.moe_layer_tables(ctypes.byref(d), _ptr(ws), *[ctypes.byref(p) for p in ptrs]))
+    base = ws.data_ptr()
+
+    def view(p, n, dtype, shape):
+        off = p.value - base
+        assert 0 <= off and off + 4 * n <= ws.numel()
+        return ws[off:off + 4 * n].view(dtype).view(shape)
+
+    P = T * k
+    return dict(idx=view(ptrs[0], P, torch.int32, (T, k)), gates=view(ptrs[1], P, torch.float32, (T, k)),
+                perm=view(ptrs[2], P, torch.int32, (P,)), pos=view(ptrs[3], P, torch.int32, (P,)),
+                offsets=view(ptrs[4], E + 1, torch.int32, (E + 1,)))
 
 
 def moe_quant_rows_f32(v, stream=None):

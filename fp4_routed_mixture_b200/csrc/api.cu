@@ -203,10 +203,18 @@ size_t moe_workspace_bytes(const moe_dims* d, int T_max) {
     return ws_layout(*d, T_max).total;
 }
 
-int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, const float* gates,
-                const int32_t* perm, const int32_t* pos, const int32_t* offsets, const void* packed,
-                void* y_bf16, void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
-    g_last_error.clear();
+}  // extern "C"
+
+namespace {
+
+// The layer from its routing tables on.  With logits == NULL, topk_idx, gates,
+// perm, pos and offsets are inputs (moe_forward).  With logits != NULL
+// (moe_layer_forward on a call with T below the tensor-core threshold and at
+// most kFrontMaxPairs pairs) route, sort, x quant and plan run as one fused
+// launch that writes those tables.
+int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int32_t* topk_idx, float* gates,
+                 int32_t* perm, int32_t* pos, int32_t* offsets, const void* packed, void* y_bf16, void* ws,
+                 size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
     if (int rc = check_dims(d, true)) return rc;
     if (!ws || !packed || !offsets) return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if (d->T > 0 && (!x_bf16 || !topk_idx || !gates || !perm || !pos || !y_bf16))
@@ -243,12 +251,9 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
         if (_e != cudaSuccess) return cuda_fail(_e, what); \
     } while (0)
     // an expert has at most T rows, so the tensor-core path is skipped without
-    // reading any count when T < tc_min
-    const bool use_tc = T >= g_tc_min_rows;
+    // reading any count when T < tc_min (always so with the fused front)
+    const bool use_tc = !logits && T >= g_tc_min_rows;
     uint8_t* xtp = (uint8_t*)(w + L.xtp);
-    MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
-                               dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
-            "x quant + header check");
     int32_t* toff1 = (int32_t*)(w + L.toff1);
     int32_t* toff2 = (int32_t*)(w + L.toff2);
     uint8_t* px = (uint8_t*)(w + L.px);
@@ -258,9 +263,20 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     int32_t* etc = (int32_t*)(w + L.etc);
     float* hbuf = (float*)(w + L.hbuf);
     float* yf = (float*)(w + L.yf);
-    MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? g_tc_min_rows : 0x7fffffff,
-                                  uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
-            "plan + row state");
+    if (logits) {
+        MOE_TRY(moe::launch_layer_front(logits, x_bf16, packed, T, H, I, E, k, topk_idx, gates, perm, pos, offsets,
+                                        uoff1, uoff2, toff1, toff2, poff, etc, prow, xq, sx, xinit,
+                                        dbg ? dbg->xq : nullptr, dbg ? dbg->sx : nullptr, gacc, yacc, flag,
+                                        stream),
+                "route + sort + x quant + plan");
+    } else {
+        MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
+                                   dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
+                "x quant + header check");
+        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? g_tc_min_rows : 0x7fffffff,
+                                      uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
+                "plan + row state");
+    }
     if (use_tc)
         MOE_TRY(moe::launch_planes(xtp, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
@@ -287,6 +303,19 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
             "combine");
 #undef MOE_TRY
     return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, const float* gates,
+                const int32_t* perm, const int32_t* pos, const int32_t* offsets, const void* packed,
+                void* y_bf16, void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
+    g_last_error.clear();
+    return forward_impl(d, nullptr, x_bf16, const_cast<int32_t*>(topk_idx), const_cast<float*>(gates),
+                        const_cast<int32_t*>(perm), const_cast<int32_t*>(pos), const_cast<int32_t*>(offsets),
+                        packed, y_bf16, ws, ws_bytes, dbg, stream);
 }
 
 // Whole-layer workspace: forward workspace, then idx/gates/perm/pos/offsets,
@@ -335,11 +364,30 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
     int32_t* perm = (int32_t*)(w + L.perm);
     int32_t* pos = (int32_t*)(w + L.pos);
     int32_t* offsets = (int32_t*)(w + L.offsets);
+    if (d->T > 0 && d->T < g_tc_min_rows && (long long)d->T * d->k <= moe::kFrontMaxPairs)
+        return forward_impl(d, logits, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
+                            L.idx - L.fwd, dbg, stream);
     if (int rc = moe_route(logits, d->T, d->E, d->k, idx, gates, stream)) return rc;
     if (int rc = moe_sort(idx, d->T, d->k, d->E, perm, pos, offsets, w + L.sortws, L.sort_bytes, stream))
         return rc;
     return moe_forward(d, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
                        L.idx - L.fwd, dbg, stream);
+}
+
+int moe_layer_tables(const moe_dims* d, void* ws, int32_t** topk_idx, float** gates, int32_t** perm,
+                     int32_t** pos, int32_t** offsets) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, true)) return rc;
+    if (!ws || !topk_idx || !gates || !perm || !pos || !offsets)
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_tables: NULL pointer");
+    const LayerWs L = layer_ws(*d, d->T);
+    char* w = (char*)ws;
+    *topk_idx = (int32_t*)(w + L.idx);
+    *gates = (float*)(w + L.gates);
+    *perm = (int32_t*)(w + L.perm);
+    *pos = (int32_t*)(w + L.pos);
+    *offsets = (int32_t*)(w + L.offsets);
+    return MOE_OK;
 }
 
 int moe_quant_rows_f32(const float* v, int rows, int cols, int8_t* q, float* s, cudaStream_t stream) {

@@ -1,0 +1,108 @@
+// The steps before the first expert GEMM of a decode-size layer call, fused
+// into one launch.
+//
+// "DeepSeek-V4-Flash on AMD gfx90a" (abstract) names per-layer
+// synchronisation among the costs of its decode path.  At decode the route,
+// sort, x quant and plan steps each move a few kilobytes, so as separate
+// launches their time is mostly launch and dependency latency.  When no expert
+// can reach the tensor-core threshold (T below it: every expert has at most T
+// rows) and the pairs fit one sort chunk, one launch runs them all, with
+// roles by block:
+//   block 0      routes every token (a warp per token, route_token), sorts the
+//                pairs (sort_cta, expert ids from shared memory) and plans the
+//                streaming units (plan_warp); it also owns the call's error
+//                word (cleared, FLAG_LAYOUT on a packed-header mismatch);
+//   blocks 1..T  x quant of token blockIdx.x - 1 (xquant_row);
+//   the rest     clear the fp64 accumulators of one sorted row each (every
+//                row is a streaming row here).
+// No role reads another's output, so no block waits for another; the first
+// GEMM waits for the whole grid (programmatic dependent launch) exactly as it
+// waited for the four launches this replaces.  The results are the same as
+// those of k_route, k_sort_single, k_xquant and k_plan_rows.
+#include "steps.cuh"
+
+namespace moe {
+
+struct FrontArgs {
+    const float* logits;        // [T, E]
+    const __nv_bfloat16* x;     // [T, H]
+    const void* packed;
+    int T, H, I, E, k;
+    int32_t* topk_idx;          // [T, k]
+    float* gates;               // [T, k]
+    int32_t* perm;              // [P]
+    int32_t* pos;               // [P]
+    int32_t* offsets;           // [E + 1]
+    int32_t *unit_off1, *unit_off2, *tile_off1, *tile_off2, *plane_off, *expert_tc, *plane_row;
+    int8_t* xq;
+    float* sx;
+    int32_t* xinit;
+    int8_t* dbg_xq;
+    float* dbg_sx;
+    double* gacc;               // [P, 2I]
+    double* yacc;               // [P, H]
+    int32_t* flag;
+};
+
+template <int KMAX, int S>
+__global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
+    pdl_begin();
+    const int P = a.T * a.k;
+    if (blockIdx.x == 0) {
+        __shared__ int s_idx[kFrontMaxPairs];
+        __shared__ int hist[kMaxExperts];
+        __shared__ int tmp[kSortThreads + 1];
+        __shared__ int offs[kMaxExperts + 1];
+        __shared__ PlanShared ps;
+        if (threadIdx.x == 0) *a.flag = packed_header_ok(a.packed, a.H, a.I, a.E) ? 0 : FLAG_LAYOUT;
+        const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+        for (int t = warp; t < a.T; t += nwarps)
+            route_token<KMAX, S>(a.logits + (size_t)t * a.E, a.E, a.k, a.topk_idx + (size_t)t * a.k,
+                                 a.gates + (size_t)t * a.k, s_idx + t * a.k);
+        __syncthreads();
+        sort_cta([&](int p) { return s_idx[p]; }, P, a.E, a.perm, a.pos, a.offsets, hist, tmp, offs, a.flag);
+        __syncthreads();
+        // no expert reaches the tensor-core threshold: plan with an unreachable one
+        if (threadIdx.x < 32)
+            plan_warp(offs, a.E, P, 2 * a.I, a.H, 0x7fffffff, a.unit_off1, a.unit_off2, a.tile_off1,
+                      a.tile_off2, a.plane_off, a.expert_tc, a.flag, true, ps);
+        for (int i = threadIdx.x; i < P; i += blockDim.x) a.plane_row[i] = -1;
+        return;
+    }
+    if ((int)blockIdx.x <= a.T) {
+        __shared__ float red[33];
+        __shared__ uint16_t lut[256];
+        xquant_row(a.x, (int)blockIdx.x - 1, a.H, a.xq, a.sx, a.xinit, nullptr, a.dbg_xq, a.dbg_sx, red, lut);
+        return;
+    }
+    const int i = (int)blockIdx.x - 1 - a.T;  // sorted row (grid: 1 + T + P blocks)
+    double2* g = reinterpret_cast<double2*>(a.gacc + (size_t)i * 2 * a.I);
+    for (int j = threadIdx.x; j < a.I; j += blockDim.x) g[j] = make_double2(0.0, 0.0);
+    double2* y = reinterpret_cast<double2*>(a.yacc + (size_t)i * a.H);
+    for (int j = threadIdx.x; j < a.H / 2; j += blockDim.x) y[j] = make_double2(0.0, 0.0);
+}
+
+cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
+                               int E, int k, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
+                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
+                               int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc, int32_t* plane_row,
+                               int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq, float* dbg_sx,
+                               double* gacc, double* yacc, int32_t* flag, cudaStream_t st) {
+    const int P = T * k;
+    if (T < 1 || P > kFrontMaxPairs || E > kMaxExperts) return cudaErrorInvalidValue;
+    FrontArgs a{logits, (const __nv_bfloat16*)x, packed, T, H, I, E, k, topk_idx, gates, perm, pos, offsets,
+                unit_off1, unit_off2, tile_off1, tile_off2, plane_off, expert_tc, plane_row, xq, sx, xinit,
+                dbg_xq, dbg_sx, gacc, yacc, flag};
+    const dim3 grid(1 + T + P), block(kSortThreads);
+    cudaError_t e;
+    if (E <= 256)
+        e = k <= 8 ? launch_pdl(k_layer_front<8, 8>, grid, block, 0, st, a)
+                   : launch_pdl(k_layer_front<16, 8>, grid, block, 0, st, a);
+    else
+        e = k <= 8 ? launch_pdl(k_layer_front<8, 32>, grid, block, 0, st, a)
+                   : launch_pdl(k_layer_front<16, 32>, grid, block, 0, st, a);
+    count_launches(1);
+    return e;
+}
+
+}  // namespace moe

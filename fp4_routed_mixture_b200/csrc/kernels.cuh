@@ -53,6 +53,16 @@ PackedLayout packed_layout(int H, int I, int E);
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
                          cudaStream_t st);
 
+// Route, sort, x quant and plan of a layer call in one launch (front.cu), for
+// calls with no tensor-core expert and at most kFrontMaxPairs pairs.
+constexpr int kFrontMaxPairs = 1024;
+cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
+                               int E, int k, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
+                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
+                               int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc, int32_t* plane_row,
+                               int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq, float* dbg_sx,
+                               double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
+
 size_t sort_workspace_bytes(int T_max, int k, int E);
 cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
                         int32_t* offsets, void* ws, cudaStream_t st);

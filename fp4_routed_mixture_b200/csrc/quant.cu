@@ -13,39 +13,17 @@
 // q = clamp(rne(fp32(v/s)), -127, 127), and q = 0, s = 0 for an all-zero row.
 // xinit/hinit hold -12 * (sum of the 32 codes of each K block): the streaming
 // GEMM decodes weight nibbles to 2*e2m1 + 12 (an unsigned byte), so this term
-// cancels the +12 bias of every block's integer dot product.
-#include "kernels.cuh"
-#include "moe_common.cuh"
+// cancels the +12 bias of every block's integer dot product.  The per-token
+// body of the x quant is xquant_row (steps.cuh).
+#include "steps.cuh"
 
 namespace moe {
 
-constexpr int kQThreads = 256;
-
-__device__ __forceinline__ float block_max(float v, float* red) {
-    v = warp_max(v);
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[w] = v;
-    __syncthreads();
-    if (w == 0) {
-        v = (lane < (int)(blockDim.x >> 5)) ? red[lane] : 0.0f;
-        v = warp_max(v);
-        if (lane == 0) red[32] = v;
-    }
-    __syncthreads();
-    const float r = red[32];
-    __syncthreads();
-    return r;
-}
-
-// One CTA per token; each thread handles chunks of 8 consecutive elements.
-// With tplanes != NULL the token's codes are also written once as E2M1 digit
-// planes in token order: per 32-input block b, 48 bytes at
-// tplanes + (t*(H/32) + b)*48: plane p's 16 bytes at +16p (element 2j of the
-// block in the low nibble of byte j).  The tensor-core GEMM's plane writer
-// copies these pieces into sorted-row order.
-// It is also the first kernel of moe_forward: thread 0 of CTA 0 clears the
-// call's device error word and sets FLAG_LAYOUT when the packed buffer was
-// built for other dims (no other CTA of this kernel touches the word).
+// One CTA per token (xquant_row).  It is also the first kernel of
+// moe_forward: thread 0 of CTA 0 clears the call's device error word and sets
+// FLAG_LAYOUT when the packed buffer was built for other dims (no other CTA of
+// this kernel touches the word).  The tensor-core GEMM's plane writer copies
+// the token-order digit planes (tplanes) into sorted-row order.
 __global__ void __launch_bounds__(kQThreads)
     k_xquant(const __nv_bfloat16* __restrict__ x, int T, int H, int8_t* __restrict__ xq,
              float* __restrict__ sx, int32_t* __restrict__ xinit, uint8_t* __restrict__ tplanes,
@@ -55,67 +33,7 @@ __global__ void __launch_bounds__(kQThreads)
     if (blockIdx.x == 0 && threadIdx.x == 0) *flag = packed_header_ok(packed, H, I, E) ? 0 : FLAG_LAYOUT;
     __shared__ float red[33];
     __shared__ uint16_t lut[256];
-    if (tplanes)
-        for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = (uint16_t)digit_codes((int)(int8_t)v);
-    const int t = blockIdx.x;
-    const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-    const int nchunk = H / 8;
-    float a = 0.0f;
-    for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-        const uint4 v = __ldg(row + c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            a = fmaxf(a, fabsf(__uint_as_float(w[j] << 16)));
-            a = fmaxf(a, fabsf(__uint_as_float(w[j] & 0xffff0000u)));
-        }
-    }
-    a = block_max(a, red);
-    const float s = quant_scale(a);
-    if (threadIdx.x == 0) {
-        sx[t] = s;
-        if (dbg_sx) dbg_sx[t] = s;
-    }
-    // chunks are handed out round-robin, so the 4 chunks of one 32-element
-    // block sit in 4 consecutive lanes of one warp (nchunk % 4 == 0)
-    for (int c0 = 0; c0 < nchunk; c0 += blockDim.x) {
-        const int c = c0 + threadIdx.x;
-        int bsum = 0;
-        if (c < nchunk) {
-            const uint4 v = __ldg(row + c);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t packed[2] = {0u, 0u};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int q0 = quant_code(__uint_as_float(w[j] << 16), a, s);
-                const int q1 = quant_code(__uint_as_float(w[j] & 0xffff0000u), a, s);
-                bsum += q0 + q1;
-                packed[j >> 1] |= ((uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8))
-                                  << (16 * (j & 1));
-            }
-            const uint2 pv = make_uint2(packed[0], packed[1]);
-            reinterpret_cast<uint2*>(xq + (size_t)t * H)[c] = pv;
-            if (dbg_xq) reinterpret_cast<uint2*>(dbg_xq + (size_t)t * H)[c] = pv;
-            if (tplanes) {
-                // 8 codes -> one 32-bit word of each plane (word c % 4 of block c / 4)
-                uint32_t d[3] = {0u, 0u, 0u};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t tc = lut[(packed[e >> 2] >> (8 * (e & 3))) & 0xffu];
-                    d[0] |= (tc & 0xFu) << (4 * e);
-                    d[1] |= ((tc >> 4) & 0xFu) << (4 * e);
-                    d[2] |= (tc >> 8) << (4 * e);
-                }
-                uint32_t* dst = reinterpret_cast<uint32_t*>(tplanes + ((size_t)t * (H / 32) + (c >> 2)) * 48) + (c & 3);
-                dst[0] = d[0];
-                dst[4] = d[1];
-                dst[8] = d[2];
-            }
-        }
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
-        bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
-        if (c < nchunk && (c & 3) == 0) xinit[(size_t)t * (H / 32) + (c >> 2)] = -12 * bsum;
-    }
+    xquant_row(x, blockIdx.x, H, xq, sx, xinit, tplanes, dbg_xq, dbg_sx, red, lut);
 }
 
 // R threads per sorted row (R = 32: a warp per row, for many rows; R = 256:

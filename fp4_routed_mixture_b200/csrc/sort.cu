@@ -14,87 +14,9 @@
 // Expert ids outside [0, E) raise FLAG_BAD_EXPERT and are skipped.
 #include <mutex>
 
-#include "kernels.cuh"
-#include "moe_common.cuh"
+#include "steps.cuh"
 
 namespace moe {
-
-constexpr int kSortChunk = 1024;
-constexpr int kSortThreads = 256;
-
-__device__ __forceinline__ bool valid_expert(int e, int E) { return (unsigned)e < (unsigned)E; }
-
-// Exclusive scan of smem[0..E) in place (blockDim == kSortThreads, E <= 1024);
-// returns the total.  Uses `tmp` [kSortThreads + 1] of shared scratch.
-__device__ int block_exclusive_scan(int* vals, int E, int* tmp) {
-    const int tid = threadIdx.x;
-    const int per = (E + kSortThreads - 1) / kSortThreads;  // <= 4
-    int local[4];
-    int s = 0;
-    for (int j = 0; j < per; ++j) {
-        const int e = tid * per + j;
-        local[j] = (e < E) ? vals[e] : 0;
-        s += local[j];
-    }
-    tmp[tid] = s;
-    __syncthreads();
-    // Hillis-Steele over kSortThreads partial sums
-    for (int o = 1; o < kSortThreads; o <<= 1) {
-        const int v = (tid >= o) ? tmp[tid - o] : 0;
-        __syncthreads();
-        tmp[tid] += v;
-        __syncthreads();
-    }
-    int run = (tid == 0) ? 0 : tmp[tid - 1];
-    const int total = tmp[kSortThreads - 1];
-    __syncthreads();
-    for (int j = 0; j < per; ++j) {
-        const int e = tid * per + j;
-        if (e < E) {
-            vals[e] = run;
-            run += local[j];
-        }
-    }
-    __syncthreads();
-    return total;
-}
-
-// Stable scatter of pairs [p0, p1) (at most 32 x 32 of them) by one warp;
-// cursor[e] is the next free sorted slot of expert e and is advanced in place.
-// The warp first loads all of its expert ids (lane l holds pairs p0 + 32s + l)
-// so the serial steps wait on no global load.
-__device__ void warp_stable_scatter(const int32_t* __restrict__ topk_idx, int p0, int p1, int E,
-                                    int* cursor, int32_t* __restrict__ perm,
-                                    int32_t* __restrict__ pos) {
-    const int lane = threadIdx.x & 31;
-    int ids[32];
-#pragma unroll
-    for (int s = 0; s < 32; ++s) {
-        const int p = p0 + 32 * s + lane;
-        ids[s] = p < p1 ? __ldg(topk_idx + p) : -1;
-    }
-#pragma unroll
-    for (int s = 0; s < 32; ++s) {
-        const int base = p0 + 32 * s;
-        if (base >= p1) break;
-        const int p = base + lane;
-        int e = ids[s];
-        if (p >= p1 || !valid_expert(e, E)) e = -1 - lane;  // unique key: never grouped, never written
-        const uint32_t same = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(same & ((1u << lane) - 1u));
-        const int leader = __ffs(same) - 1;
-        int slot = 0;
-        if (e >= 0) slot = cursor[e];  // all lanes of a group read the same value
-        __syncwarp();
-        if (e >= 0) {
-            const int dst = slot + rank;
-            perm[dst] = p;
-            pos[p] = dst;
-            if (lane == leader) cursor[e] = slot + __popc(same);
-        }
-        __syncwarp();
-    }
-}
 
 __global__ void __launch_bounds__(kSortThreads)
     k_sort_count(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ chunk_hist,
@@ -148,36 +70,19 @@ __global__ void __launch_bounds__(kSortThreads)
     __syncthreads();
     if (threadIdx.x < 32) {
         const int p0 = c * kSortChunk, p1 = min(P, p0 + kSortChunk);
-        warp_stable_scatter(topk_idx, p0, p1, E, cursor, perm, pos);
+        warp_stable_scatter([&](int p) { return (int)__ldg(topk_idx + p); }, p0, p1, E, cursor, perm, pos);
     }
 }
 
-// P <= kSortChunk: histogram, scan and scatter in one CTA.
+// P <= kSortChunk: histogram, scan and scatter in one CTA (sort_cta).
 __global__ void __launch_bounds__(kSortThreads)
     k_sort_single(const int32_t* __restrict__ topk_idx, int P, int E, int32_t* __restrict__ perm,
                   int32_t* __restrict__ pos, int32_t* __restrict__ offsets, int32_t* flag) {
     pdl_begin();
     extern __shared__ int sm[];
-    int* hist = sm;
-    int* tmp = sm + E;
     if (threadIdx.x == 0) *flag = 0;  // this single CTA is the whole sort: it owns the error word
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-    bool bad = false;
-    for (int p = threadIdx.x; p < P; p += blockDim.x) {
-        const int e = __ldg(topk_idx + p);
-        if (valid_expert(e, E))
-            atomicAdd(&hist[e], 1);
-        else
-            bad = true;
-    }
-    if (bad) raise_flag(flag, FLAG_BAD_EXPERT);
-    __syncthreads();
-    const int all = block_exclusive_scan(hist, E, tmp);
-    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = hist[e];
-    if (threadIdx.x == 0) offsets[E] = all;
-    __syncthreads();
-    if (threadIdx.x < 32) warp_stable_scatter(topk_idx, 0, P, E, hist, perm, pos);
+    sort_cta([&](int p) { return (int)__ldg(topk_idx + p); }, P, E, perm, pos, offsets, sm, sm + E, nullptr,
+             flag);
 }
 
 size_t sort_workspace_bytes(int T_max, int k, int E) {

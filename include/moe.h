@@ -198,11 +198,24 @@ int moe_forward(const moe_dims *d, const void *x_bf16, const int32_t *topk_idx,
  * ws: moe_layer_workspace_bytes(d, T_max) bytes, 256-byte aligned, T <= T_max;
  * it holds the forward workspace (device error word first), the routing and
  * sort outputs and the sort scratch.  Asynchronous, graph-capturable.
+ * Decode-size calls (0 < T < MOE_OPT_TC_MIN_ROWS and T * k <= 1024, so that
+ * every expert takes the streaming GEMM) run route, sort, x quant and the
+ * work plan as one fused launch; the results are the same as those of the
+ * separate calls (the same device code runs in both).
  * ------------------------------------------------------------------------- */
 size_t moe_layer_workspace_bytes(const moe_dims *d, int T_max);
 int moe_layer_forward(const moe_dims *d, const float *logits, const void *x_bf16,
                       const void *packed, void *y_bf16, void *ws, size_t ws_bytes,
                       const moe_debug *dbg, cudaStream_t stream);
+
+/* Device pointers to the routing tables moe_layer_forward leaves in its
+ * workspace `ws` for dims d (d->T = the call's T): topk_idx [T, k] and gates
+ * [T, k] as moe_route writes them, perm [T*k], pos [T*k] and offsets [E + 1]
+ * as moe_sort writes them.  Pure pointer arithmetic (nothing is launched or
+ * read); the tables are valid once that call has completed on its stream and
+ * until the next call that uses ws.  MOE_ERR_INVALID_ARG on NULL pointers. */
+int moe_layer_tables(const moe_dims *d, void *ws, int32_t **topk_idx, float **gates,
+                     int32_t **perm, int32_t **pos, int32_t **offsets);
 
 /* Stage entry point: per-row symmetric INT8 quantisation of fp32 rows
  * v [rows, cols] -> q [rows, cols] int8, s [rows] fp32 (rule as for x above). */
