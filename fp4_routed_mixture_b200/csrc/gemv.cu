@@ -6,8 +6,9 @@
 // limits.  On B200 the same regime is HBM-bound: every touched expert's FP4
 // weights are read exactly once, in coalesced 16-byte pieces.
 //
-// Work: for every expert e with M_e > 0, units (tile of 32 weight rows, group
-// of up to kGroup tokens); each unit is K/128 items of 4 scale blocks.  The
+// Work: for every expert e with M_e > 0, units (tile of kGemvTileRows = 64
+// weight rows, group of up to kGroup tokens); each unit is K/128 items of 4
+// scale blocks.  The
 // flat item range is split evenly over all warps of the grid (stream-K), so
 // the load is balanced to within one item whatever the expert counts are.
 //
@@ -16,11 +17,13 @@
 // slices, a warp-wide 512-byte coalesced access per block), the group's
 // activation bytes and block terms -- are in flight while item i is computed.
 //
-// Lane l of a warp owns weight row 32*tile + l and the full dot products of
-// that row with the group's token rows:
-//   * a 16-byte code slice gives the lane one 32-element block (one scale);
-//     the warp's 32 slices of a block are one contiguous 512-byte piece of the
-//     packed chunk (layout in pack.cu);
+// Lane l of a warp owns weight rows 64*tile + l and 64*tile + 32 + l (two
+// independent dot-product chains per lane, which share the activation loads)
+// and their full dot products with the group's token rows:
+//   * a 16-byte code slice gives the lane one 32-element block (one scale) of
+//     one row; the warp's 32 slices of a block are one contiguous 512-byte
+//     piece of the packed chunk, the two rows' pieces are adjacent (layout in
+//     pack.cu);
 //   * nibbles become bytes 2*e2m1 + 12 in [0, 24] through two byte
 //     permutes (positive and negative code tables) and an OR;
 //   * __dp4a against the int8 activation bytes, started from -12 * (sum of
@@ -35,19 +38,27 @@
 
 namespace moe {
 
-// Tuning (measured on B200, decode T=8 and T=64): a 2-deep ring per warp,
-// 32 warps per SM.  Giving a warp two 32-row tiles per item (two weight
-// streams 69 KB apart), deeper rings with fewer warps, more warps with fewer
-// registers, and TMA bulk copies in place of the per-lane 16-byte copies were
-// all slower.  The kernel is bound by integer issue (the nibble decode), at
-// about 0.6 of the measured copy bandwidth.
+// Tuning (measured on B200, decode T=8 and T=64): two adjacent 32-row tiles
+// per warp (a lane owns two rows) with a 2-deep ring, 20 warps per SM (shared
+// memory bound), beat one tile per warp at 32 warps per SM by 5-8% (decode_T8:
+// 3.93 -> 4.19 TB/s): the second row gives every lane a second independent
+// chain and halves the activation loads and the per-item bookkeeping per
+// weight.  Four tiles per warp (11 warps per SM), a 3-deep ring (14 warps),
+// one-tile variants with more or fewer registers, and TMA bulk copies in place
+// of the per-lane 16-byte copies were all slower.  The kernel is bound by
+// integer issue (the nibble decode), at about 0.65 of the measured copy
+// bandwidth.
 constexpr int kGroup = kGemvGroup;  // token rows per unit
 // One warp per CTA, 32 CTAs per SM: every warp runs its own pipeline anyway,
 // and single-warp CTAs measured ~10% faster than 8-warp CTAs at the same 32
 // warps per SM (decode_T8: 3.58 -> 3.96 TB/s; 4 warps/CTA: 3.70).
 constexpr int kGemvWarps = 1;
-constexpr int kStages = 2;         // shared-memory ring depth per warp
-constexpr int kGroupBytes = 2176;  // 4 scale blocks of 32 rows: 128 B scales + 4 x 512 B codes
+constexpr int kStages = 2;                   // shared-memory ring depth per warp
+constexpr int kMinBlocks = 18;               // register budget: CTAs per SM (shared memory allows 20)
+constexpr int TP = kGemvTileRows / 32;       // 32-row tiles per unit: a lane owns TP rows
+static_assert(TP == 1 || TP == 2 || TP == 4, "a lane's scale words are one 4-, 8- or 16-byte copy");
+constexpr int kScaleBytes = 32 * 4 * TP;     // the lanes' scale words (TP per lane)
+constexpr int kGroupBytes = kScaleBytes + 4 * TP * 512;  // + 4 blocks x TP tiles x 512 B codes
 constexpr int kChunkBytes = 8704;  // packed chunk: 4 scale blocks of 128 rows (see pack.cu)
 
 // One ring slot: one K group (4 blocks of 32 elements) of one 32-row tile,
@@ -103,6 +114,9 @@ __device__ __forceinline__ void cp_async16(uint32_t smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async4(uint32_t smem, const void* gmem) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t smem, const void* gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -198,7 +212,7 @@ __device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, 
     return d0 + d1;
 }
 
-__global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
+__global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a) {
     pdl_begin();
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -219,7 +233,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
     // (token lane%4) this lane copies.  In the packed chunk of 8704 bytes the
     // lane's scale word of tile t is at lane*16 + t*4 and its code slice of
     // block j at 512 + j*2048 + t*512 + lane*16.
-    const uint32_t o_sc = lane * 4, o_code = 128 + lane * 16;
+    const uint32_t o_sc = lane * 4 * TP, o_code = kScaleBytes + lane * 16;
     const uint32_t o_x = (uint32_t)offsetof(Slot, x) + (lane >> 3) * 128 + (lane & 7) * 16;
     const uint32_t o_init = (uint32_t)offsetof(Slot, init) + (lane & (kGroup - 1)) * 16;
 
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
     const int32_t* f_i = nullptr;
     uint32_t g_sc = 0, g_code = 0;  // this lane's offsets inside a packed chunk (tile dependent)
     auto start_unit = [&](int kg) {
-        const int rb = fu.tile >> 2, t = fu.tile & 3;
+        const int rb = (fu.tile * TP) >> 2, t = (fu.tile * TP) & 3;
         g_sc = lane * 16 + t * 4;
         g_code = 512 + t * 512 + lane * 16;
         f_w = a.w + (size_t)fu.e * a.expert_bytes + ((size_t)rb * KG + kg) * kChunkBytes;
@@ -243,9 +257,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
     start_unit(f_kg);
     auto issue = [&]() {
         const uint32_t sb = ring_s + f_slot * kSlotBytes;
-        cp_async4(sb + o_sc, f_w + g_sc);
+        if (TP == 4) cp_async16(sb + o_sc, f_w + g_sc);
+        else if (TP == 2) cp_async8(sb + o_sc, f_w + g_sc);
+        else cp_async4(sb + o_sc, f_w + g_sc);
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb) cp_async16(sb + o_code + bb * 512, f_w + g_code + bb * 2048);
+        for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+            for (int u = 0; u < TP; ++u)
+                cp_async16(sb + o_code + (bb * TP + u) * 512, f_w + g_code + bb * 2048 + u * 512);
         if ((lane >> 3) < fu.mc) cp_async16(sb + o_x, f_x);
         if (lane < fu.mc) cp_async16(sb + o_init, f_i);
         cp_async_commit();
@@ -273,44 +292,56 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
     // ---- compute side ----
     Unit cu = unit_at(a, it0 / KG);
     int c_kg = it0 % KG, c_slot = 0;
-    double acc[kGroup];
+    double acc[TP][kGroup];
 #pragma unroll
-    for (int m = 0; m < kGroup; ++m) acc[m] = 0.0;
+    for (int u = 0; u < TP; ++u)
+#pragma unroll
+        for (int m = 0; m < kGroup; ++m) acc[u][m] = 0.0;
     for (int it = it0; it < it1; ++it) {
         if (f_left > 0) issue();
         else cp_async_commit();
         cp_async_wait<kStages - 1>();  // item `it` has landed (this lane's copies) ...
         __syncwarp();                  // ... and every other lane's
         const Slot& sl = ring[c_slot];
-        const uint32_t sw = *reinterpret_cast<const uint32_t*>(sl.w + o_sc);
-#ifndef MOE_GEMV_SPLIT
-#define MOE_GEMV_SPLIT 1
-#endif
-        if (MOE_GEMV_SPLIT && cu.mc == 1) {
+        uint32_t sw[TP];
+#pragma unroll
+        for (int u = 0; u < TP; ++u) sw[u] = *reinterpret_cast<const uint32_t*>(sl.w + o_sc + 4 * u);
+        if (cu.mc == 1) {
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + bb * 512);
                 const uint4 x0 = *reinterpret_cast<const uint4*>(&sl.x[0][bb * 32]);
                 const uint4 x1 = *reinterpret_cast<const uint4*>(&sl.x[0][bb * 32 + 16]);
-                const int d = block_dot_split(tb, c, x0, x1, sl.init[0][bb]);
-                acc[0] = __fma_rn((double)d, block_scale(sw, bb), acc[0]);
+                const int ini = sl.init[0][bb];
+#pragma unroll
+                for (int u = 0; u < TP; ++u) {
+                    const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + (bb * TP + u) * 512);
+                    const int d = block_dot_split(tb, c, x0, x1, ini);
+                    acc[u][0] = __fma_rn((double)d, block_scale(sw[u], bb), acc[u][0]);
+                }
             }
         } else {
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + bb * 512);
-                uint32_t v[8];
-                decode8(tb, c.x, v[0], v[1]);
-                decode8(tb, c.y, v[2], v[3]);
-                decode8(tb, c.z, v[4], v[5]);
-                decode8(tb, c.w, v[6], v[7]);
-                const double sc = block_scale(sw, bb);
+                uint32_t v[TP][8];
+                double sc[TP];
+#pragma unroll
+                for (int u = 0; u < TP; ++u) {
+                    const uint4 c = *reinterpret_cast<const uint4*>(sl.w + o_code + (bb * TP + u) * 512);
+                    decode8(tb, c.x, v[u][0], v[u][1]);
+                    decode8(tb, c.y, v[u][2], v[u][3]);
+                    decode8(tb, c.z, v[u][4], v[u][5]);
+                    decode8(tb, c.w, v[u][6], v[u][7]);
+                    sc[u] = block_scale(sw[u], bb);
+                }
 #pragma unroll
                 for (int m = 0; m < kGroup; ++m) {
                     if (m < cu.mc) {
                         const uint4 x0 = *reinterpret_cast<const uint4*>(&sl.x[m][bb * 32]);
                         const uint4 x1 = *reinterpret_cast<const uint4*>(&sl.x[m][bb * 32 + 16]);
-                        acc[m] = __fma_rn((double)block_dot(v, x0, x1, sl.init[m][bb]), sc, acc[m]);
+                        const int ini = sl.init[m][bb];
+#pragma unroll
+                        for (int u = 0; u < TP; ++u)
+                            acc[u][m] = __fma_rn((double)block_dot(v[u], x0, x1, ini), sc[u], acc[u][m]);
                     }
                 }
             }
@@ -318,11 +349,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 32) k_gemv(GemvArgs a) {
         __syncwarp();  // every lane is done with the slot before it is refilled
         c_slot = (c_slot + 1 == kStages) ? 0 : c_slot + 1;
         if (++c_kg == KG || it + 1 == it1) {
-            const int n = canonical_row(cu.tile * 32 + lane, a.gate_up_half);
 #pragma unroll
-            for (int m = 0; m < kGroup; ++m) {
-                if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.i0 + m) * a.N + n, acc[m]);
-                acc[m] = 0.0;
+            for (int u = 0; u < TP; ++u) {
+                const int n = canonical_row((cu.tile * TP + u) * 32 + lane, a.gate_up_half);
+#pragma unroll
+                for (int m = 0; m < kGroup; ++m) {
+                    if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.i0 + m) * a.N + n, acc[u][m]);
+                    acc[u][m] = 0.0;
+                }
             }
             if (c_kg == KG && it + 1 < it1) {
                 c_kg = 0;

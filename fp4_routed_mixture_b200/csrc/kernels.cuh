@@ -8,10 +8,12 @@
 
 namespace moe {
 
+// Unit of the streaming grouped GEMM: kGemvTileRows weight rows by up to
+// kGemvGroup token rows (shared by it and the planner).
+constexpr int kGemvTileRows = 64;
+constexpr int kGemvGroup = 4;   // 6 and 8 measured slower on decode_T8 and decode_T64
 // Tile of the tensor-core grouped GEMM: 128 weight rows (the MMA's M) by up to
 // 128 sorted token rows (its N); shared by the planner and the kernel.
-// Token rows per unit of the streaming GEMM (shared by it and the planner).
-constexpr int kGemvGroup = 4;   // 6 and 8 measured slower on decode_T8 and decode_T64
 constexpr int kMaxExperts = 1024;   // the API's limit on E
 constexpr int kTcWeightTile = 128;
 constexpr int kTcTokenTile = 128;

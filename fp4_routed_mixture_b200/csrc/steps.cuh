@@ -309,8 +309,8 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 // ---- plan ----------------------------------------------------------------------------
 // Work split per expert: experts with at least tc_min rows go to the
 // tensor-core GEMM (tiles of kTcWeightTile weight rows x kTcTokenTile token
-// rows), the others to the streaming GEMM (units of 32 weight rows x
-// kGemvGroup tokens).  Forms the exclusive scans over experts of the streaming
+// rows), the others to the streaming GEMM (units of kGemvTileRows weight rows
+// x kGemvGroup tokens).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
 // tile starts on a 16-row boundary of the plane buffers), and expert_tc[e] = 1
@@ -343,8 +343,8 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
         const bool tc = m >= tc_min;
         const int g = tc ? 0 : (m + kGemvGroup - 1) / kGemvGroup;
         const int nb = tc ? (m + kTcTokenTile - 1) / kTcTokenTile : 0;
-        c[0] = g * (n1 / 32);
-        c[1] = g * (n2 / 32);
+        c[0] = g * (n1 / kGemvTileRows);
+        c[1] = g * (n2 / kGemvTileRows);
         c[2] = nb * (n1 / kTcWeightTile);
         c[3] = nb * (n2 / kTcWeightTile);
         c[4] = tc ? (m + 15) & ~15 : 0;
