@@ -55,3 +55,24 @@ def test_product_path_does_not_use_the_oracle():
         if path.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
             src = open(path).read()
             assert not re.search(r"(import\s+oracle|from\s+oracle|liboracle|oracle/)", src), path
+
+
+def test_layer_tables_point_into_the_layer_workspace():
+    # pure pointer arithmetic: a fake workspace address is never dereferenced
+    import fp4_routed_mixture_b200 as m
+    lib = m.lib
+    for (T, H, I, E, k) in [(8, 4096, 2048, 256, 6), (1, 128, 128, 1, 1), (31, 128, 128, 1024, 16)]:
+        d = m.binding.moe_dims(T, H, I, E, k)
+        base = 1 << 32
+        ptrs = [ctypes.c_void_p() for _ in range(5)]
+        assert lib.moe_layer_tables(ctypes.byref(d), ctypes.c_void_p(base), *[ctypes.byref(p) for p in ptrs]) == 0
+        off = [p.value - base for p in ptrs]
+        P = T * k
+        sizes = [4 * P, 4 * P, 4 * P, 4 * P, 4 * (E + 1)]   # idx, gates, perm, pos, offsets
+        fwd = m.moe_workspace_bytes(T, H, I, E, k)
+        total = m.moe_layer_workspace_bytes(T, H, I, E, k)
+        assert off[0] >= fwd                                 # after the forward workspace
+        for o, sz, nxt in zip(off, sizes, off[1:] + [total]):
+            assert o % 256 == 0 and o + sz <= nxt
+    null = ctypes.c_void_p()
+    assert m.binding.STATUS[lib.moe_layer_tables(ctypes.byref(d), None, *[ctypes.byref(null)] * 5)] == "MOE_ERR_INVALID_ARG"
