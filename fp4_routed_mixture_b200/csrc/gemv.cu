@@ -61,8 +61,9 @@ constexpr int kScaleBytes = 32 * 4 * TP;     // the lanes' scale words (TP per l
 constexpr int kGroupBytes = kScaleBytes + 4 * TP * 512;  // + 4 blocks x TP tiles x 512 B codes
 constexpr int kChunkBytes = 8704;  // packed chunk: 4 scale blocks of 128 rows (see pack.cu)
 
-// One ring slot: one K group (4 blocks of 32 elements) of one 32-row tile,
-// plus the group's activation bytes and block terms.
+// One ring slot: one K group (4 blocks of 32 elements) of one unit's TP
+// 32-row tiles -- the lanes' scale words, then per block the TP tiles' 512-byte
+// code slices -- plus the group's activation bytes and block terms.
 struct alignas(16) Slot {
     uint8_t w[kGroupBytes];
     int8_t x[kGroup][128];

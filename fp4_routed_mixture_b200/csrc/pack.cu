@@ -17,9 +17,9 @@
 //                 codes (canonical nibble order) of that row and block; i.e. for
 //                 every block j the 128 rows' 16-byte pieces back to back, the
 //                 no-swizzle K-major core-matrix order of the tensor cores
-// A warp of the streaming GEMM (lane = row of a 32-row tile t) reads one
-// 512-byte contiguous slice per block; the tensor-core producer fetches a whole
-// chunk with one bulk copy.
+// A warp of the streaming GEMM (lane l = rows l of two adjacent 32-row tiles t,
+// t + 1) reads two adjacent 512-byte slices, 1 KB contiguous, per block; the
+// tensor-core producer fetches a whole chunk with one bulk copy.
 // Device rows of W2 are its canonical rows.  Device rows of W1 interleave gate
 // and up rows per 32-row tile: device row 32*tau + r is gate row 16*tau + r
 // for r < 16 and up row I + 16*tau + (r - 16) otherwise, so every warp-sized
