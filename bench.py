@@ -79,7 +79,7 @@ class Dist:
             torch.cuda.set_device(self.local if self.world > 1 else 0)
         if self.world > 1:
             import datetime
-            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=300))
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=120))
         if n_expected != self.world:
             print(f"warning: --gpus {n_expected} but WORLD_SIZE {self.world}", file=sys.stderr)
 
