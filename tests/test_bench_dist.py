@@ -63,3 +63,25 @@ def test_whole_job_value_is_weak_scaling():
     assert b.whole_job_value(1, 8, 1000, 200.0) == pytest.approx(40000.0)
     # twice the replicas in the same time: twice the tokens/s
     assert b.whole_job_value(2, 8, 1000, 200.0) == pytest.approx(80000.0)
+
+
+def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    # the committed summaries match their kernels; a summary whose recorded hash
+    # differs from the source (the kernel changed since the capture) gives None
+    import bench
+    assert bench.profiled_traffic("k_gemv_decode_T8.md") > 0
+    assert bench.profiled_traffic("k_tc_gemm_prefill_T4604.md") > 0
+    assert bench.profiled_traffic("no_such_summary.md") is None
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = tmp_path / "kernel.cu"
+    src.write_text("// a kernel\n")
+    import hashlib
+    good = hashlib.sha256(src.read_bytes()).hexdigest()
+    (prof / "ok.md").write_text(f"    kernel_source: kernel.cu\n    kernel_source_sha256: {good}\n"
+                                "    dram_bytes_per_launch: 1234\n")
+    (prof / "stale.md").write_text(f"    kernel_source: kernel.cu\n    kernel_source_sha256: {'0' * 64}\n"
+                                   "    dram_bytes_per_launch: 1234\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("ok.md") == 1234
+    assert bench.profiled_traffic("stale.md") is None
