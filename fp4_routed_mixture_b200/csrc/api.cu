@@ -253,6 +253,9 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
     // an expert has at most T rows, so the tensor-core path is skipped without
     // reading any count when T < tc_min (always so with the fused front)
     const bool use_tc = !logits && T >= g_tc_min_rows;
+    // token rows per streaming-GEMM unit: 2 for small calls (nearly every expert
+    // has one or two rows; the smaller ring slot fits more warps per SM), else 4
+    const int group = T <= moe::kGemvSmallGroupMaxT ? moe::kGemvSmallGroup : moe::kGemvGroup;
     uint8_t* xtp = (uint8_t*)(w + L.xtp);
     int32_t* toff1 = (int32_t*)(w + L.toff1);
     int32_t* toff2 = (int32_t*)(w + L.toff2);
@@ -264,7 +267,8 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
     float* hbuf = (float*)(w + L.hbuf);
     float* yf = (float*)(w + L.yf);
     if (logits) {
-        MOE_TRY(moe::launch_layer_front(logits, x_bf16, packed, T, H, I, E, k, topk_idx, gates, perm, pos, offsets,
+        MOE_TRY(moe::launch_layer_front(logits, x_bf16, packed, T, H, I, E, k, group, topk_idx, gates, perm, pos,
+                                        offsets,
                                         uoff1, uoff2, toff1, toff2, poff, etc, prow, xq, sx, xinit,
                                         dbg ? dbg->xq : nullptr, dbg ? dbg->sx : nullptr, gacc, yacc, flag,
                                         stream),
@@ -274,7 +278,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
         MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? g_tc_min_rows : 0x7fffffff,
-                                      uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
+                                      group, uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
                 "plan + row state");
     }
     if (use_tc)
@@ -282,7 +286,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                             uoff1, E, gacc, flag, I, P, stream), "W1");
+                             uoff1, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
                                     offsets, toff1, E, flag, sx, perm, k, hbuf, stream),
@@ -293,7 +297,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
             "SwiGLU + h quant + h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                             uoff2, E, yacc, flag, 0, P, stream), "W2");
+                             uoff2, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
                                     offsets, toff2, E, flag, sh, perm, 0, yf, stream),

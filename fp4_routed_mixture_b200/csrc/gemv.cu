@@ -48,7 +48,6 @@ namespace moe {
 // of the per-lane 16-byte copies were all slower.  The kernel is bound by
 // integer issue (the nibble decode), at about 0.65 of the measured copy
 // bandwidth.
-constexpr int kGroup = kGemvGroup;  // token rows per unit
 // One warp per CTA, 32 CTAs per SM: every warp runs its own pipeline anyway,
 // and single-warp CTAs measured ~10% faster than 8-warp CTAs at the same 32
 // warps per SM (decode_T8: 3.58 -> 3.96 TB/s; 4 warps/CTA: 3.70).
@@ -64,13 +63,18 @@ constexpr int kChunkBytes = 8704;  // packed chunk: 4 scale blocks of 128 rows (
 // One ring slot: one K group (4 blocks of 32 elements) of one unit's TP
 // 32-row tiles -- the lanes' scale words, then per block the TP tiles' 512-byte
 // code slices -- plus the group's activation bytes and block terms.
+// G = token rows per unit (2 or 4): the slot holds G activation rows, so a
+// smaller group leaves room for more warps per SM.
+template <int G>
 struct alignas(16) Slot {
     uint8_t w[kGroupBytes];
-    int8_t x[kGroup][128];
-    int32_t init[kGroup][4];
+    int8_t x[G][128];
+    int32_t init[G][4];
 };
-constexpr int kSlotBytes = (int)sizeof(Slot);
-constexpr int kSmemBytes = kGemvWarps * kStages * kSlotBytes;
+template <int G>
+constexpr int slot_bytes() { return (int)sizeof(Slot<G>); }
+template <int G>
+constexpr int smem_bytes() { return kGemvWarps * kStages * slot_bytes<G>(); }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
@@ -156,6 +160,7 @@ struct Unit {
     int id, e, tile, i0, mc;
 };
 
+template <int G>
 __device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
     int lo = 0, hi = a.E;  // last e with unit_off[e] <= unit
     while (hi - lo > 1) {
@@ -166,11 +171,11 @@ __device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
     u.id = unit;
     u.e = lo;
     const int r0 = __ldg(a.offsets + lo), r1 = __ldg(a.offsets + lo + 1);
-    const int ngroups = (r1 - r0 + kGroup - 1) / kGroup;
+    const int ngroups = (r1 - r0 + G - 1) / G;
     const int local = unit - __ldg(a.unit_off + lo);
     u.tile = local / ngroups;
-    u.i0 = r0 + (local % ngroups) * kGroup;
-    u.mc = min(kGroup, r1 - u.i0);
+    u.i0 = r0 + (local % ngroups) * G;
+    u.mc = min(G, r1 - u.i0);
     return u;
 }
 
@@ -213,7 +218,16 @@ __device__ __forceinline__ int block_dot_split(const Tables& t, const uint4& c, 
     return d0 + d1;
 }
 
-__global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a) {
+// Warps per SM are bounded by each scheduler's 16 K registers (5 warps of up to
+// 96 registers, 6 of up to 80) and by shared memory (one-warp CTAs with two
+// slots: 21 for G = 4, 22 for G = 2).  G = 4 keeps 86 registers (5 warps per
+// scheduler, 20 per SM); G = 2 is held to at most 80 so that its smaller slots
+// can fill 22 warps.
+template <int G>
+__global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_gemv(GemvArgs a) {
+    constexpr int kGroup = G;
+    using Slot = moe::Slot<G>;
+    constexpr int kSlotBytes = slot_bytes<G>();
     pdl_begin();
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -241,7 +255,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a
     // ---- fetch side: cp.async copies of one item into its slot ----
     int f_left = it1 - it0;
     int f_kg = it0 % KG, f_slot = 0;
-    Unit fu = unit_at(a, it0 / KG);
+    Unit fu = unit_at<G>(a, it0 / KG);
     const uint8_t* f_w = nullptr;  // this lane's sources for the current item
     const int8_t* f_x = nullptr;
     const int32_t* f_i = nullptr;
@@ -274,7 +288,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a
         if (++f_kg == KG) {
             if (f_left > 0) {
                 f_kg = 0;
-                fu = unit_at(a, fu.id + 1);
+                fu = unit_at<G>(a, fu.id + 1);
                 start_unit(0);
             }
         } else {
@@ -291,7 +305,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a
     }
 
     // ---- compute side ----
-    Unit cu = unit_at(a, it0 / KG);
+    Unit cu = unit_at<G>(a, it0 / KG);
     int c_kg = it0 % KG, c_slot = 0;
     double acc[TP][kGroup];
 #pragma unroll
@@ -361,21 +375,22 @@ __global__ void __launch_bounds__(kGemvWarps * 32, kMinBlocks) k_gemv(GemvArgs a
             }
             if (c_kg == KG && it + 1 < it1) {
                 c_kg = 0;
-                cu = unit_at(a, cu.id + 1);
+                cu = unit_at<G>(a, cu.id + 1);
             }
         }
     }
     cp_async_wait<0>();
 }
 
+template <int G>
 static int gemv_grid() {
     static int grid = 0;
     if (!grid) {
         int dev = 0, sms = 0, per_sm = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(k_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv, kGemvWarps * 32, kSmemBytes);
+        cudaFuncSetAttribute(k_gemv<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<G>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv<G>, kGemvWarps * 32, smem_bytes<G>());
         grid = sms * (per_sm > 0 ? per_sm : 1);
     }
     return grid;
@@ -384,10 +399,12 @@ static int gemv_grid() {
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, int P, cudaStream_t st) {
+                        const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st) {
     GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
                gate_up_half, P, 0u};
-    const cudaError_t e = launch_pdl(k_gemv, dim3(gemv_grid()), dim3(kGemvWarps * 32), kSmemBytes, st, a);
+    const cudaError_t e =
+        group == 2 ? launch_pdl(k_gemv<2>, dim3(gemv_grid<2>()), dim3(kGemvWarps * 32), smem_bytes<2>(), st, a)
+                   : launch_pdl(k_gemv<4>, dim3(gemv_grid<4>()), dim3(kGemvWarps * 32), smem_bytes<4>(), st, a);
     count_launches(1);
     return e;
 }

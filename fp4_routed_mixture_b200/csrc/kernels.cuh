@@ -12,6 +12,8 @@ namespace moe {
 // kGemvGroup token rows (shared by it and the planner).
 constexpr int kGemvTileRows = 64;
 constexpr int kGemvGroup = 4;   // 6 and 8 measured slower on decode_T8 and decode_T64
+constexpr int kGemvSmallGroup = 2;       // token rows per unit for calls with T <= kGemvSmallGroupMaxT
+constexpr int kGemvSmallGroupMaxT = 16;
 // Tile of the tensor-core grouped GEMM: 128 weight rows (the MMA's M) by up to
 // 128 sorted token rows (its N); shared by the planner and the kernel.
 constexpr int kMaxExperts = 1024;   // the API's limit on E
@@ -22,7 +24,7 @@ constexpr int kTcTokenTile = 128;
 void count_launches(int n);
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
-                             int I, int H, int tc_min, int32_t* unit_off1, int32_t* unit_off2,
+                             int I, int H, int tc_min, int group, int32_t* unit_off1, int32_t* unit_off2,
                              int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc,
                              int32_t* plane_row, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
 
@@ -59,7 +61,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk
 // calls with no tensor-core expert and at most kFrontMaxPairs pairs.
 constexpr int kFrontMaxPairs = 1024;
 cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
-                               int E, int k, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
+                               int E, int k, int group, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
                                int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
                                int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc, int32_t* plane_row,
                                int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq, float* dbg_sx,
@@ -98,7 +100,7 @@ cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, flo
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, int P, cudaStream_t st);
+                        const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st);
 
 size_t tc_smem_bytes();
 // Digit planes, per 128-input stage g and group of 8 plane rows, hold

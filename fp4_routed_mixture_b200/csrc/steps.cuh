@@ -310,7 +310,7 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 // Work split per expert: experts with at least tc_min rows go to the
 // tensor-core GEMM (tiles of kTcWeightTile weight rows x kTcTokenTile token
 // rows), the others to the streaming GEMM (units of kGemvTileRows weight rows
-// x kGemvGroup tokens).  Forms the exclusive scans over experts of the streaming
+// x `group` tokens, the group size the streaming GEMM is launched with).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
 // tile starts on a 16-row boundary of the plane buffers), and expert_tc[e] = 1
@@ -324,6 +324,7 @@ struct PlanShared {
 };
 
 static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
+                                 int group,
                                  int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                                  int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                                  int32_t* __restrict__ plane_off, int32_t* __restrict__ expert_tc, int32_t* flag,
@@ -341,7 +342,7 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
     auto counts = [&](int e, int (&c)[NS]) {
         const int m = any_bad ? 0 : offsets[e + 1] - offsets[e];
         const bool tc = m >= tc_min;
-        const int g = tc ? 0 : (m + kGemvGroup - 1) / kGemvGroup;
+        const int g = tc ? 0 : (m + group - 1) / group;
         const int nb = tc ? (m + kTcTokenTile - 1) / kTcTokenTile : 0;
         c[0] = g * (n1 / kGemvTileRows);
         c[1] = g * (n2 / kGemvTileRows);
