@@ -12,13 +12,13 @@ same names.  Build the library with ``python fp4_routed_mixture_b200/build.py``.
 """
 from .binding import (FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_BOUNDS, FLAG_LAYOUT, FLAG_TIMEOUT,
                       LIB_PATH, SYMBOLS, MoeError, lib, moe_check_device_flag, moe_forward,
-                      moe_pack_weights, moe_packed_bytes, moe_quant_rows_f32, moe_route, moe_sort,
+                      moe_pack_weights, moe_packed_bytes, moe_quant_rows_f32, moe_route, moe_router_logits, moe_sort,
                       moe_sort_workspace_bytes, moe_unpack_weights, moe_workspace_bytes,
                       moe_exp_f32, moe_swiglu_f32, moe_layer_forward, moe_layer_tables,
                       moe_layer_workspace_bytes, make_debug, moe_launch_count,
                       moe_set_option, moe_get_option, MOE_OPT_TC_MIN_ROWS,
                       moe_sort_static)
 
-__all__ = ["moe_layer_forward", "moe_layer_tables", "moe_layer_workspace_bytes", "make_debug", "moe_pack_weights", "moe_unpack_weights", "moe_route", "moe_sort", "moe_forward",
+__all__ = ["moe_layer_forward", "moe_layer_tables", "moe_layer_workspace_bytes", "make_debug", "moe_pack_weights", "moe_unpack_weights", "moe_router_logits", "moe_route", "moe_sort", "moe_forward",
            "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32", "moe_check_device_flag", "moe_packed_bytes", "moe_workspace_bytes",
            "moe_sort_workspace_bytes", "MoeError", "LIB_PATH", "SYMBOLS", "lib"]

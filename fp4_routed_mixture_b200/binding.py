@@ -23,7 +23,7 @@ FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_LAYOUT, FLAG_TIMEOUT, FLAG_BOUNDS = 1, 2, 
 
 # Exported symbols of include/moe.h, in declaration order.
 SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack_weights",
-           "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_sort_static", "moe_workspace_bytes",
+           "moe_router_logits", "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_sort_static", "moe_workspace_bytes",
            "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_tables",
            "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
            "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
@@ -56,6 +56,7 @@ def _load():
         "moe_packed_bytes": ([D], sz),
         "moe_pack_weights": ([D, vp, vp, vp, vp, vp, vp], i32),
         "moe_unpack_weights": ([D, vp, vp, vp, vp, vp, vp], i32),
+        "moe_router_logits": ([vp, vp, vp, i32, i32, i32, vp, vp], i32),
         "moe_route": ([vp, i32, i32, i32, vp, vp, vp], i32),
         "moe_sort_workspace_bytes": ([i32, i32, i32], sz),
         "moe_sort": ([vp, i32, i32, i32, vp, vp, vp, vp, sz, vp], i32),
@@ -162,6 +163,16 @@ def moe_unpack_weights(packed, H: int, I: int, E: int, stream=None):
     _check(lib.moe_unpack_weights(ctypes.byref(d), _ptr(packed), _ptr(w1c), _ptr(w1s), _ptr(w2c),
                                   _ptr(w2s), _stream(stream)))
     return w1c, w1s, w2c, w2s
+
+
+def moe_router_logits(x, w_router, bias=None, out=None, stream=None):
+    """x [T,H] bf16, w_router [E,H] fp32, bias [E] fp32 or None -> logits [T,E] fp32."""
+    T, H = x.shape
+    E = w_router.shape[0]
+    if out is None:
+        out = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    _check(lib.moe_router_logits(_ptr(x), _ptr(w_router), _ptr(bias), T, H, E, _ptr(out), _stream(stream)))
+    return out
 
 
 def moe_route(logits, k: int, out=None, stream=None):

@@ -148,6 +148,21 @@ int moe_unpack_weights(const moe_dims* d, const void* packed, uint8_t* w1_codes,
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_unpack_weights launch");
 }
 
+int moe_router_logits(const void* x_bf16, const float* w_router, const float* bias, int T, int H, int E,
+                      float* logits, cudaStream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: T < 0");
+    if (H <= 0 || H % 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_logits: H must be a positive multiple of 32");
+    if (E < 1 || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_logits: E must be in [1, 1024]");
+    if ((long long)T * H >= (1LL << 40) || (long long)T * E >= (1LL << 31))
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_router_logits: T too large");
+    if (T > 0 && (!x_bf16 || !w_router || !logits)) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: NULL pointer");
+    if (!aligned(x_bf16, 16) || !aligned(w_router, 16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: x and w_router need 16-byte alignment");
+    cudaError_t e = moe::launch_router_logits(x_bf16, w_router, bias, T, H, E, logits, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_router_logits launch");
+}
+
 int moe_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
               cudaStream_t stream) {
     g_last_error.clear();

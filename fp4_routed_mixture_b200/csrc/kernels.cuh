@@ -56,6 +56,8 @@ PackedLayout packed_layout(int H, int I, int E);
 
 cudaError_t launch_route(const float* logits, int T, int E, int k, int32_t* topk_idx, float* gates,
                          cudaStream_t st);
+cudaError_t launch_router_logits(const void* x, const float* wr, const float* bias, int T, int H, int E,
+                                 float* logits, cudaStream_t st);
 
 // Route, sort, x quant and plan of a layer call in one launch (front.cu), for
 // calls with no tensor-core expert and at most kFrontMaxPairs pairs.

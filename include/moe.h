@@ -120,6 +120,20 @@ int moe_unpack_weights(const moe_dims *d, const void *packed, uint8_t *w1_codes,
                        cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Router projection ([B]: one logit per routed expert), in front of routing:
+ *   logits[t, e] = sum_h x[t, h] * w_router[e, h] (+ bias[e])
+ * x [T, H] bf16 (16-byte aligned), w_router [E, H] fp32 (16-byte aligned),
+ * bias [E] fp32 or NULL, logits [T, E] fp32; all device pointers owned by the
+ * caller.  fp32 fused multiply-adds in ascending h: |logits - S| <=
+ * gamma_(H+1) * sum_h |x w| plus one rounding of the bias addition, where S is
+ * the exact value and gamma_n = n u / (1 - n u), u = 2^-24.  H % 32 == 0,
+ * 1 <= E <= 1024.  Asynchronous, graph-capturable; MOE_ERR_INVALID_ARG on NULL
+ * or misaligned pointers, MOE_ERR_UNSUPPORTED_SHAPE on other shapes.
+ * ------------------------------------------------------------------------- */
+int moe_router_logits(const void *x_bf16, const float *w_router, const float *bias, int T, int H,
+                      int E, float *logits, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Routing ([B]: each token picks k of E routed experts).
  * logits [T, E] fp32 -> topk_idx [T, k] int32, gates [T, k] fp32.
  * topk_idx[t] lists the k largest logits in descending order, equal logits

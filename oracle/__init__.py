@@ -46,6 +46,7 @@ def _L():
         _lib.orc_quant_rows.argtypes = [vp, i64, i32, vp, vp]
         _lib.orc_quant_x.argtypes = [vp, i32, i32, vp, vp, i32]
         _lib.orc_route.argtypes = [vp, i32, i32, i32, vp, vp]
+        _lib.orc_router_logits.argtypes = [vp, vp, vp, i32, i32, i32, vp, i32]
         _lib.orc_sort.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp]
         _lib.orc_sort.restype = i32
         _lib.orc_row_dot.argtypes, _lib.orc_row_dot.restype = [vp, vp, vp, i32], d
@@ -116,6 +117,19 @@ def quant_x(x_bf16: np.ndarray):
     s = np.empty(T, np.float32)
     _L().orc_quant_x(_p(x), T, H, _p(q), _p(s), nthreads())
     return q, s
+
+
+def router_logits(x_bits: np.ndarray, wr: np.ndarray, bias: np.ndarray | None = None) -> np.ndarray:
+    """S[t,e] = sum_h x[t,h] * wr[e,h] (+ bias[e]) in fp64; x as raw bf16 bits."""
+    x = _c(x_bits, np.uint16)
+    w = _c(wr, np.float32)
+    T, H = x.shape
+    E = w.shape[0]
+    assert w.shape[1] == H
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((T, E), np.float64)
+    _L().orc_router_logits(_p(x), _p(w), None if b is None else _p(b), T, H, E, _p(out), nthreads())
+    return out
 
 
 def route(logits: np.ndarray, k: int):

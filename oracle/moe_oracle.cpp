@@ -281,6 +281,24 @@ void orc_quant_x(const uint16_t* x, int T, int H, int8_t* xq, float* sx, int nth
     });
 }
 
+// Step 1, the router projection in front of the path (the layer takes its
+// logits as an input; this is the reference for the router kernel).  Reading:
+// the router is a plain linear map of the bf16 activations with fp32 weights,
+// one logit per routed expert ("DeepSeek V4 Flash on 8x R9600D", model facts:
+// 256 routed experts):
+//   S[t, e] = sum_h x[t, h] * Wr[e, h] + b[e],
+// in fp64, h in ascending order, x decoded from bf16 exactly, b optional (NULL
+// = no bias).  x: raw bf16 bits [T, H]; Wr [E, H] fp32; out [T, E] fp64.
+void orc_router_logits(const uint16_t* x, const float* wr, const float* bias, int T, int H, int E, double* out,
+                       int nthreads) {
+    parallel_for((int64_t)T * E, nthreads, [&](int64_t te) {
+        const int64_t t = te / E, e = te % E;
+        double s = 0.0;
+        for (int h = 0; h < H; ++h) s += (double)bf16_bits_to_float(x[t * H + h]) * (double)wr[e * H + h];
+        out[te] = bias ? s + (double)bias[e] : s;
+    });
+}
+
 void orc_route(const float* logits, int T, int E, int k, int32_t* idx, double* gates) {
     for (int t = 0; t < T; ++t)
         route_token(logits + (int64_t)t * E, E, k, idx + (int64_t)t * k, gates + (int64_t)t * k);

@@ -131,6 +131,56 @@ def test_quant_error_bound_random():
 
 # ---- routing ------------------------------------------------------------------------
 
+# ---- router projection (the reference of the router kernel) ------------------------------
+
+def _bf16_bits(v):
+    """bf16 bits of fp32 values that bf16 holds exactly (small integers, 0, 1)."""
+    b = (np.asarray(v, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(synth.bf16_to_f32(b), np.asarray(v, np.float32))
+    return b
+
+
+def test_router_integer_case_equals_int64_matmul():
+    # small integers are exact in bf16 (|v| <= 256) and fp32, and every partial
+    # sum stays far below 2^53: the fp64 sum is exact and must equal numpy's
+    # int64 matrix product plus the (integer) bias
+    rng = np.random.default_rng(5)
+    T, H, E = 7, 96, 5
+    xi = rng.integers(-8, 9, size=(T, H))
+    wi = rng.integers(-50, 51, size=(E, H))
+    bi = rng.integers(-1000, 1001, size=E)
+    got = oracle.router_logits(_bf16_bits(xi.astype(np.float32)), wi.astype(np.float32), bi.astype(np.float32))
+    assert np.array_equal(got, (xi @ wi.T + bi).astype(np.float64))
+
+
+def test_router_one_hot_rows_pick_weight_columns():
+    # x[t] = e_{h_t}: S[t, e] = Wr[e, h_t] exactly (a transposed or shifted
+    # operand fails this on a non-square shape); x = 0 gives the bias
+    rng = np.random.default_rng(6)
+    T, H, E = 5, 40, 3
+    wr = rng.standard_normal((E, H)).astype(np.float32)
+    hs = [0, 7, 39, 12, 7]
+    x = np.zeros((T + 1, H), np.float32)
+    for t, h in enumerate(hs):
+        x[t, h] = 1.0
+    b = rng.standard_normal(E).astype(np.float32)
+    got = oracle.router_logits(_bf16_bits(x), wr, b)
+    for t, h in enumerate(hs):
+        assert np.array_equal(got[t], wr[:, h].astype(np.float64) + b.astype(np.float64))
+    assert np.array_equal(got[T], b.astype(np.float64))
+    assert np.array_equal(oracle.router_logits(_bf16_bits(x), wr)[T], np.zeros(E))
+
+
+def test_router_matches_harness_logits(workload_data):
+    # the harness rounds the same fp64 sum to fp32 once: they must agree to
+    # within that rounding on a workload
+    w = synth.WORKLOADS["tiny_T4"]
+    d = workload_data("tiny_T4")
+    wr = synth.router_weight(w.seed, w.E, w.H)
+    got = oracle.router_logits(d["x"], wr)
+    assert np.array_equal(got.astype(np.float32), d["logits"])
+
+
 def test_route_matches_full_stable_sort_with_ties():
     rng = np.random.default_rng(3)
     for E, k in [(16, 2), (16, 16), (256, 6), (7, 3)]:
