@@ -314,6 +314,7 @@ def moe_swiglu_f32(g, u, stream=None):
 
 
 MOE_OPT_TC_MIN_ROWS = 1
+MOE_OPT_TC_PAIR = 2
 
 
 def moe_set_option(option: int, value: int):

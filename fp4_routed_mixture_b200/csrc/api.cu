@@ -55,6 +55,8 @@ int check_dims(const moe_dims* d, bool need_T) {
 // Experts with at least this many rows use the tensor-core GEMM (see
 // moe_set_option); the others the streaming GEMM.
 int g_tc_min_rows = 32;
+// Tensor-core GEMM in SM pairs (cta_group::2) where the shape allows (MOE_OPT_TC_PAIR).
+int g_tc_pair = 0;
 
 struct WsLayout {
     size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xtp, xinit, hq, sh, hinit, px, ph,
@@ -304,7 +306,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
                              uoff1, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, stream),
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, g_tc_pair != 0, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, prow, L.plane_rows, ph, P, k, E, I, hq,
@@ -315,7 +317,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
                              uoff2, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, stream),
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, g_tc_pair != 0, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, yf, etc, topk_idx, sh, gates, pos, T, k, E, H, y_bf16, flag, stream),
@@ -440,11 +442,17 @@ int moe_set_option(int option, int value) {
         g_tc_min_rows = value;
         return MOE_OK;
     }
+    if (option == MOE_OPT_TC_PAIR) {
+        if (value != 0 && value != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_PAIR must be 0 or 1");
+        g_tc_pair = value;
+        return MOE_OK;
+    }
     return fail(MOE_ERR_INVALID_ARG, "moe_set_option: unknown option %d", option);
 }
 
 int moe_get_option(int option) {
     if (option == MOE_OPT_TC_MIN_ROWS) return g_tc_min_rows;
+    if (option == MOE_OPT_TC_PAIR) return g_tc_pair;
     return -1;
 }
 

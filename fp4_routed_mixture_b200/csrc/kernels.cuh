@@ -118,7 +118,7 @@ cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, in
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
-                           const float* row_scale, const int32_t* perm, int k_div, float* out,
+                           const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
                            cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,

@@ -197,6 +197,66 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---- the SM-pair form (cta_group::2) ----------------------------------------
+// Two CTAs of a cluster share one MMA: the even CTA issues it with M = 256; each
+// CTA supplies its own 128 weight rows (A) and half of the token rows (B) from
+// the same shared-memory offsets, and each CTA's TMEM receives the accumulator
+// rows of its own weight rows.
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t bar, uint32_t rank) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_addr(bar, rank))
+                 : "memory");
+}
+__device__ __forceinline__ void store_peer_u32(uint32_t addr, uint32_t rank, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_addr(addr, rank)), "r"(v) : "memory");
+}
+// Waits on barriers that CTA-pair operations arrive on use cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// tcgen05.commit of the pair's MMAs, arriving on the barrier at this offset in
+// both CTAs.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_mxf4_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 // Shared-memory matrix descriptor, no swizzle, K-major: 8-row x 16-byte core
 // matrices; lbo = byte distance between the two K-adjacent core matrices of one
 // MMA, sbo = byte distance between 8-row groups.  Bit 46 marks the sm100 format.
@@ -210,6 +270,7 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uin
 
 // Instruction descriptor of kind::mxf4 block-scaled MMA: E2M1 x E2M1, UE8M0
 // scales, fp32 accumulate, both operands K-major, M = 128, K = 64.
+template <int M = TC_BM>
 __device__ __forceinline__ uint32_t make_idesc(int n, int a_sf_id, int b_sf_id) {
     uint32_t d = 0;
     d |= (uint32_t)(b_sf_id & 3) << 4;
@@ -217,7 +278,7 @@ __device__ __forceinline__ uint32_t make_idesc(int n, int a_sf_id, int b_sf_id) 
     d |= 1u << 10;                         // B format: E2M1
     d |= (uint32_t)(n >> 3) << 17;         // N / 8
     d |= 1u << 23;                         // scale format UE8M0
-    d |= (uint32_t)(TC_BM >> 4) << 24;     // M / 16
+    d |= (uint32_t)(M >> 4) << 24;         // M / 16 (the pair form: 256)
     d |= (uint32_t)(a_sf_id & 3) << 29;
     return d;
 }
@@ -246,6 +307,17 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     return tt;
 }
 
+// PAIR = false: one CTA per SM, 128-row tiles.  PAIR = true: clusters of two
+// CTAs; the pair takes the adjacent 128-row tiles 2m (even CTA) and 2m + 1
+// (odd CTA) of one expert and token tile and computes them with M = 256 MMAs
+// issued by the even CTA.  Each CTA loads its own A chunk and half of the
+// tile's token rows (B), so a stage moves 8.7 KB + 12.3 KB into each SM
+// instead of 8.7 KB + 24.6 KB.  Roles in the pair: the odd CTA's MMA warps
+// relay "stage landed" to the even CTA (its copies complete on its own
+// barrier; a remote arrive joins the even CTA's), the even CTA's MMA commits
+// arrive on the barriers of both CTAs, and the odd CTA's epilogue warps release
+// accumulators with remote arrives.
+template <bool PAIR>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     pdl_begin();
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
@@ -253,22 +325,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KG = a.K / 128;
     const int total = __ldg(a.tile_off + a.E);
+    // (both CTAs of a pair read the same values, so they leave together)
     if (*(volatile int32_t*)a.flag & FLAG_LAYOUT) return;
     if (total == 0) return;
-    // this CTA's tiles: t_j = blockIdx.x + j * gridDim.x, j < ntiles; tile j
-    // belongs to pipe j % TC_PIPES and accumulator j % TC_ACC
-    const int ntiles = (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u, peer = rank ^ 1u;
+    const bool leader = rank == 0;
+    // work units: tiles (PAIR: pairs of tiles), unit u_j = unit0 + j * nunits,
+    // j < ntiles; unit j belongs to pipe j % TC_PIPES and accumulator j % TC_ACC
+    const int unit0 = PAIR ? (int)blockIdx.x >> 1 : (int)blockIdx.x;
+    const int nunits = PAIR ? (int)gridDim.x >> 1 : (int)gridDim.x;
+    const int units = PAIR ? total / 2 : total;
+    const int ntiles = unit0 < units ? (units - unit0 + nunits - 1) / nunits : 0;
+    auto tile_of = [&](int j) { return PAIR ? 2 * (unit0 + j * nunits) + (int)rank : unit0 + j * nunits; };
 
     // ---- set-up: barriers, constant plane scales, TMEM ----
     if (threadIdx.x == 0) {
         for (int r = 0; r < TC_PIPES; ++r)
             for (int s = 0; s < TC_STAGES; ++s) {
-                mbar_init(smem_u32(&sh.full[r][s]), 1);
+                // the even CTA of a pair also waits for the odd CTA's relay
+                mbar_init(smem_u32(&sh.full[r][s]), PAIR && leader ? 2 : 1);
                 mbar_init(smem_u32(&sh.empty[r][s]), 1);
             }
         for (int b = 0; b < TC_ACC; ++b) {
             mbar_init(smem_u32(&sh.acc_full[b]), 1);
-            mbar_init(smem_u32(&sh.acc_empty[b]), TC_EPI_WARPS);
+            mbar_init(smem_u32(&sh.acc_empty[b]), PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
         }
         for (int r = 0; r < TC_PIPES; ++r) mbar_init(smem_u32(&sh.drain[r]), 1);
         sh.abort = 0;
@@ -278,20 +358,43 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         sh.sfb[i / 512][i % 512] = (uint8_t)(133 - 3 * (i / 512));  // 2^6, 2^3, 2^0
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(&sh.tmem_base)),
-                     "r"(TC_TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&sh.tmem_base)),
+                         "r"(TC_TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(&sh.tmem_base)),
+                         "r"(TC_TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // the peer's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
     volatile int32_t* abort = &sh.abort;
     auto give_up = [&]() {
         *abort = 1;
+        if (PAIR) store_peer_u32(smem_u32(&sh.abort), peer, 1u);
         raise_flag(a.flag, FLAG_TIMEOUT);
+    };
+    // bounded waits; barriers that pair operations arrive on are read at
+    // cluster scope
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (!PAIR) return mbar_wait(bar, parity, abort);
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        const uint64_t t0 = global_ns();
+        for (;;) {
+            for (int i = 0; i < 64; ++i)
+                if (mbar_try_wait_cluster(bar, parity)) return true;
+            if (*abort) return false;
+            if (global_ns() - t0 > 1000000000ull) return false;
+        }
     };
 
     if (warp < TC_PIPES) {
@@ -302,16 +405,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         bool filled[TC_STAGES] = {};
         uint32_t fill_parity[TC_STAGES] = {};
         for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
-            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
+            const TcTile tt = tile_at(a, tile_of(j));
             const uint8_t* wsrc = a.w + (size_t)tt.e * a.expert_bytes + (size_t)tt.rb * KG * TC_A_BYTES;
-            const uint32_t bbytes = (uint32_t)(tt.n_mma / 8) * kPlaneGroupBytes;  // B of one stage
+            // token rows this CTA supplies: all of them, or its half of the pair's
+            const int nb_rows = PAIR ? tt.n_mma / 2 : tt.n_mma;
+            const int b_row0 = tt.pr0 + (PAIR ? (int)rank * nb_rows : 0);
+            const uint32_t bbytes = (uint32_t)(nb_rows / 8) * kPlaneGroupBytes;  // B of one stage
             // the tile's rows must lie inside the plane buffer (a plane_off
             // table that did not come from the planner is refused here)
             const bool rows_ok = tt.pr0 >= 0 && (tt.pr0 & 15) == 0 && tt.pr0 + tt.n_mma <= a.plane_rows;
             if (!rows_ok && lane == 0) raise_flag(a.flag, FLAG_BOUNDS);
             for (int g = 0; g < KG; ++g) {
                 const uint32_t fb = smem_u32(&sh.full[r][stage]), eb = smem_u32(&sh.empty[r][stage]);
-                if (!mbar_wait(eb, phase ^ 1u, abort)) {
+                if (!wait(eb, phase ^ 1u)) {
                     give_up();
                     break;
                 }
@@ -321,7 +427,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                         mbar_expect_tx(fb, TC_A_BYTES + bbytes);
                         bulk_g2s(sbase, wsrc + (size_t)g * TC_A_BYTES, TC_A_BYTES, fb);
                         const uint8_t* src =
-                            a.planes + ((size_t)g * (a.plane_rows / 8) + tt.pr0 / 8) * kPlaneGroupBytes;
+                            a.planes + ((size_t)g * (a.plane_rows / 8) + b_row0 / 8) * kPlaneGroupBytes;
                         bulk_g2s(sbase + TC_A_BYTES, src, bbytes, fb);
                     } else {
                         mbar_arrive(fb);  // keep the ring moving; the tile's result is not used
@@ -340,23 +446,59 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         // normal path the MMA warp has already waited for all of them)
         for (int s = 0; s < TC_STAGES; ++s)
             if (filled[s]) mbar_wait_bounded(smem_u32(&sh.full[r][s]), fill_parity[s]);
+    } else if (warp < TC_EPI_WARP0 && PAIR && !leader) {
+        // ---------------- relay of pipe r (odd CTA of a pair) ----------------
+        // Passes "this CTA's half of the stage has landed" to the even CTA,
+        // stage by stage in the producer's order, then waits for the pair's
+        // last MMAs (they write this CTA's TMEM) before the CTA may free it.
+        const int r = warp - TC_PIPES;
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
+            bool ok = true;
+            for (int g = 0; g < KG; ++g) {
+                if (!wait(smem_u32(&sh.full[r][stage]), phase)) {
+                    give_up();
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_peer(smem_u32(&sh.full[r][stage]), peer);
+                __syncwarp();
+                if (++stage == TC_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+        }
+        if (lane == 0 && ntiles > r) {
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait_cluster(smem_u32(&sh.drain[r]), 0))
+                if (global_ns() - t0 > 1000000000ull) break;
+        }
+        __syncwarp();
     } else if (warp < TC_EPI_WARP0) {
-        // ---------------- MMA issuer of pipe r ----------------
+        // ---------------- MMA issuer of pipe r (even CTA of a pair) ----------------
         const int r = warp - TC_PIPES;
         const uint32_t sfa_col = tmem + TC_SF_COL + TC_SF_PIPE_COLS * r;
         const uint32_t sfb_col = sfa_col + 4 * TC_STAGES;
         if (lane == 0) {
-            for (int p = 0; p < 3; ++p)
-                tc_cp_sf(sfb_col + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
+            for (int p = 0; p < 3; ++p) {
+                if (PAIR)
+                    tc_cp_sf_pair(sfb_col + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
+                else
+                    tc_cp_sf(sfb_col + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
+            }
         }
         __syncwarp();
         int stage = 0;
         uint32_t phase = 0;
+        int issued = 0;
         for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
-            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
+            const TcTile tt = tile_at(a, tile_of(j));
             const int buf = j % TC_ACC;
             const uint32_t use = (uint32_t)(j / TC_ACC);
-            if (!mbar_wait(smem_u32(&sh.acc_empty[buf]), (use & 1u) ^ 1u, abort)) {
+            if (!wait(smem_u32(&sh.acc_empty[buf]), (use & 1u) ^ 1u)) {
                 give_up();
                 break;
             }
@@ -364,7 +506,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             const uint32_t dcol = tmem + buf * TC_BN;
             bool ok = true;
             for (int g = 0; g < KG; ++g) {
-                if (!mbar_wait(smem_u32(&sh.full[r][stage]), phase, abort)) {
+                if (!wait(smem_u32(&sh.full[r][stage]), phase)) {
                     give_up();
                     ok = false;
                     break;
@@ -373,7 +515,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                 if (lane == 0) {
                     const uint32_t sbase = smem_u32(sh.stage[r][stage]);
                     const uint32_t sfa = sfa_col + 4 * stage;
-                    tc_cp_sf(sfa, make_sdesc(sbase, 0, 128));
+                    if (PAIR)
+                        tc_cp_sf_pair(sfa, make_sdesc(sbase, 0, 128));
+                    else
+                        tc_cp_sf(sfa, make_sdesc(sbase, 0, 128));
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
                         const uint64_t adesc = make_sdesc(sbase + 512 + ks * 2 * 2048, 2048, 128);
@@ -383,11 +528,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                             // matrices 128 bytes apart, 8-row groups 1536 apart
                             const uint64_t bdesc = make_sdesc(sbase + TC_A_BYTES + p * 512 + ks * 256, 128,
                                                               kPlaneGroupBytes);
-                            const uint32_t idesc = make_idesc(tt.n_mma, 2 * ks, 0);
-                            tc_mma_mxf4(dcol, adesc, bdesc, idesc, sfa, sfb_col + 4 * p, (g | ks | p) != 0);
+                            if (PAIR)
+                                tc_mma_mxf4_pair(dcol, adesc, bdesc, make_idesc<2 * TC_BM>(tt.n_mma, 2 * ks, 0), sfa,
+                                                 sfb_col + 4 * p, (g | ks | p) != 0);
+                            else
+                                tc_mma_mxf4(dcol, adesc, bdesc, make_idesc(tt.n_mma, 2 * ks, 0), sfa,
+                                            sfb_col + 4 * p, (g | ks | p) != 0);
                         }
                     }
-                    tc_commit(smem_u32(&sh.empty[r][stage]));
+                    if (PAIR)
+                        tc_commit_pair(smem_u32(&sh.empty[r][stage]));
+                    else
+                        tc_commit(smem_u32(&sh.empty[r][stage]));
                 }
                 __syncwarp();
                 if (++stage == TC_STAGES) {
@@ -396,16 +548,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                 }
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(smem_u32(&sh.acc_full[buf]));
+            if (lane == 0) {
+                if (PAIR)
+                    tc_commit_pair(smem_u32(&sh.acc_full[buf]));
+                else
+                    tc_commit(smem_u32(&sh.acc_full[buf]));
+            }
             __syncwarp();
+            ++issued;
         }
         // before the CTA frees TMEM, every MMA this warp issued must be done
         // (on the normal path the epilogue has already seen them finish; after a
-        // timeout some may still be in flight)
+        // timeout some may still be in flight).  In a pair the commit also
+        // reaches the odd CTA, whose relay waits for it.
         if (lane == 0) {
-            tc_commit(smem_u32(&sh.drain[r]));
-            mbar_wait_bounded(smem_u32(&sh.drain[r]), 0);
+            if (PAIR) {
+                if (ntiles > r) {
+                    tc_commit_pair(smem_u32(&sh.drain[r]));
+                    const uint64_t t0 = global_ns();
+                    while (!mbar_try_wait_cluster(smem_u32(&sh.drain[r]), 0))
+                        if (global_ns() - t0 > 1000000000ull) break;
+                }
+            } else {
+                tc_commit(smem_u32(&sh.drain[r]));
+                mbar_wait_bounded(smem_u32(&sh.drain[r]), 0);
+            }
         }
+        (void)issued;
         __syncwarp();
     } else {
         // ---------------- epilogue (warps TC_EPI_WARP0 ..) ----------------
@@ -421,7 +590,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         // in pairs: lanes 0-15 form h for column j (up value shuffled down),
         // lanes 16-31 for column j+1 (gate value shuffled up), h = SwiGLU(g, u),
         // stored in fp32 (the row maximum of |h| is taken when h is
-        // requantised).  W2: Y = s * acc straight out.
+        // requantised).  W2: Y = s * acc straight out.  In a pair each CTA
+        // drains its own tile (its TMEM holds its weight rows); the odd CTA
+        // releases the accumulator to the even CTA's MMA warps remotely.
         const int ew = warp - TC_EPI_WARP0;
         const int q = warp & 3;            // TMEM lane quadrant this warp may access
         const int n0 = 32 * (ew >> 2);     // this warp's column chunk
@@ -429,7 +600,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         const bool w1 = a.gate_up_half > 0;
         float* csc = sh.col_scale[ew];
         for (int j = 0; j < ntiles && !*abort; ++j) {
-            const TcTile tt = tile_at(a, (int)blockIdx.x + j * (int)gridDim.x);
+            const TcTile tt = tile_at(a, tile_of(j));
             const int buf = j % TC_ACC;
             const uint32_t use = (uint32_t)(j / TC_ACC);
             const bool mine = n0 < tt.n_mma;
@@ -439,7 +610,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                 csc[lane] = __ldg(a.row_scale + src);
             }
             __syncwarp();
-            if (!mbar_wait(smem_u32(&sh.acc_full[buf]), use & 1u, abort)) {
+            if (!wait(smem_u32(&sh.acc_full[buf]), use & 1u)) {
                 give_up();
                 break;
             }
@@ -469,16 +640,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[buf]));
+            if (lane == 0) {
+                if (PAIR && !leader)
+                    mbar_arrive_peer(smem_u32(&sh.acc_empty[buf]), peer);
+                else
+                    mbar_arrive(smem_u32(&sh.acc_empty[buf]));
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if (PAIR) cluster_sync();  // no remote arrive or MMA targets this CTA any more
     tc_fence_after();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
-                     : "memory");
+    if (warp == 0) {
+        if (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TC_TMEM_COLS)
+                         : "memory");
+    }
 }
 
 // Copies the x digit planes of every sorted row of a tensor-core expert from
@@ -522,8 +704,37 @@ static int tc_grid() {
         int dev = 0, sms = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(k_tc_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
+        cudaFuncSetAttribute(k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
         grid = sms;  // one CTA per SM: it allocates all of the SM's TMEM
+    }
+    return grid;
+}
+
+// Clusters of two CTAs that can be resident at once (0: the pair form is not
+// available); the grid is two CTAs per such cluster, so no cluster waits for
+// another to finish.
+static int tc_pair_grid() {
+    static int grid = -1;
+    if (grid < 0) {
+        grid = 0;
+        if (cudaFuncSetAttribute(k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(TcShared)) != cudaSuccess)
+            return grid;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * tc_grid());
+        cfg.blockDim = dim3(TC_THREADS);
+        cfg.dynamicSmemBytes = sizeof(TcShared);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true>, &cfg) == cudaSuccess && clusters > 0)
+            grid = 2 * clusters;
+        cudaGetLastError();
     }
     return grid;
 }
@@ -544,11 +755,32 @@ cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, in
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
-                           const float* row_scale, const int32_t* perm, int k_div, float* out,
+                           const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
                            cudaStream_t st) {
     TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
              E, flag, row_scale, perm, k_div, out};
-    const cudaError_t e = launch_pdl(k_tc_gemm, dim3(tc_grid()), dim3(TC_THREADS), sizeof(TcShared), st, a);
+    cudaError_t e;
+    // the pair takes two adjacent 128-row tiles of one expert: N % 256 == 0
+    const int pgrid = (pair && N % (2 * TC_BM) == 0) ? tc_pair_grid() : 0;
+    if (pgrid > 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(pgrid);
+        cfg.blockDim = dim3(TC_THREADS);
+        cfg.dynamicSmemBytes = sizeof(TcShared);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<true>, a);
+    } else {
+        e = launch_pdl(k_tc_gemm<false>, dim3(tc_grid()), dim3(TC_THREADS), sizeof(TcShared), st, a);
+    }
     count_launches(1);
     return e;
 }

@@ -254,6 +254,10 @@ int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStre
  * moe_set_option returns MOE_OK or MOE_ERR_INVALID_ARG; moe_get_option returns
  * the current value (-1 for an unknown option). */
 #define MOE_OPT_TC_MIN_ROWS 1
+/*   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
+ *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
+ *   multiple of 256); 0 (default) one CTA per SM.  Same results. */
+#define MOE_OPT_TC_PAIR 2
 int moe_set_option(int option, int value);
 int moe_get_option(int option);
 
