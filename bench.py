@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--workload", default="decode_T8")
     ap.add_argument("--prefill-workload", default="prefill_T4604")
     ap.add_argument("--no-prefill", action="store_true")
-    ap.add_argument("--no-skew", action="store_true", help="skip the skewed prefill line")
+    ap.add_argument("--no-skew", action="store_true", help="skip the skewed prefill lines")
+    ap.add_argument("--no-decode-t64", action="store_true", help="skip the decode_T64 line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
@@ -373,12 +374,26 @@ def main():
         "clocks": r["clocks"],
         "kernel_ms_per_step": {"w1": round(r["w1_ms"] / steps, 5), "w2": round(r["w2_ms"] / steps, 5)},
     }
+    if not a.no_decode_t64:
+        # the larger decode batch (most experts get 1-3 rows): same HBM roofline
+        dw = synth.WORKLOADS["decode_T64"]
+        dsteps = max(3, min(500, steps // 4))
+        rd = run_gpu_workload(dw.name, dsteps, max(3, warmup), dist, want_e2e=False, want_clocks=False)
+        out["decode_T64"] = {
+            "workload": dw.name, "T": dw.T, "steps": dsteps,
+            "value": round(whole_job_value(N, dw.T, dsteps, rd["ms"]), 1), "unit": "tokens/s",
+            "ms_per_step": round(rd["ms"] / dsteps, 5), "touched_experts": rd["touched"],
+            "roofline": roofline_hbm(rd, peaks, profiled_traffic(f"k_gemv_{dw.name}.md")),
+        }
     if not a.no_prefill:
-        # prefill lines (tensor-core path): the prefill chunk, and the skewed
-        # prefill (one expert takes almost every row) as an informational line
+        # prefill lines (tensor-core path): the prefill chunk, the skewed
+        # prefill as specified (one expert takes almost every row) and its
+        # labelled milder variant (c = 1.25: empty experts, thousands of rows on
+        # the top experts, many small experts on the streaming GEMM)
         fp8_peak = 2.0 * peaks["bf16_tflops"]
-        for key, pname, cap in (("prefill", a.prefill_workload, 20), ("prefill_skew", "prefill_skew_T16384", 5)):
-            if key == "prefill_skew" and a.no_skew:
+        for key, pname, cap in (("prefill", a.prefill_workload, 20), ("prefill_skew", "prefill_skew_T16384", 5),
+                                ("prefill_skew1.25", "prefill_skew1.25_T16384", 5)):
+            if key.startswith("prefill_skew") and a.no_skew:
                 continue
             pw = synth.WORKLOADS[pname]
             psteps = max(3, min(cap, steps // 100))
@@ -389,8 +404,10 @@ def main():
                 "value": round(whole_job_value(N, pw.T, psteps, rp["ms"]), 1), "unit": "tokens/s",
                 "ms_per_step": round(rp["ms"] / psteps, 4),
                 "gemm_ms_per_step": round(rp["gemm_ms"] / psteps, 4),
+                "touched_experts": rp["touched"],
                 "roofline": {"bound": "tensor",
-                             "kernel": "k_tc_gemm (tcgen05 kind::mxf4 block-scaled, W1 and W2 launches)",
+                             "kernel": "W1 and W2 grouped GEMM launches (k_tc_gemm tcgen05 kind::mxf4 "
+                                       "block-scaled, plus k_gemv for experts below the row threshold)",
                              "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
                              "frac": round(ptf / fp8_peak, 5),
                              "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
@@ -401,6 +418,7 @@ def main():
                              "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
                              "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
+                "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
             }
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)

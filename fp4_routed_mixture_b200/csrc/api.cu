@@ -52,11 +52,23 @@ int check_dims(const moe_dims* d, bool need_T) {
     return MOE_OK;
 }
 
-// Experts with at least this many rows use the tensor-core GEMM (see
-// moe_set_option); the others the streaming GEMM.
-int g_tc_min_rows = 32;
-// Tensor-core GEMM in SM pairs (cta_group::2) where the shape allows (MOE_OPT_TC_PAIR).
-int g_tc_pair = 0;
+// Process-wide options (moe_set_option).  Every public call reads them once
+// into an Options value, so a call sees one consistent set even while another
+// host thread changes them.
+std::atomic<int> g_tc_min_rows{32};        // experts with at least this many rows use the tensor-core GEMM
+std::atomic<int> g_tc_pair{0};             // tensor-core GEMM in SM pairs (cta_group::2) where the shape allows
+std::atomic<int> g_wait_limit_us{1000000}; // limit of the tensor-core GEMM's bounded waits
+std::atomic<int> g_test_timeout{0};        // one-shot: the next tensor-core launch withholds a stage
+
+struct Options {
+    int tc_min_rows;
+    bool tc_pair;
+    uint64_t wait_ns;
+};
+
+Options load_options() {
+    return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, 1000ull * (uint64_t)g_wait_limit_us.load()};
+}
 
 struct WsLayout {
     size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xtp, xinit, hq, sh, hinit, px, ph,
@@ -229,9 +241,9 @@ namespace {
 // (moe_layer_forward on a call with T below the tensor-core threshold and at
 // most kFrontMaxPairs pairs) route, sort, x quant and plan run as one fused
 // launch that writes those tables.
-int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int32_t* topk_idx, float* gates,
-                 int32_t* perm, int32_t* pos, int32_t* offsets, const void* packed, void* y_bf16, void* ws,
-                 size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
+int forward_impl(const Options& opt, const moe_dims* d, const float* logits, const void* x_bf16, int32_t* topk_idx,
+                 float* gates, int32_t* perm, int32_t* pos, int32_t* offsets, const void* packed, void* y_bf16,
+                 void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
     if (int rc = check_dims(d, true)) return rc;
     if (!ws || !packed || !offsets) return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if (d->T > 0 && (!x_bf16 || !topk_idx || !gates || !perm || !pos || !y_bf16))
@@ -269,7 +281,9 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
     } while (0)
     // an expert has at most T rows, so the tensor-core path is skipped without
     // reading any count when T < tc_min (always so with the fused front)
-    const bool use_tc = !logits && T >= g_tc_min_rows;
+    const bool use_tc = !logits && T >= opt.tc_min_rows;
+    // the timeout test applies to the first tensor-core launch after it is armed
+    const int withhold = use_tc ? g_test_timeout.exchange(0) : 0;
     // token rows per streaming-GEMM unit: 2 for small calls (nearly every expert
     // has one or two rows; the smaller ring slot fits more warps per SM), else 4
     const int group = T <= moe::kGemvSmallGroupMaxT ? moe::kGemvSmallGroup : moe::kGemvGroup;
@@ -294,7 +308,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
         MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
-        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? g_tc_min_rows : 0x7fffffff,
+        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? opt.tc_min_rows : 0x7fffffff,
                                       group, uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
                 "plan + row state");
     }
@@ -306,7 +320,8 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
                              uoff1, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, g_tc_pair != 0, stream),
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, opt.tc_pair, opt.wait_ns, withhold,
+                                    stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, prow, L.plane_rows, ph, P, k, E, I, hq,
@@ -317,7 +332,7 @@ int forward_impl(const moe_dims* d, const float* logits, const void* x_bf16, int
                              uoff2, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, g_tc_pair != 0, stream),
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, opt.tc_pair, opt.wait_ns, 0, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, yf, etc, topk_idx, sh, gates, pos, T, k, E, H, y_bf16, flag, stream),
@@ -334,7 +349,7 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
                 const int32_t* perm, const int32_t* pos, const int32_t* offsets, const void* packed,
                 void* y_bf16, void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
     g_last_error.clear();
-    return forward_impl(d, nullptr, x_bf16, const_cast<int32_t*>(topk_idx), const_cast<float*>(gates),
+    return forward_impl(load_options(), d, nullptr, x_bf16, const_cast<int32_t*>(topk_idx), const_cast<float*>(gates),
                         const_cast<int32_t*>(perm), const_cast<int32_t*>(pos), const_cast<int32_t*>(offsets),
                         packed, y_bf16, ws, ws_bytes, dbg, stream);
 }
@@ -385,14 +400,15 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
     int32_t* perm = (int32_t*)(w + L.perm);
     int32_t* pos = (int32_t*)(w + L.pos);
     int32_t* offsets = (int32_t*)(w + L.offsets);
-    if (d->T > 0 && d->T < g_tc_min_rows && (long long)d->T * d->k <= moe::kFrontMaxPairs)
-        return forward_impl(d, logits, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
+    const Options opt = load_options();
+    if (d->T > 0 && d->T < opt.tc_min_rows && (long long)d->T * d->k <= moe::kFrontMaxPairs)
+        return forward_impl(opt, d, logits, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
                             L.idx - L.fwd, dbg, stream);
     if (int rc = moe_route(logits, d->T, d->E, d->k, idx, gates, stream)) return rc;
     if (int rc = moe_sort(idx, d->T, d->k, d->E, perm, pos, offsets, w + L.sortws, L.sort_bytes, stream))
         return rc;
-    return moe_forward(d, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
-                       L.idx - L.fwd, dbg, stream);
+    return forward_impl(opt, d, nullptr, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
+                        L.idx - L.fwd, dbg, stream);
 }
 
 int moe_layer_tables(const moe_dims* d, void* ws, int32_t** topk_idx, float** gates, int32_t** perm,
@@ -447,12 +463,25 @@ int moe_set_option(int option, int value) {
         g_tc_pair = value;
         return MOE_OK;
     }
+    if (option == MOE_OPT_WAIT_LIMIT_US) {
+        if (value < 1 || value > 10000000)
+            return fail(MOE_ERR_INVALID_ARG, "moe_set_option: WAIT_LIMIT_US must be in [1, 10^7]");
+        g_wait_limit_us = value;
+        return MOE_OK;
+    }
+    if (option == MOE_OPT_TEST_TIMEOUT) {
+        if (value != 0 && value != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TEST_TIMEOUT must be 0 or 1");
+        g_test_timeout = value;
+        return MOE_OK;
+    }
     return fail(MOE_ERR_INVALID_ARG, "moe_set_option: unknown option %d", option);
 }
 
 int moe_get_option(int option) {
     if (option == MOE_OPT_TC_MIN_ROWS) return g_tc_min_rows;
     if (option == MOE_OPT_TC_PAIR) return g_tc_pair;
+    if (option == MOE_OPT_WAIT_LIMIT_US) return g_wait_limit_us;
+    if (option == MOE_OPT_TEST_TIMEOUT) return g_test_timeout;
     return -1;
 }
 

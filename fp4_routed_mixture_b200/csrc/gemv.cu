@@ -384,16 +384,18 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
 
 template <int G>
 static int gemv_grid() {
-    static int grid = 0;
-    if (!grid) {
+    static PerContext cache;
+    return cache.get([] {
         int dev = 0, sms = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(k_gemv<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<G>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv<G>, kGemvWarps * 32, smem_bytes<G>());
-        grid = sms * (per_sm > 0 ? per_sm : 1);
-    }
-    return grid;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaFuncSetAttribute(k_gemv<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<G>()) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv<G>, kGemvWarps * 32, smem_bytes<G>()) !=
+                cudaSuccess)
+            return -1;
+        return sms * (per_sm > 0 ? per_sm : 1);
+    });
 }
 
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
@@ -402,9 +404,11 @@ cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, con
                         const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st) {
     GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
                gate_up_half, P, 0u};
+    const int grid = group == 2 ? gemv_grid<2>() : gemv_grid<4>();
+    if (grid <= 0) return cudaErrorInvalidConfiguration;
     const cudaError_t e =
-        group == 2 ? launch_pdl(k_gemv<2>, dim3(gemv_grid<2>()), dim3(kGemvWarps * 32), smem_bytes<2>(), st, a)
-                   : launch_pdl(k_gemv<4>, dim3(gemv_grid<4>()), dim3(kGemvWarps * 32), smem_bytes<4>(), st, a);
+        group == 2 ? launch_pdl(k_gemv<2>, dim3(grid), dim3(kGemvWarps * 32), smem_bytes<2>(), st, a)
+                   : launch_pdl(k_gemv<4>, dim3(grid), dim3(kGemvWarps * 32), smem_bytes<4>(), st, a);
     count_launches(1);
     return e;
 }

@@ -1,12 +1,64 @@
 // Launch wrappers shared between the kernel files and the C-ABI layer.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include <algorithm>
 #include <cstddef>
+#include <mutex>
 
 namespace moe {
+
+// Launch set-up computed once per device context: the grid size of a
+// persistent kernel and the function attributes it needs (the dynamic
+// shared-memory limit is an attribute of the function in the current context).
+// get(init) runs init() with the calling thread's device current the first
+// time that device -- or a new context on it, after cudaDeviceReset or under a
+// caller-created context -- asks, and returns the cached value afterwards.
+// init() returns a negative value on failure, which is returned and not cached.
+// (The current context is read through the driver entry point that the CUDA
+// runtime hands out, so the library does not link against the driver.)
+class PerContext {
+  public:
+    template <class F>
+    int get(F init) {
+        int dev = 0;
+        CUcontext ctx = nullptr;
+        const auto get_ctx = ctx_getter();
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSlots || !get_ctx ||
+            get_ctx(&ctx) != CUDA_SUCCESS)
+            return init();
+        std::lock_guard<std::mutex> lock(mu_);
+        if (ctx_[dev] != ctx || !ctx) {
+            const int v = init();
+            if (v < 0) return v;
+            ctx_[dev] = ctx;
+            val_[dev] = v;
+        }
+        return val_[dev];
+    }
+
+  private:
+    typedef CUresult (*CtxGetCurrent)(CUcontext*);
+    static CtxGetCurrent ctx_getter() {
+        static const CtxGetCurrent fn = [] {
+            void* p = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess) {
+                cudaGetLastError();
+                p = nullptr;
+            }
+            return reinterpret_cast<CtxGetCurrent>(p);
+        }();
+        return fn;
+    }
+    static constexpr int kSlots = 64;
+    std::mutex mu_;
+    CUcontext ctx_[kSlots] = {};
+    int val_[kSlots] = {};
+};
 
 // Unit of the streaming grouped GEMM: kGemvTileRows weight rows by up to
 // kGemvGroup token rows (shared by it and the planner).
@@ -119,7 +171,7 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           cudaStream_t st);
+                           uint64_t wait_ns, int withhold, cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
                            const int32_t* topk_idx, const float* sh, const float* gates,

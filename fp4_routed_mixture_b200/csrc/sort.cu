@@ -12,8 +12,6 @@
 //                  step, which keeps the sort stable.
 // A single chunk (P <= 1024, the decode case) runs both phases in one launch.
 // Expert ids outside [0, E) raise FLAG_BAD_EXPERT and are skipped.
-#include <mutex>
-
 #include "steps.cuh"
 
 namespace moe {
@@ -134,24 +132,16 @@ static __device__ __align__(256) uint8_t g_sort_scratch[kSortStaticBytes];
 static_assert(kSortStaticMaxPairs % kSortChunk == 0, "whole chunks");
 static_assert(kSortChunk <= 32 * 32, "warp_stable_scatter holds 32 ids per lane");
 
-// Device address of g_sort_scratch on the current device, looked up once per
-// device (the host-side name is only a stand-in for it).
+// Device address of g_sort_scratch in the calling thread's current context.
+// The host-side name is only a stand-in; the address belongs to this
+// library's module as loaded in that context, which a cudaDeviceReset or a
+// caller-created context replaces, so it is looked up on every call (a host
+// table lookup once the module is loaded).
 static cudaError_t sort_static_scratch(void** out) {
-    constexpr int kMaxDevices = 64;
-    static void* ptrs[kMaxDevices] = {};
-    static std::mutex mu;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_sort_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_sort_scratch);
-        if (e != cudaSuccess) return e;
-        ptrs[dev] = p;
-    }
-    *out = ptrs[dev];
+    *out = p;
     return cudaSuccess;
 }
 

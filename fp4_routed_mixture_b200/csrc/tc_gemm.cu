@@ -105,6 +105,8 @@ struct TcArgs {
     const int32_t* perm;       // sorted row -> pair id (W1: source row = perm[i] / k_div)
     int k_div;                 // W1: k; W2: 0 (source row = sorted row)
     float* out;                // W1: h [P, I]; W2: Y [P, H]  (fp32, final values)
+    uint64_t wait_ns;          // limit of every bounded wait (global-timer nanoseconds)
+    int withhold;              // test of the timeout path: 1 = see launch_tc_gemm
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -132,28 +134,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Waits on barriers that CTA-pair operations arrive on use cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Bounded wait (about one second; a stage lands in microseconds).  Gives up
-// early when another role has aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int32_t* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait on a phase of an mbarrier: true once the phase with the given
+// parity has completed, false after limit_ns of global time (the limit is a
+// kernel argument, about one second by default; a stage lands in
+// microseconds) or, when abort is not NULL, as soon as another role has
+// aborted.  CLUSTER: the barrier is also arrived on by the peer CTA of an SM
+// pair, so it is read with cluster-scope acquire.
+template <bool CLUSTER>
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                              volatile int32_t* abort) {
+    auto poll = [&]() { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (poll()) return true;
     const uint64_t t0 = global_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_ns() - t0 > 1000000000ull) return false;
+            if (poll()) return true;
+        if (abort && *abort) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
-}
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > 1000000000ull) return false;
-    return true;
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile(
@@ -222,18 +237,6 @@ __device__ __forceinline__ void mbar_arrive_peer(uint32_t bar, uint32_t rank) {
 }
 __device__ __forceinline__ void store_peer_u32(uint32_t addr, uint32_t rank, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer_addr(addr, rank)), "r"(v) : "memory");
-}
-// Waits on barriers that CTA-pair operations arrive on use cluster scope.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
 }
 // tcgen05.commit of the pair's MMAs, arriving on the barrier at this offset in
 // both CTAs.
@@ -386,15 +389,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     // bounded waits; barriers that pair operations arrive on are read at
     // cluster scope
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (!PAIR) return mbar_wait(bar, parity, abort);
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        const uint64_t t0 = global_ns();
-        for (;;) {
-            for (int i = 0; i < 64; ++i)
-                if (mbar_try_wait_cluster(bar, parity)) return true;
-            if (*abort) return false;
-            if (global_ns() - t0 > 1000000000ull) return false;
-        }
+        return mbar_wait_for<PAIR>(bar, parity, a.wait_ns, abort);
+    };
+    // the last waits before TMEM is freed ignore the abort flag: a wait that
+    // still runs out raises FLAG_TIMEOUT (the caller must then treat the whole
+    // call's results as invalid; the CTA still frees TMEM and exits)
+    auto final_wait = [&](uint32_t bar, uint32_t parity) {
+        if (!mbar_wait_for<PAIR>(bar, parity, a.wait_ns, nullptr)) raise_flag(a.flag, FLAG_TIMEOUT);
     };
 
     if (warp < TC_PIPES) {
@@ -422,7 +423,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                     break;
                 }
                 const uint32_t sbase = smem_u32(sh.stage[r][stage]);
-                if (lane == 0) {
+                // timeout test: CTA 0's first producer issues neither the copies
+                // nor the arrival of its first stage, so the MMA issuer waiting
+                // for that stage runs out of time
+                const bool withheld = !PAIR && a.withhold && blockIdx.x == 0 && r == 0 && j == 0 && g == 0;
+                if (lane == 0 && !withheld) {
                     if (rows_ok) {
                         mbar_expect_tx(fb, TC_A_BYTES + bbytes);
                         bulk_g2s(sbase, wsrc + (size_t)g * TC_A_BYTES, TC_A_BYTES, fb);
@@ -434,7 +439,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                     }
                 }
                 __syncwarp();
-                filled[stage] = true;
+                filled[stage] = !withheld;
                 fill_parity[stage] = phase;
                 if (++stage == TC_STAGES) {
                     stage = 0;
@@ -445,7 +450,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         // let every copy this warp issued land before the CTA can exit (on the
         // normal path the MMA warp has already waited for all of them)
         for (int s = 0; s < TC_STAGES; ++s)
-            if (filled[s]) mbar_wait_bounded(smem_u32(&sh.full[r][s]), fill_parity[s]);
+            if (filled[s] && lane == 0) final_wait(smem_u32(&sh.full[r][s]), fill_parity[s]);
+        __syncwarp();
     } else if (warp < TC_EPI_WARP0 && PAIR && !leader) {
         // ---------------- relay of pipe r (odd CTA of a pair) ----------------
         // Passes "this CTA's half of the stage has landed" to the even CTA,
@@ -471,11 +477,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             }
             if (!ok) break;
         }
-        if (lane == 0 && ntiles > r) {
-            const uint64_t t0 = global_ns();
-            while (!mbar_try_wait_cluster(smem_u32(&sh.drain[r]), 0))
-                if (global_ns() - t0 > 1000000000ull) break;
-        }
+        if (lane == 0 && ntiles > r) final_wait(smem_u32(&sh.drain[r]), 0);
         __syncwarp();
     } else if (warp < TC_EPI_WARP0) {
         // ---------------- MMA issuer of pipe r (even CTA of a pair) ----------------
@@ -565,13 +567,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             if (PAIR) {
                 if (ntiles > r) {
                     tc_commit_pair(smem_u32(&sh.drain[r]));
-                    const uint64_t t0 = global_ns();
-                    while (!mbar_try_wait_cluster(smem_u32(&sh.drain[r]), 0))
-                        if (global_ns() - t0 > 1000000000ull) break;
+                    final_wait(smem_u32(&sh.drain[r]), 0);
                 }
             } else {
                 tc_commit(smem_u32(&sh.drain[r]));
-                mbar_wait_bounded(smem_u32(&sh.drain[r]), 0);
+                final_wait(smem_u32(&sh.drain[r]), 0);
             }
         }
         (void)issued;
@@ -698,30 +698,35 @@ __global__ void __launch_bounds__(256)
         for (int p = 0; p < 3; ++p) *reinterpret_cast<uint4*>(dst + p * 512 + cc * 128) = v[3 * cc + p];
 }
 
+// One CTA per SM: it allocates all of the SM's TMEM.
 static int tc_grid() {
-    static int grid = 0;
-    if (!grid) {
+    static PerContext cache;
+    return cache.get([] {
         int dev = 0, sms = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcShared));
-        grid = sms;  // one CTA per SM: it allocates all of the SM's TMEM
-    }
-    return grid;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaFuncSetAttribute(k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(TcShared)) != cudaSuccess)
+            return -1;
+        return sms;
+    });
 }
 
 // Clusters of two CTAs that can be resident at once (0: the pair form is not
 // available); the grid is two CTAs per such cluster, so no cluster waits for
 // another to finish.
 static int tc_pair_grid() {
-    static int grid = -1;
-    if (grid < 0) {
-        grid = 0;
+    static PerContext cache;
+    return cache.get([] {
+        const int single = tc_grid();
+        if (single <= 0) return -1;
         if (cudaFuncSetAttribute(k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(TcShared)) != cudaSuccess)
-            return grid;
+                                 (int)sizeof(TcShared)) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * tc_grid());
+        cfg.gridDim = dim3(2 * single);
         cfg.blockDim = dim3(TC_THREADS);
         cfg.dynamicSmemBytes = sizeof(TcShared);
         cudaLaunchAttribute attr[1];
@@ -732,11 +737,12 @@ static int tc_pair_grid() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true>, &cfg) == cudaSuccess && clusters > 0)
-            grid = 2 * clusters;
-        cudaGetLastError();
-    }
-    return grid;
+        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true>, &cfg) != cudaSuccess || clusters <= 0) {
+            cudaGetLastError();
+            return 0;
+        }
+        return 2 * clusters;
+    });
 }
 
 size_t tc_smem_bytes() { return sizeof(TcShared); }
@@ -756,9 +762,11 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           cudaStream_t st) {
+                           uint64_t wait_ns, int withhold, cudaStream_t st) {
     TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
-             E, flag, row_scale, perm, k_div, out};
+             E, flag, row_scale, perm, k_div, out, wait_ns, withhold};
+    // the timeout test runs on the one-CTA form (withhold applies to it only)
+    if (withhold) pair = false;
     cudaError_t e;
     // the pair takes two adjacent 128-row tiles of one expert: N % 256 == 0
     const int pgrid = (pair && N % (2 * TC_BM) == 0) ? tc_pair_grid() : 0;
@@ -779,7 +787,9 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
         cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, k_tc_gemm<true>, a);
     } else {
-        e = launch_pdl(k_tc_gemm<false>, dim3(tc_grid()), dim3(TC_THREADS), sizeof(TcShared), st, a);
+        const int grid = tc_grid();
+        if (grid <= 0) return cudaErrorInvalidConfiguration;
+        e = launch_pdl(k_tc_gemm<false>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a);
     }
     count_launches(1);
     return e;

@@ -154,7 +154,8 @@ int moe_route(const float *logits, int T, int E, int k, int32_t *topk_idx, float
  *   pos     [P] int32:   inverse permutation, pos[perm[i]] = i.
  * ws: moe_sort_workspace_bytes(T, k, E) bytes, 256-byte aligned, any contents.
  * An expert id outside [0, E) raises MOE_FLAG_BAD_EXPERT in ws; such pairs are
- * left out of the sort (perm/pos are then incomplete).
+ * left out of the sort: perm/pos are then incomplete and offsets[E], the
+ * number of pairs sorted, is below T*k.
  * ------------------------------------------------------------------------- */
 size_t moe_sort_workspace_bytes(int T_max, int k, int E);
 int moe_sort(const int32_t *topk_idx, int T, int k, int E, int32_t *perm, int32_t *pos,
@@ -169,13 +170,17 @@ int moe_sort(const int32_t *topk_idx, int T, int k, int E, int32_t *perm, int32_
  *   - Scratch is a fixed 256 KB array inside the library (held on every GPU
  *     that loads it, until process exit): T*k <= 65536 pairs and E <= 1024;
  *     larger calls return MOE_ERR_UNSUPPORTED_SHAPE (use moe_sort).
- *   - The first call on a device looks up that array's device address for the
- *     current device (cudaGetSymbolAddress); make that first call before any
- *     stream capture.
+ *   - Every call looks up that array's device address in the calling
+ *     thread's current context (cudaGetSymbolAddress; the address belongs to
+ *     the library's module in that context, so it is not cached).  The first
+ *     call in a context may load the module: make it before any stream
+ *     capture.
  *   - All calls share the array: calls that overlap on a GPU race.  Each call
  *     clears and rewrites what it reads.
- *   - Expert ids outside [0, E) are skipped as in moe_sort; the error word is
- *     internal to this variant (use moe_sort to observe it). */
+ *   - Expert ids outside [0, E) are skipped as in moe_sort.  The caller sees
+ *     it in the outputs, without any extra read: offsets[E] is the number of
+ *     pairs sorted, so offsets[E] < T*k means that T*k - offsets[E] pairs had
+ *     a bad id (and perm/pos are incomplete). */
 int moe_sort_static(const int32_t *topk_idx, int T, int k, int E, int32_t *perm, int32_t *pos,
                     int32_t *offsets, cudaStream_t stream);
 
@@ -245,19 +250,33 @@ int moe_quant_rows_f32(const float *v, int rows, int cols, int8_t *q, float *s,
 int moe_exp_f32(const float *x, float *y, int64_t n, cudaStream_t stream);
 int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStream_t stream);
 
-/* Process-wide tuning options (not thread-safe; set them before launching work).
+/* Process-wide options.  Each call reads them once when it starts, so a call
+ * sees one consistent set; a change made while calls are being enqueued on
+ * other host threads applies from the next call that starts after it.
  *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
  *   run on the tensor-core grouped GEMM (tcgen05, tiles of 128 weight rows x
  *   128 token rows); experts with fewer rows run on the CUDA-core streaming
  *   GEMM.  Default 32; must be >= 1.  Both paths give the same results inside
  *   the exactness domains stated at moe_forward.
+ *   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
+ *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
+ *   multiple of 256); 0 one CTA per SM.  Same results.
+ *   MOE_OPT_WAIT_LIMIT_US: limit, in microseconds, of every bounded wait inside
+ *   the tensor-core GEMM (a pipeline stage normally lands in a few
+ *   microseconds).  A wait that runs out raises MOE_FLAG_TIMEOUT in the call's
+ *   error word; the kernel still waits (again bounded) for its own copies and
+ *   MMAs, frees its tensor memory and returns, and the call's results are
+ *   invalid.  Default 1000000 (one second); range [1, 10^7].
+ *   MOE_OPT_TEST_TIMEOUT: 1 arms a test of that path: the next call that runs
+ *   the tensor-core W1 GEMM has its first CTA's first pipeline stage withheld
+ *   (neither copied nor signalled), so the MMA waiting for it runs out of
+ *   time.  The arming is consumed by that call; 0 disarms.  For tests only.
  * moe_set_option returns MOE_OK or MOE_ERR_INVALID_ARG; moe_get_option returns
  * the current value (-1 for an unknown option). */
 #define MOE_OPT_TC_MIN_ROWS 1
-/*   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
- *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
- *   multiple of 256); 0 (default) one CTA per SM.  Same results. */
 #define MOE_OPT_TC_PAIR 2
+#define MOE_OPT_WAIT_LIMIT_US 3
+#define MOE_OPT_TEST_TIMEOUT 4
 int moe_set_option(int option, int value);
 int moe_get_option(int option);
 

@@ -6,7 +6,8 @@ fixed-token and hash-based checks before optimising further.  These digests
 play that role here.  Every value comes from the oracle (oracle/) fed by the
 seeded input generator (synth/); nothing here touches the CUDA library.
 
-Usage: python tests/golden/make_golden.py
+Usage: python tests/golden/make_golden.py [workload ...]
+(with names, only those entries are recomputed; the others are kept)
 """
 import hashlib
 import json
@@ -23,7 +24,8 @@ import synth  # noqa: E402
 
 OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "digests.json")
 FULL = ["tiny_T4", "decode_T8", "decode_T64"]        # whole layer
-SAMPLED = ["prefill_T4604", "prefill_skew_T16384"]     # route/sort whole, layer on sampled tokens
+SAMPLED = ["prefill_T4604", "prefill_skew_T16384",     # route/sort whole, layer on sampled tokens
+           "prefill_skew1.25_T16384"]
 
 
 def sha(a: np.ndarray) -> str:
@@ -61,8 +63,9 @@ def digests(name: str) -> dict:
 
 
 def main():
-    res = {}
-    for name in FULL + SAMPLED:
+    names = sys.argv[1:] or FULL + SAMPLED
+    res = json.load(open(OUT)) if sys.argv[1:] and os.path.exists(OUT) else {}
+    for name in names:
         res[name] = digests(name)
         print(name, "done", flush=True)
     with open(OUT, "w") as f:

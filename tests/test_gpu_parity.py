@@ -308,11 +308,41 @@ def test_forward_rejects_bad_args(moe):
         moe.moe_workspace_bytes(4, 128, 128, 4, 5)
 
 
-@pytest.mark.parametrize("name", ["prefill_T4604", "prefill_skew_T16384"])
+def chosen_tokens(offsets, perm, k, T, n_total=256, seed=7):
+    """Tokens for a sampled comparison, chosen to cover the layer's structure:
+    the token of the first sorted row of every touched expert (so every
+    expert, streaming or tensor-core, is hit), the token of the last row of 32
+    of them (ragged tails), the tokens of the first, a middle and the last
+    128-row token tile of the largest expert, the first and last token, then
+    seeded random tokens up to n_total (the oracle evaluates each token
+    separately)."""
+    counts = np.diff(offsets)
+    tok = {0, T - 1}
+    touched = np.nonzero(counts)[0]
+    for e in touched:
+        tok.add(int(perm[offsets[e]]) // k)
+    for e in touched[:: max(1, len(touched) // 32)]:
+        tok.add(int(perm[offsets[e + 1] - 1]) // k)
+    big = int(np.argmax(counts))
+    nblk = (int(counts[big]) + 127) // 128
+    for b in sorted({0, nblk // 2, nblk - 1}):
+        r0 = offsets[big] + 128 * b
+        r1 = min(offsets[big + 1], r0 + 128)
+        tok.update(int(perm[r]) // k for r in (r0, (r0 + r1) // 2, r1 - 1))
+    rng = np.random.default_rng(seed)
+    while len(tok) < n_total:
+        tok.add(int(rng.integers(0, T)))
+    return np.array(sorted(tok), np.int32)
+
+
+@pytest.mark.parametrize("name", ["prefill_T4604", "prefill_skew_T16384", "prefill_skew1.25_T16384"])
 def test_forward_parity_sampled_full_size(moe, workload_data, name):
-    """Full-size prefill workloads: every routing/sort value is compared whole;
-    the layer's outputs on sampled tokens are compared with the oracle's
-    per-token computation (INT8 codes bit-exact, y within tolerance)."""
+    """Full-size prefill workloads in the default configuration (experts with
+    at least 32 rows on the tensor-core GEMM, the others on the streaming
+    GEMM): every routing/sort value is compared whole; the layer's outputs on
+    chosen tokens (every touched expert, the largest expert's first, middle and
+    last token tile) are compared with the oracle's per-token computation
+    (INT8 codes bit-exact, y within tolerance)."""
     d, w = workload_data(name), synth.WORKLOADS[name]
     r = run_layer(moe, d, w)
     oi, og = oracle.route(d["logits"], w.k)
@@ -320,14 +350,18 @@ def test_forward_parity_sampled_full_size(moe, workload_data, name):
     counts, ooff, operm, opos = oracle.sort(oi, w.E)
     assert np.array_equal(r["perm"].cpu().numpy(), operm)
     assert np.array_equal(r["offsets"].cpu().numpy(), ooff)
-    rng = np.random.default_rng(7)
-    tok = np.unique(np.concatenate([[0, w.T - 1], rng.integers(0, w.T, 14)])).astype(np.int32)
+    tok = chosen_tokens(ooff, operm, w.k, w.T)
     ot = oracle.forward_tokens(d["x"], d["logits"], d["w1_codes"], d["w1_scales"], d["w2_codes"],
                                d["w2_scales"], w.k, tok)
     assert np.array_equal(r["dbg"]["xq"].cpu().numpy()[tok], ot["xq"])
     assert np.array_equal(r["dbg"]["sx"].cpu().numpy()[tok], ot["sx"])
     pairs = (tok[:, None] * w.k + np.arange(w.k)[None, :]).ravel()
     rows = opos[pairs]
+    # both kernels are covered wherever the workload has both kinds of expert
+    tc_rows = counts[oi.ravel()[pairs]] >= moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS)
+    if ((counts > 0) & (counts < 32)).any():
+        assert (~tc_rows).any()
+    assert tc_rows.any()
     assert np.array_equal(r["dbg"]["hq"].cpu().numpy()[rows], ot["hq"])
     assert np.array_equal(r["dbg"]["sh"].cpu().numpy()[rows], ot["sh"])
     y_check(r["y"][torch.from_numpy(tok).long().cuda()], ot["y"])

@@ -44,8 +44,36 @@ def test_sort_static_matches_sort_twice_in_a_row(moe):
             assert torch.equal(a, b)
 
 
+def test_sort_static_at_its_limits(moe):
+    # the largest accepted call fills the whole array: T*k = 65536 pairs over
+    # E = 1024 experts (64 chunk histograms of 1024 entries)
+    idx = _idx(4096, 16, 1024, 4)
+    ref = moe.moe_sort(idx, 1024)
+    got = moe.moe_sort_static(idx, 1024)
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+
+
 def test_sort_static_refuses_oversized_calls(moe):
     idx = torch.zeros((65536 // 6 + 1, 6), dtype=torch.int32, device="cuda")
     with pytest.raises(moe.MoeError) as ei:
         moe.moe_sort_static(idx, 256)
     assert ei.value.status == -2
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_sort_static(torch.zeros((4, 2), dtype=torch.int32, device="cuda"), 1025)
+    assert ei.value.status == -2
+
+
+def test_sort_static_reports_bad_ids_in_offsets(moe):
+    # a caller of this variant has no workspace to read an error word from:
+    # offsets[E] counts the pairs sorted, so bad ids show as offsets[E] < T*k
+    for T, k, E in [(6, 2, 4), (3000, 2, 8)]:
+        idx = _idx(T, k, E, 5)
+        idx[1, 1] = E + 3
+        idx[T - 1, 0] = -1
+        ref = moe.moe_sort(idx, E)
+        got = moe.moe_sort_static(idx, E)
+        torch.cuda.synchronize()
+        assert int(got[2][E]) == T * k - 2
+        assert torch.equal(got[2], ref[2])
