@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-skew", action="store_true", help="skip the skewed prefill lines")
     ap.add_argument("--no-decode-t64", action="store_true", help="skip the decode_T64 line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tc-pair", type=int, choices=[0, 1], default=None,
+                    help="MOE_OPT_TC_PAIR for the run (default: the library's default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
                     help="no timing, no JSON: pack the workload and run --steps layer calls "
@@ -350,6 +352,10 @@ def main():
     assert warmup >= 3 or a.warmup is not None
     dist = Dist(a.gpus)
     import torch
+
+    import fp4_routed_mixture_b200 as moe
+    if a.tc_pair is not None:
+        moe.moe_set_option(moe.MOE_OPT_TC_PAIR, a.tc_pair)
     rank0 = dist.rank == 0
     peaks = measured_peaks()
     r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
@@ -419,6 +425,7 @@ def main():
                              "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
                 "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
+                "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
             }
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)

@@ -71,14 +71,25 @@ Options load_options() {
 }
 
 struct WsLayout {
-    size_t flag, uoff1, uoff2, toff1, toff2, poff, etc, prow, sx, xq, xtp, xinit, hq, sh, hinit, px, ph,
+    size_t flag, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, sx, xq, xtp, xinit, hq, sh, hinit, px, ph,
         hbuf, yf, gacc, yacc, total;
     int plane_rows;
+    int stream_rows;   // capacity of the buffers of streaming-GEMM rows
 };
 
-WsLayout ws_layout(const moe_dims& d, long long T) {
+// Rows the streaming GEMM can own in a call of T tokens: every row when no
+// expert can reach the tensor-core threshold (T < tc_min), otherwise at most
+// tc_min - 1 rows of each of the E experts.
+long long stream_row_capacity(const moe_dims& d, long long T, int tc_min) {
+    const long long P = T * d.k;
+    if (T < tc_min) return P;
+    return std::min(P, (long long)d.E * (tc_min - 1));
+}
+
+WsLayout ws_layout(const moe_dims& d, long long T, int tc_min) {
     using moe::align_up;
     const size_t P = (size_t)T * d.k;
+    const size_t S = (size_t)stream_row_capacity(d, T, tc_min);
     WsLayout L;
     size_t o = 0;
     L.flag = o; o += 256;
@@ -87,24 +98,26 @@ WsLayout ws_layout(const moe_dims& d, long long T) {
     L.toff1 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.toff2 = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.poff = o; o += align_up(4 * (size_t)(d.E + 1), 256);
+    L.soff = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.etc = o; o += align_up(4 * (size_t)d.E, 256);
     L.prow = o; o += align_up(4 * P, 256);
     L.sx = o; o += align_up(4 * (size_t)T, 256);
     L.xq = o; o += align_up((size_t)T * d.H, 256);
     L.xtp = o; o += align_up((size_t)T * (d.H / 32) * 48, 256);   // x digit planes, token order
     L.xinit = o; o += align_up(4 * (size_t)T * (d.H / 32), 256);
-    L.hq = o; o += align_up(P * d.I, 256);
+    L.stream_rows = (int)S;
+    L.hq = o; o += align_up(S * d.I, 256);                  // h codes of streaming rows
     L.sh = o; o += align_up(4 * P, 256);
-    L.hinit = o; o += align_up(4 * P * (d.I / 32), 256);
+    L.hinit = o; o += align_up(4 * S * (d.I / 32), 256);
     // digit planes of the tensor-core GEMM (stage-major, see kernels.cuh):
     // each tensor-core expert's rows are padded to a multiple of 16
     L.plane_rows = (int)align_up(P + 16 * (size_t)d.E + 16, 16);
     L.px = o; o += align_up(moe::plane_bytes(d.H, L.plane_rows), 256);
     L.ph = o; o += align_up(moe::plane_bytes(d.I, L.plane_rows), 256);
-    L.hbuf = o; o += align_up(4 * P * d.I, 256);        // h of tensor-core rows
+    L.hbuf = o; o += align_up(4 * P * d.I, 256);        // h of every row (fp32)
     L.yf = o; o += align_up(4 * P * d.H, 256);          // Y of tensor-core rows
-    L.gacc = o; o += align_up(8 * P * 2 * d.I, 256);   // fp64 sums of streaming-GEMM rows
-    L.yacc = o; o += align_up(8 * P * d.H, 256);
+    L.gacc = o; o += align_up(8 * S * 2 * d.I, 256);   // fp64 sums of streaming-GEMM rows
+    L.yacc = o; o += align_up(8 * S * d.H, 256);
     L.total = o;
     return L;
 }
@@ -229,7 +242,7 @@ int moe_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* perm,
 
 size_t moe_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
-    return ws_layout(*d, T_max).total;
+    return ws_layout(*d, T_max, g_tc_min_rows.load()).total;
 }
 
 }  // extern "C"
@@ -243,18 +256,20 @@ namespace {
 // launch that writes those tables.
 int forward_impl(const Options& opt, const moe_dims* d, const float* logits, const void* x_bf16, int32_t* topk_idx,
                  float* gates, int32_t* perm, int32_t* pos, int32_t* offsets, const void* packed, void* y_bf16,
-                 void* ws, size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
+                 void* ws, size_t ws_bytes, int32_t* flag_word, const moe_debug* dbg, cudaStream_t stream) {
     if (int rc = check_dims(d, true)) return rc;
     if (!ws || !packed || !offsets) return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if (d->T > 0 && (!x_bf16 || !topk_idx || !gates || !perm || !pos || !y_bf16))
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if (!aligned(ws, 256) || !aligned(packed, 256) || !aligned(x_bf16, 16) || !aligned(y_bf16, 16))
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws/packed need 256-byte, x/y 16-byte alignment");
-    const WsLayout L = ws_layout(*d, d->T);
+    const WsLayout L = ws_layout(*d, d->T, opt.tc_min_rows);
     if (ws_bytes < L.total)
-        return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws_bytes %zu < %zu", ws_bytes, L.total);
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_forward: ws_bytes %zu < %zu (the size depends on MOE_OPT_TC_MIN_ROWS: size the "
+                    "workspace after setting it)", ws_bytes, L.total);
     char* w = (char*)ws;
-    int32_t* flag = (int32_t*)(w + L.flag);
+    int32_t* flag = flag_word ? flag_word : (int32_t*)(w + L.flag);
     if (d->T == 0) {  // no kernel runs; otherwise the first kernel clears the word
         cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int32_t), stream);
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_forward memset");
@@ -293,6 +308,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     uint8_t* px = (uint8_t*)(w + L.px);
     uint8_t* ph = (uint8_t*)(w + L.ph);
     int32_t* poff = (int32_t*)(w + L.poff);
+    int32_t* soff = (int32_t*)(w + L.soff);
     int32_t* prow = (int32_t*)(w + L.prow);
     int32_t* etc = (int32_t*)(w + L.etc);
     float* hbuf = (float*)(w + L.hbuf);
@@ -300,7 +316,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (logits) {
         MOE_TRY(moe::launch_layer_front(logits, x_bf16, packed, T, H, I, E, k, group, topk_idx, gates, perm, pos,
                                         offsets,
-                                        uoff1, uoff2, toff1, toff2, poff, etc, prow, xq, sx, xinit,
+                                        uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, xq, sx, xinit,
                                         dbg ? dbg->xq : nullptr, dbg ? dbg->sx : nullptr, gacc, yacc, flag,
                                         stream),
                 "route + sort + x quant + plan");
@@ -309,7 +325,8 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
         MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? opt.tc_min_rows : 0x7fffffff,
-                                      group, uoff1, uoff2, toff1, toff2, poff, etc, prow, gacc, yacc, flag, stream),
+                                      group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
+                                      stream),
                 "plan + row state");
     }
     if (use_tc)
@@ -317,25 +334,25 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                             uoff1, E, gacc, flag, I, P, group, stream), "W1");
+                             uoff1, soff, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
                                     offsets, toff1, E, flag, sx, perm, k, hbuf, opt.tc_pair, opt.wait_ns, withhold,
                                     stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
-    MOE_TRY(moe::launch_hquant(gacc, hbuf, etc, topk_idx, sx, perm, prow, L.plane_rows, ph, P, k, E, I, hq,
-                               sh, hinit, dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
+    MOE_TRY(moe::launch_hquant(gacc, hbuf, sx, perm, prow, L.plane_rows, L.stream_rows, ph, P, k, I, hq, sh,
+                               hinit, dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
             "SwiGLU + h quant + h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                             uoff2, E, yacc, flag, 0, P, group, stream), "W2");
+                             uoff2, soff, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
                                     offsets, toff2, E, flag, sh, perm, 0, yf, opt.tc_pair, opt.wait_ns, 0, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
-    MOE_TRY(moe::launch_combine(yacc, yf, etc, topk_idx, sh, gates, pos, T, k, E, H, y_bf16, flag, stream),
+    MOE_TRY(moe::launch_combine(yacc, yf, prow, L.stream_rows, sh, gates, pos, T, k, H, y_bf16, flag, stream),
             "combine");
 #undef MOE_TRY
     return MOE_OK;
@@ -351,21 +368,24 @@ int moe_forward(const moe_dims* d, const void* x_bf16, const int32_t* topk_idx, 
     g_last_error.clear();
     return forward_impl(load_options(), d, nullptr, x_bf16, const_cast<int32_t*>(topk_idx), const_cast<float*>(gates),
                         const_cast<int32_t*>(perm), const_cast<int32_t*>(pos), const_cast<int32_t*>(offsets),
-                        packed, y_bf16, ws, ws_bytes, dbg, stream);
+                        packed, y_bf16, ws, ws_bytes, nullptr, dbg, stream);
 }
 
-// Whole-layer workspace: forward workspace, then idx/gates/perm/pos/offsets,
-// then the sort scratch.
+// Whole-layer workspace: the call's device error word, then
+// idx/gates/perm/pos/offsets and the sort scratch (their offsets depend on T,
+// k and E only, so moe_layer_tables needs no option), then the forward
+// workspace (whose own error-word slot is not used: the layer's kernels report
+// into the word at offset 0).
 struct LayerWs {
-    size_t fwd, idx, gates, perm, pos, offsets, sortws, sort_bytes, total;
+    size_t flag, fwd, idx, gates, perm, pos, offsets, sortws, sort_bytes, total;
 };
 
-static LayerWs layer_ws(const moe_dims& d, long long T) {
+static LayerWs layer_ws(const moe_dims& d, long long T, int tc_min) {
     using moe::align_up;
     LayerWs L;
     const size_t P = (size_t)T * d.k;
     size_t o = 0;
-    L.fwd = o; o += ws_layout(d, T).total;
+    L.flag = o; o += 256;
     L.idx = o; o += align_up(4 * P, 256);
     L.gates = o; o += align_up(4 * P, 256);
     L.perm = o; o += align_up(4 * P, 256);
@@ -373,14 +393,15 @@ static LayerWs layer_ws(const moe_dims& d, long long T) {
     L.offsets = o; o += align_up(4 * (size_t)(d.E + 1), 256);
     L.sortws = o;
     L.sort_bytes = moe::sort_workspace_bytes((int)T, d.k, d.E);
-    o += L.sort_bytes;
+    o += align_up(L.sort_bytes, 256);
+    L.fwd = o; o += ws_layout(d, T, tc_min).total;
     L.total = o;
     return L;
 }
 
 size_t moe_layer_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
-    return layer_ws(*d, T_max).total;
+    return layer_ws(*d, T_max, g_tc_min_rows.load()).total;
 }
 
 int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16, const void* packed,
@@ -391,24 +412,26 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
     if (!ws || !packed || (d->T > 0 && (!logits || !x_bf16 || !y_bf16)))
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: NULL pointer");
     if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: ws must be 256-byte aligned");
-    const LayerWs L = layer_ws(*d, d->T);
+    const Options opt = load_options();
+    const LayerWs L = layer_ws(*d, d->T, opt.tc_min_rows);
     if (ws_bytes < L.total)
-        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: ws_bytes %zu < %zu", ws_bytes, L.total);
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_layer_forward: ws_bytes %zu < %zu (the size depends on MOE_OPT_TC_MIN_ROWS: size the "
+                    "workspace after setting it)", ws_bytes, L.total);
     char* w = (char*)ws;
     int32_t* idx = (int32_t*)(w + L.idx);
     float* gates = (float*)(w + L.gates);
     int32_t* perm = (int32_t*)(w + L.perm);
     int32_t* pos = (int32_t*)(w + L.pos);
     int32_t* offsets = (int32_t*)(w + L.offsets);
-    const Options opt = load_options();
     if (d->T > 0 && d->T < opt.tc_min_rows && (long long)d->T * d->k <= moe::kFrontMaxPairs)
         return forward_impl(opt, d, logits, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
-                            L.idx - L.fwd, dbg, stream);
+                            L.total - L.fwd, (int32_t*)(w + L.flag), dbg, stream);
     if (int rc = moe_route(logits, d->T, d->E, d->k, idx, gates, stream)) return rc;
     if (int rc = moe_sort(idx, d->T, d->k, d->E, perm, pos, offsets, w + L.sortws, L.sort_bytes, stream))
         return rc;
     return forward_impl(opt, d, nullptr, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
-                        L.idx - L.fwd, dbg, stream);
+                        L.total - L.fwd, (int32_t*)(w + L.flag), dbg, stream);
 }
 
 int moe_layer_tables(const moe_dims* d, void* ws, int32_t** topk_idx, float** gates, int32_t** perm,
@@ -417,7 +440,7 @@ int moe_layer_tables(const moe_dims* d, void* ws, int32_t** topk_idx, float** ga
     if (int rc = check_dims(d, true)) return rc;
     if (!ws || !topk_idx || !gates || !perm || !pos || !offsets)
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_tables: NULL pointer");
-    const LayerWs L = layer_ws(*d, d->T);
+    const LayerWs L = layer_ws(*d, d->T, 1);   // (the tables' offsets do not depend on the threshold)
     char* w = (char*)ws;
     *topk_idx = (int32_t*)(w + L.idx);
     *gates = (float*)(w + L.gates);

@@ -1,6 +1,7 @@
 // Gate-weighted combine back to token order (the "mixture" of the routed
 // mixture-of-experts, "DeepSeek-V4-Flash on AMD gfx90a", abstract):
-//   Y[i, n] = fp32(fp64(sh[i]) * acc[i, n])   (streaming-GEMM rows: fp64 sums)
+//   Y[i, n] = fp32(fp64(sh[i]) * acc[s, n])   (streaming-GEMM rows: fp64 sums
+//                                               at the row's streaming row s)
 //   Y[i, n] read as is                         (tensor-core rows: final fp32)
 //   y[t, n] = bf16( sum_{j<k} gates[t,j] * Y[pos[t*k+j], n] ), fp32, slot order.
 // Deterministic gather: each output element is owned by one thread, no atomics.
@@ -17,15 +18,14 @@ namespace moe {
 template <int KMAX>
 __global__ void __launch_bounds__(256)
     k_combine(const double* __restrict__ yacc, const float* __restrict__ yf,
-              const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
-              const float* __restrict__ sh, const float* __restrict__ gates,
-              const int32_t* __restrict__ pos, int P, int k, int E, int H, uint2* __restrict__ y,
-              int32_t* flag) {
+              const int32_t* __restrict__ plane_row, int stream_rows, const float* __restrict__ sh,
+              const float* __restrict__ gates, const int32_t* __restrict__ pos, int P, int k, int H,
+              uint2* __restrict__ y, int32_t* flag) {
     pdl_begin();
     const int t = blockIdx.y;
     const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
     if (4 * n4 >= H) return;
-    int row[KMAX];
+    int row[KMAX], srow[KMAX];
     float g[KMAX];
     bool tc[KMAX];
 #pragma unroll
@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(256)
             const int p = t * k + j;
             row[j] = checked_index(__ldg(pos + p), P, flag);
             g[j] = __ldg(gates + p);
-            tc[j] = __ldg(expert_tc + checked_index(__ldg(topk_idx + p), E, flag)) != 0;
+            const int slot = __ldg(plane_row + row[j]);   // >= 0: tensor-core row; else ~streaming row
+            tc[j] = slot >= 0;
+            srow[j] = tc[j] ? 0 : checked_index(~slot, stream_rows, flag);
         }
     }
     float4 v[KMAX];
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(256)
                 v[j] = __ldg(reinterpret_cast<const float4*>(yf + (size_t)row[j] * H) + n4);
             } else {
                 const double s = (double)__ldg(sh + row[j]);
-                const double2* r = reinterpret_cast<const double2*>(yacc + (size_t)row[j] * H) + 2 * n4;
+                const double2* r = reinterpret_cast<const double2*>(yacc + (size_t)srow[j] * H) + 2 * n4;
                 const double2 d0 = __ldg(r), d1 = __ldg(r + 1);
                 v[j] = make_float4((float)__dmul_rn(s, d0.x), (float)__dmul_rn(s, d0.y), (float)__dmul_rn(s, d1.x),
                                    (float)__dmul_rn(s, d1.y));
@@ -68,17 +70,16 @@ __global__ void __launch_bounds__(256)
                                              *reinterpret_cast<const uint32_t*>(&hi));
 }
 
-cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
-                           const int32_t* topk_idx, const float* sh, const float* gates,
-                           const int32_t* pos, int T, int k, int E, int H, void* y, int32_t* flag,
-                           cudaStream_t st) {
+cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
+                           const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,
+                           int32_t* flag, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     dim3 grid((H / 4 + 255) / 256, T);
     const cudaError_t e =
-        k <= 8 ? launch_pdl(k_combine<8>, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates, pos, T * k,
-                            k, E, H, (uint2*)y, flag)
-               : launch_pdl(k_combine<16>, grid, dim3(256), 0, st, yacc, yf, expert_tc, topk_idx, sh, gates, pos,
-                            T * k, k, E, H, (uint2*)y, flag);
+        k <= 8 ? launch_pdl(k_combine<8>, grid, dim3(256), 0, st, yacc, yf, plane_row, stream_rows, sh, gates, pos,
+                            T * k, k, H, (uint2*)y, flag)
+               : launch_pdl(k_combine<16>, grid, dim3(256), 0, st, yacc, yf, plane_row, stream_rows, sh, gates,
+                            pos, T * k, k, H, (uint2*)y, flag);
     count_launches(1);
     return e;
 }

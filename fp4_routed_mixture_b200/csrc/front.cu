@@ -34,7 +34,7 @@ struct FrontArgs {
     int32_t* perm;              // [P]
     int32_t* pos;               // [P]
     int32_t* offsets;           // [E + 1]
-    int32_t *unit_off1, *unit_off2, *tile_off1, *tile_off2, *plane_off, *expert_tc, *plane_row;
+    int32_t *unit_off1, *unit_off2, *tile_off1, *tile_off2, *plane_off, *stream_off, *expert_tc, *plane_row;
     int8_t* xq;
     float* sx;
     int32_t* xinit;
@@ -66,8 +66,10 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
         // no expert reaches the tensor-core threshold: plan with an unreachable one
         if (threadIdx.x < 32)
             plan_warp(offs, a.E, P, 2 * a.I, a.H, 0x7fffffff, a.group, a.unit_off1, a.unit_off2, a.tile_off1,
-                      a.tile_off2, a.plane_off, a.expert_tc, a.flag, true, ps);
-        for (int i = threadIdx.x; i < P; i += blockDim.x) a.plane_row[i] = -1;
+                      a.tile_off2, a.plane_off, a.stream_off, a.expert_tc, a.flag, true, ps);
+        // every row is a streaming row and every expert's streaming rows start
+        // at its sorted offset, so sorted row i is streaming row i
+        for (int i = threadIdx.x; i < P; i += blockDim.x) a.plane_row[i] = ~i;
         return;
     }
     if ((int)blockIdx.x <= a.T) {
@@ -86,13 +88,13 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
 cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
                                int E, int k, int group, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
                                int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
-                               int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc, int32_t* plane_row,
-                               int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq, float* dbg_sx,
-                               double* gacc, double* yacc, int32_t* flag, cudaStream_t st) {
+                               int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
+                               int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
+                               float* dbg_sx, double* gacc, double* yacc, int32_t* flag, cudaStream_t st) {
     const int P = T * k;
     if (T < 1 || P > kFrontMaxPairs || E > kMaxExperts) return cudaErrorInvalidValue;
     FrontArgs a{logits, (const __nv_bfloat16*)x, packed, T, H, I, E, k, group, topk_idx, gates, perm, pos, offsets,
-                unit_off1, unit_off2, tile_off1, tile_off2, plane_off, expert_tc, plane_row, xq, sx, xinit,
+                unit_off1, unit_off2, tile_off1, tile_off2, plane_off, stream_off, expert_tc, plane_row, xq, sx, xinit,
                 dbg_xq, dbg_sx, gacc, yacc, flag};
     const dim3 grid(1 + T + P), block(kSortThreads);
     cudaError_t e;

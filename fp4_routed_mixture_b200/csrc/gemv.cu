@@ -137,11 +137,12 @@ struct GemvArgs {
     const int8_t* act;         // activation codes, rows of K bytes
     const int32_t* act_init;   // rows of K/32 block terms
     const int32_t* perm;       // sorted row -> pair id
-    int k_div;                 // >0: activation row = perm[i] / k_div; 0: = i
+    int k_div;                 // >0: activation row = perm[i] / k_div (sorted row i); 0: = the streaming row
     const int32_t* offsets;    // [E+1]
     const int32_t* unit_off;   // [E+1] exclusive scan of units per expert
+    const int32_t* stream_off; // [E+1] first compact streaming row of each expert
     int E;
-    double* out;               // [P, N] fp64 accumulators, zeroed
+    double* out;               // [streaming rows, N] fp64 accumulators, zeroed
     const int32_t* flag;       // device error word: a layout mismatch stops the kernel
     int gate_up_half;          // > 0 (= I) for W1: device rows interleave gate and up rows
     int P;                     // pairs (rows of the sorted tables)
@@ -155,9 +156,9 @@ __device__ __forceinline__ int canonical_row(int d, int gate_up_half) {
     return (r < 16) ? tau * 16 + r : gate_up_half + tau * 16 + (r - 16);
 }
 
-// A unit: expert, tile, first sorted row, number of rows.
+// A unit: expert, tile, first sorted row, its compact streaming row, number of rows.
 struct Unit {
-    int id, e, tile, i0, mc;
+    int id, e, tile, i0, o0, mc;
 };
 
 template <int G>
@@ -175,12 +176,15 @@ __device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
     const int local = unit - __ldg(a.unit_off + lo);
     u.tile = local / ngroups;
     u.i0 = r0 + (local % ngroups) * G;
+    u.o0 = __ldg(a.stream_off + lo) + (u.i0 - r0);
     u.mc = min(G, r1 - u.i0);
     return u;
 }
 
-__device__ __forceinline__ int act_row(const GemvArgs& a, int i) {
-    return a.k_div ? checked_index(__ldg(a.perm + i), a.P, const_cast<int32_t*>(a.flag)) / a.k_div : i;
+// Activation row of row m of unit u: the token (W1) or the streaming row (W2).
+__device__ __forceinline__ int act_row(const GemvArgs& a, const Unit& u, int m) {
+    return a.k_div ? checked_index(__ldg(a.perm + u.i0 + m), a.P, const_cast<int32_t*>(a.flag)) / a.k_div
+                   : u.o0 + m;
 }
 
 // Integer dot product of one 32-element block (8 decoded words) with one
@@ -265,8 +269,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
         g_sc = lane * 16 + t * 4;
         g_code = 512 + t * 512 + lane * 16;
         f_w = a.w + (size_t)fu.e * a.expert_bytes + ((size_t)rb * KG + kg) * kChunkBytes;
-        f_x = a.act + (size_t)act_row(a, fu.i0 + min(lane >> 3, fu.mc - 1)) * a.K + kg * 128 + (lane & 7) * 16;
-        f_i = a.act_init + (size_t)act_row(a, fu.i0 + min(lane & (kGroup - 1), fu.mc - 1)) * (a.K / 32) +
+        f_x = a.act + (size_t)act_row(a, fu, min(lane >> 3, fu.mc - 1)) * a.K + kg * 128 + (lane & 7) * 16;
+        f_i = a.act_init + (size_t)act_row(a, fu, min(lane & (kGroup - 1), fu.mc - 1)) * (a.K / 32) +
               kg * 4;
     };
     start_unit(f_kg);
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
                 const int n = canonical_row((cu.tile * TP + u) * 32 + lane, a.gate_up_half);
 #pragma unroll
                 for (int m = 0; m < kGroup; ++m) {
-                    if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.i0 + m) * a.N + n, acc[u][m]);
+                    if (m < cu.mc) atomicAdd(a.out + (size_t)(cu.o0 + m) * a.N + n, acc[u][m]);
                     acc[u][m] = 0.0;
                 }
             }
@@ -400,9 +404,9 @@ static int gemv_grid() {
 
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
-                        const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st) {
-    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, E, out, flag,
+                        const int32_t* offsets, const int32_t* unit_off, const int32_t* stream_off, int E,
+                        double* out, const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st) {
+    GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, stream_off, E, out, flag,
                gate_up_half, P, 0u};
     const int grid = group == 2 ? gemv_grid<2>() : gemv_grid<4>();
     if (grid <= 0) return cudaErrorInvalidConfiguration;

@@ -77,8 +77,9 @@ void count_launches(int n);
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
                              int I, int H, int tc_min, int group, int32_t* unit_off1, int32_t* unit_off2,
-                             int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc,
-                             int32_t* plane_row, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
+                             int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off,
+                             int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc, int32_t* flag,
+                             cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may be
 // scheduled before the preceding kernel in the stream completes.  Every kernel
@@ -117,9 +118,9 @@ constexpr int kFrontMaxPairs = 1024;
 cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
                                int E, int k, int group, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
                                int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
-                               int32_t* tile_off2, int32_t* plane_off, int32_t* expert_tc, int32_t* plane_row,
-                               int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq, float* dbg_sx,
-                               double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
+                               int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
+                               int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
+                               float* dbg_sx, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
 
 size_t sort_workspace_bytes(int T_max, int k, int E);
 cudaError_t launch_sort(const int32_t* topk_idx, int T, int k, int E, int32_t* perm, int32_t* pos,
@@ -139,11 +140,10 @@ const int32_t* packed_flag_ptr(const void* packed);
 cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, int32_t* xinit,
                           uint8_t* tplanes, int8_t* dbg_xq, float* dbg_sx, const void* packed, int I, int E,
                           int32_t* flag, cudaStream_t st);
-cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
-                          const int32_t* topk_idx, const float* sx, const int32_t* perm,
-                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
-                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
-                          int32_t* flag, cudaStream_t st);
+cudaError_t launch_hquant(const double* gacc, float* hbuf, const float* sx, const int32_t* perm,
+                          const int32_t* plane_row, int plane_rows, int stream_rows, uint8_t* planes, int P, int k,
+                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag,
+                          cudaStream_t st);
 
 cudaError_t launch_exp(const float* x, float* y, int64_t n, cudaStream_t st);
 cudaError_t launch_swiglu(const float* g, const float* u, float* h, int64_t n, cudaStream_t st);
@@ -153,8 +153,8 @@ cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, flo
 
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
-                        const int32_t* offsets, const int32_t* unit_off, int E, double* out,
-                        const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st);
+                        const int32_t* offsets, const int32_t* unit_off, const int32_t* stream_off, int E,
+                        double* out, const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st);
 
 size_t tc_smem_bytes();
 // Digit planes, per 128-input stage g and group of 8 plane rows, hold
@@ -173,9 +173,8 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
                            uint64_t wait_ns, int withhold, cudaStream_t st);
 
-cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc,
-                           const int32_t* topk_idx, const float* sh, const float* gates,
-                           const int32_t* pos, int T, int k, int E, int H, void* y, int32_t* flag,
-                           cudaStream_t st);
+cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
+                           const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,
+                           int32_t* flag, cudaStream_t st);
 
 }  // namespace moe

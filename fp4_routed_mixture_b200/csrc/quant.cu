@@ -52,13 +52,11 @@ __global__ void __launch_bounds__(kQThreads)
 // the values in registers for pass 2 instead of reading them again.
 template <int R, int KEEP>
 __global__ void __launch_bounds__(kQThreads)
-    k_hquant(const double* __restrict__ gacc, float* __restrict__ hbuf,
-             const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ topk_idx,
-             const float* __restrict__ sx, const int32_t* __restrict__ perm,
-             const int32_t* __restrict__ plane_row, int plane_rows, uint8_t* __restrict__ planes,
-             int P, int k, int E, int I, int8_t* __restrict__ hq, float* __restrict__ sh,
-             int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq, float* __restrict__ dbg_sh,
-             int32_t* flag) {
+    k_hquant(const double* __restrict__ gacc, float* __restrict__ hbuf, const float* __restrict__ sx,
+             const int32_t* __restrict__ perm, const int32_t* __restrict__ plane_row, int plane_rows,
+             int stream_rows, uint8_t* __restrict__ planes, int P, int k, int I, int8_t* __restrict__ hq,
+             float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
+             float* __restrict__ dbg_sh, int32_t* flag) {
     pdl_begin();
     static_assert(R == 32 || R == kQThreads, "a warp or a CTA per row");
     float4 keep[KEEP > 0 ? KEEP : 1];
@@ -71,14 +69,16 @@ __global__ void __launch_bounds__(kQThreads)
     const int steps = I / (4 * R);          // I % 128 == 0; for R = 256 also I % 1024 == 0 (checked by the launcher)
     for (int i0 = blockIdx.x * rows_per_cta; i0 < P; i0 += gridDim.x * rows_per_cta) {
         const int i = i0 + (int)threadIdx.x / R;
-        const bool row_ok = i < P;           // (R = 256: always)
+        // (R = 256: always in range; a row's R threads take the same branches)
+        const int slot = i < P ? plane_row[i] : kNoRow;
+        const bool tc = slot >= 0;
+        const int srow = ~slot;              // streaming row (slot < 0)
+        const bool slot_ok = tc ? slot < plane_rows : (slot != kNoRow && srow < stream_rows);
+        if (i < P && !slot_ok && threadIdx.x % R == 0) raise_flag(flag, FLAG_BOUNDS);
+        const bool row_ok = i < P && slot_ok;
         float a = 0.0f;
-        bool tc = false;
         int p = 0;
-        if (row_ok) {
-            p = checked_index(perm[i], P, flag);
-            tc = expert_tc[checked_index(topk_idx[p], E, flag)] != 0;
-        }
+        if (row_ok) p = checked_index(perm[i], P, flag);
         float4* hr = reinterpret_cast<float4*>(hbuf + (size_t)(row_ok ? i : 0) * I);
         if (row_ok && tc) {
             if (KEEP > 0) {
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kQThreads)
             }
         } else if (row_ok) {
             const double s = (double)sx[p / k];
-            const double* gr = gacc + (size_t)i * 2 * I;
+            const double* gr = gacc + (size_t)srow * 2 * I;
             for (int g = 0; g < steps; ++g) {
                 const int e0 = 4 * (g * R + l);
                 float hv[4];
@@ -122,14 +122,7 @@ __global__ void __launch_bounds__(kQThreads)
             sh[i] = sc;
             if (dbg_sh) dbg_sh[i] = sc;
         }
-        int pr = -1;
-        if (tc) {
-            pr = plane_row[i];
-            if (pr >= plane_rows || pr < 0) {
-                if (l == 0) raise_flag(flag, FLAG_BOUNDS);
-                pr = -1;
-            }
-        }
+        const int pr = tc ? slot : -1;
 #pragma unroll(KEEP > 0 ? KEEP : 4)
         for (int g = 0; g < steps; ++g) {
             const int e0 = 4 * (g * R + l);
@@ -148,12 +141,12 @@ __global__ void __launch_bounds__(kQThreads)
                                     (uint32_t)(q[2] & 0xff) << 16 | (uint32_t)(q[3] & 0xff) << 24;
             if (dbg_hq) *reinterpret_cast<uint32_t*>(dbg_hq + (size_t)i * I + e0) = packed;
             if (!tc) {
-                *reinterpret_cast<uint32_t*>(hq + (size_t)i * I + e0) = packed;
+                *reinterpret_cast<uint32_t*>(hq + (size_t)srow * I + e0) = packed;
                 int bsum = q[0] + q[1] + q[2] + q[3];
                 bsum += __shfl_xor_sync(0xffffffffu, bsum, 1);
                 bsum += __shfl_xor_sync(0xffffffffu, bsum, 2);
                 bsum += __shfl_xor_sync(0xffffffffu, bsum, 4);
-                if ((l & 7) == 0) hinit[(size_t)i * (I / 32) + (e0 >> 5)] = -12 * bsum;
+                if ((l & 7) == 0) hinit[(size_t)srow * (I / 32) + (e0 >> 5)] = -12 * bsum;
             } else if (pr >= 0) {
                 // 4 codes = 16 bits of each plane's 16-byte piece of chunk e0/32
                 uint32_t d[3] = {0u, 0u, 0u};
@@ -228,26 +221,25 @@ cudaError_t launch_xquant(const void* x, int T, int H, int8_t* xq, float* sx, in
     return e;
 }
 
-cudaError_t launch_hquant(const double* gacc, float* hbuf, const int32_t* expert_tc,
-                          const int32_t* topk_idx, const float* sx, const int32_t* perm,
-                          const int32_t* plane_row, int plane_rows, uint8_t* planes, int P, int k, int E,
-                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh,
-                          int32_t* flag, cudaStream_t st) {
+cudaError_t launch_hquant(const double* gacc, float* hbuf, const float* sx, const int32_t* perm,
+                          const int32_t* plane_row, int plane_rows, int stream_rows, uint8_t* planes, int P, int k,
+                          int I, int8_t* hq, float* sh, int32_t* hinit, int8_t* dbg_hq, float* dbg_sh, int32_t* flag,
+                          cudaStream_t st) {
     if (P == 0) return cudaSuccess;
     // few rows (decode): a CTA per row keeps every row's chain short; many
     // rows (prefill): a warp per row needs no block barriers
     cudaError_t e;
     if (P < 4096 && I % (4 * kQThreads) == 0) {
-        e = launch_pdl(k_hquant<kQThreads, 0>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf,
-                       expert_tc, topk_idx, sx, perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit,
-                       dbg_hq, dbg_sh, flag);
+        e = launch_pdl(k_hquant<kQThreads, 0>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf, sx,
+                       perm, plane_row, plane_rows, stream_rows, planes, P, k, I, hq, sh, hinit, dbg_hq, dbg_sh,
+                       flag);
     } else {
         const int warps = kQThreads / 32;
         const int grid = std::min((P + warps - 1) / warps, 148 * 8);
         // (keeping a row in registers between the passes, k_hquant<32, 16>,
         // measured slower: 112 registers halve the rows in flight)
-        e = launch_pdl(k_hquant<32, 0>, dim3(grid), dim3(kQThreads), 0, st, gacc, hbuf, expert_tc, topk_idx, sx,
-                       perm, plane_row, plane_rows, planes, P, k, E, I, hq, sh, hinit, dbg_hq, dbg_sh, flag);
+        e = launch_pdl(k_hquant<32, 0>, dim3(grid), dim3(kQThreads), 0, st, gacc, hbuf, sx, perm, plane_row,
+                       plane_rows, stream_rows, planes, P, k, I, hq, sh, hinit, dbg_hq, dbg_sh, flag);
     }
     count_launches(1);
     return e;

@@ -313,23 +313,33 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 // x `group` tokens, the group size the streaming GEMM is launched with).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
-// tile starts on a 16-row boundary of the plane buffers), and expert_tc[e] = 1
-// for tensor-core experts.  Run by one warp; lane l owns a contiguous slice of
+// tile starts on a 16-row boundary of the plane buffers), of the rows of
+// streaming experts (their compact streaming rows), and expert_tc[e] = 1 for
+// tensor-core experts.  Run by one warp; lane l owns a contiguous slice of
 // experts.  The tables go to ps (shared memory) and, with global_out, to the
 // global tables the GEMM launches index.
 struct PlanShared {
     int32_t plane_off[kMaxExperts];
+    int32_t stream_off[kMaxExperts];
     uint8_t tc[kMaxExperts];
     int32_t units1;   // streaming units of W1 (0: no streaming rows)
 };
+
+// The per-row slot table (plane_row) the planner writes for every sorted row:
+// a value >= 0 is the digit-plane row of a tensor-core row; a negative value v
+// marks a streaming row whose compact streaming row is ~v (its fp64
+// accumulators, h codes and block terms live at that row of buffers sized for
+// the streaming rows only); kNoRow marks a row that failed the planner's
+// bounds check (its kernels skip it).
+constexpr int32_t kNoRow = INT32_MIN;
 
 static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
                                  int group,
                                  int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                                  int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
-                                 int32_t* __restrict__ plane_off, int32_t* __restrict__ expert_tc, int32_t* flag,
-                                 bool global_out, PlanShared& ps) {
-    constexpr int NS = 5;
+                                 int32_t* __restrict__ plane_off, int32_t* __restrict__ stream_off,
+                                 int32_t* __restrict__ expert_tc, int32_t* flag, bool global_out, PlanShared& ps) {
+    constexpr int NS = 6;
     const int lane = threadIdx.x & 31;
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
@@ -349,6 +359,7 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
         c[2] = nb * (n1 / kTcWeightTile);
         c[3] = nb * (n2 / kTcWeightTile);
         c[4] = tc ? (m + 15) & ~15 : 0;
+        c[5] = tc ? 0 : m;
     };
     int s[NS] = {};
     for (int e = e0; e < e1; ++e) {
@@ -368,12 +379,13 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
     }
     int r[NS];
     for (int j = 0; j < NS; ++j) r[j] = x[j] - s[j];  // exclusive prefix
-    int32_t* outs[NS] = {unit_off1, unit_off2, tile_off1, tile_off2, plane_off};
+    int32_t* outs[NS] = {unit_off1, unit_off2, tile_off1, tile_off2, plane_off, stream_off};
     for (int e = e0; e < e1; ++e) {
         int c[NS];
         counts(e, c);
         const bool tc = !any_bad && (offsets[e + 1] - offsets[e]) >= tc_min;
         ps.plane_off[e] = r[4];
+        ps.stream_off[e] = r[5];
         ps.tc[e] = tc ? 1 : 0;
         if (global_out) {
             for (int j = 0; j < NS; ++j) outs[j][e] = r[j];
