@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tc-pair", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_PAIR for the run (default: the library's default)")
+    ap.add_argument("--tc-a-tmem", type=int, choices=[0, 1], default=None,
+                    help="MOE_OPT_TC_A_TMEM for the run (default: the library's default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
                     help="no timing, no JSON: pack the workload and run --steps layer calls "
@@ -356,6 +358,8 @@ def main():
     import fp4_routed_mixture_b200 as moe
     if a.tc_pair is not None:
         moe.moe_set_option(moe.MOE_OPT_TC_PAIR, a.tc_pair)
+    if a.tc_a_tmem is not None:
+        moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, a.tc_a_tmem)
     rank0 = dist.rank == 0
     peaks = measured_peaks()
     r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
@@ -426,6 +430,7 @@ def main():
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
                 "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
+                "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
             }
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)

@@ -317,6 +317,7 @@ MOE_OPT_TC_MIN_ROWS = 1
 MOE_OPT_TC_PAIR = 2
 MOE_OPT_WAIT_LIMIT_US = 3
 MOE_OPT_TEST_TIMEOUT = 4
+MOE_OPT_TC_A_TMEM = 5
 
 
 def moe_set_option(option: int, value: int):

@@ -59,15 +59,18 @@ std::atomic<int> g_tc_min_rows{32};        // experts with at least this many ro
 std::atomic<int> g_tc_pair{0};             // tensor-core GEMM in SM pairs (cta_group::2) where the shape allows
 std::atomic<int> g_wait_limit_us{1000000}; // limit of the tensor-core GEMM's bounded waits
 std::atomic<int> g_test_timeout{0};        // one-shot: the next tensor-core launch withholds a stage
+std::atomic<int> g_tc_a_tmem{0};           // tensor-core GEMM with the weight operand staged in TMEM
 
 struct Options {
     int tc_min_rows;
     bool tc_pair;
+    bool tc_a_tmem;
     uint64_t wait_ns;
 };
 
 Options load_options() {
-    return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, 1000ull * (uint64_t)g_wait_limit_us.load()};
+    return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, g_tc_a_tmem.load() != 0,
+                   1000ull * (uint64_t)g_wait_limit_us.load()};
 }
 
 struct WsLayout {
@@ -337,8 +340,8 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                              uoff1, soff, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, opt.tc_pair, opt.wait_ns, withhold,
-                                    stream),
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns,
+                                    withhold, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_hquant(gacc, hbuf, sx, perm, prow, L.plane_rows, L.stream_rows, ph, P, k, I, hq, sh,
@@ -349,7 +352,8 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                              uoff2, soff, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, opt.tc_pair, opt.wait_ns, 0, stream),
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns, 0,
+                                    stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, yf, prow, L.stream_rows, sh, gates, pos, T, k, H, y_bf16, flag, stream),
@@ -486,6 +490,11 @@ int moe_set_option(int option, int value) {
         g_tc_pair = value;
         return MOE_OK;
     }
+    if (option == MOE_OPT_TC_A_TMEM) {
+        if (value != 0 && value != 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_A_TMEM must be 0 or 1");
+        g_tc_a_tmem = value;
+        return MOE_OK;
+    }
     if (option == MOE_OPT_WAIT_LIMIT_US) {
         if (value < 1 || value > 10000000)
             return fail(MOE_ERR_INVALID_ARG, "moe_set_option: WAIT_LIMIT_US must be in [1, 10^7]");
@@ -504,6 +513,7 @@ int moe_get_option(int option) {
     if (option == MOE_OPT_TC_MIN_ROWS) return g_tc_min_rows;
     if (option == MOE_OPT_TC_PAIR) return g_tc_pair;
     if (option == MOE_OPT_WAIT_LIMIT_US) return g_wait_limit_us;
+    if (option == MOE_OPT_TC_A_TMEM) return g_tc_a_tmem;
     if (option == MOE_OPT_TEST_TIMEOUT) return g_test_timeout;
     return -1;
 }

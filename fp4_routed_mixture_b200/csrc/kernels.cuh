@@ -171,7 +171,7 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           uint64_t wait_ns, int withhold, cudaStream_t st);
+                           bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,

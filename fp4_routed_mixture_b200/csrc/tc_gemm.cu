@@ -75,6 +75,19 @@ constexpr int TC_SF_PIPE_COLS = 4 * TC_STAGES + 12;
 static_assert(TC_SF_COL + TC_PIPES * TC_SF_PIPE_COLS <= TC_TMEM_COLS, "accumulators and scale factors exceed TMEM");
 static_assert(TC_SF_COL % 4 == 0 && TC_SF_PIPE_COLS % 4 == 0, "scale-factor columns hold 4 bytes per lane");
 static_assert(TC_BN % 32 == 0 && TC_BN <= 256, "MMA N, whole column chunks");
+// The A-in-TMEM form (ATMEM): every stage's weight chunk is copied into TMEM
+// once (tcgen05.cp, two 128 x 256-bit halves, 16 columns) and the six plane
+// MMAs read A from there, so shared memory feeds only B.  Columns: the
+// accumulators, then per pipe r and stage s the A slot at TC_AT_A + 48r + 16s,
+// the A scale factors at TC_AT_SFA + 12r + 4s, and two constant B scale
+// regions shared by the pipes: X (bytes 2^6, 2^6, 2^3, 2^3 in every 4-byte
+// group) serves planes 0 and 1 through the scale-factor byte selector (0 and
+// 2), Y (all 2^0) plane 2.
+constexpr int TC_AT_A = TC_ACC * TC_BN;
+constexpr int TC_AT_SFA = TC_AT_A + TC_PIPES * TC_STAGES * 16;
+constexpr int TC_AT_SFB = TC_AT_SFA + TC_PIPES * TC_STAGES * 4;
+static_assert(TC_AT_SFB + 8 <= TC_TMEM_COLS, "A slots and scale factors exceed TMEM");
+static_assert(TC_AT_A % 16 == 0, "A slots on 16-column boundaries");
 
 struct TcShared {
     uint8_t stage[TC_PIPES][TC_STAGES][TC_STAGE_BYTES];
@@ -82,6 +95,7 @@ struct TcShared {
     float col_scale[TC_EPI_WARPS][32];  // per epilogue warp: activation scale of its 32 columns
     uint64_t full[TC_PIPES][TC_STAGES], empty[TC_PIPES][TC_STAGES], acc_full[TC_ACC], acc_empty[TC_ACC];
     uint64_t drain[TC_PIPES];   // each issuer's last commit: all of its MMAs are done
+    uint64_t sfb_ready;         // ATMEM: the shared B scale regions are in TMEM
     uint32_t tmem_base;
     int32_t abort;
 };
@@ -188,6 +202,21 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 }
 __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Copies a 128-row x 32-byte K-major matrix (two 16-byte core-matrix columns,
+// LBO apart) into 128 TMEM lanes x 8 columns.
+__device__ __forceinline__ void tc_cp_a(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// The same MMA with A read from TMEM (lane = row, K packed along columns).
+__device__ __forceinline__ void tc_mma_mxf4_at(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                               uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], [%1], %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
 }
 __device__ __forceinline__ void tc_mma_mxf4(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
@@ -320,8 +349,9 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
 // barrier; a remote arrive joins the even CTA's), the even CTA's MMA commits
 // arrive on the barriers of both CTAs, and the odd CTA's epilogue warps release
 // accumulators with remote arrives.
-template <bool PAIR>
+template <bool PAIR, bool ATMEM>
 __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
+    static_assert(!(PAIR && ATMEM), "the A-in-TMEM form is one CTA per SM");
     pdl_begin();
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
@@ -354,11 +384,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
             mbar_init(smem_u32(&sh.acc_empty[b]), PAIR ? 2 * TC_EPI_WARPS : TC_EPI_WARPS);
         }
         for (int r = 0; r < TC_PIPES; ++r) mbar_init(smem_u32(&sh.drain[r]), 1);
+        mbar_init(smem_u32(&sh.sfb_ready), 1);
         sh.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    for (int i = threadIdx.x; i < 3 * 512; i += TC_THREADS)
-        sh.sfb[i / 512][i % 512] = (uint8_t)(133 - 3 * (i / 512));  // 2^6, 2^3, 2^0
+    for (int i = threadIdx.x; i < 3 * 512; i += TC_THREADS) {
+        const int p = i / 512;
+        if (ATMEM)  // regions X (2^6, 2^6, 2^3, 2^3 per 4 bytes) and Y (2^0)
+            sh.sfb[p][i % 512] = (uint8_t)(p == 0 ? ((i & 3) < 2 ? 133 : 130) : 127);
+        else
+            sh.sfb[p][i % 512] = (uint8_t)(133 - 3 * p);  // 2^6, 2^3, 2^0
+    }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     if (warp == 0) {
         if (PAIR) {
@@ -482,9 +518,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
     } else if (warp < TC_EPI_WARP0) {
         // ---------------- MMA issuer of pipe r (even CTA of a pair) ----------------
         const int r = warp - TC_PIPES;
-        const uint32_t sfa_col = tmem + TC_SF_COL + TC_SF_PIPE_COLS * r;
-        const uint32_t sfb_col = sfa_col + 4 * TC_STAGES;
-        if (lane == 0) {
+        const uint32_t sfa_col = ATMEM ? tmem + TC_AT_SFA + 4 * TC_STAGES * r : tmem + TC_SF_COL + TC_SF_PIPE_COLS * r;
+        const uint32_t sfb_col = ATMEM ? tmem + TC_AT_SFB : sfa_col + 4 * TC_STAGES;
+        const uint32_t a_col = tmem + TC_AT_A + 16 * TC_STAGES * r;
+        bool sfb_ok = true;
+        if (ATMEM) {
+            // pipe 0 copies the two shared B scale regions; pipe 1 waits for them
+            if (lane == 0) {
+                if (r == 0) {
+                    tc_cp_sf(sfb_col, make_sdesc(smem_u32(sh.sfb[0]), 0, 128));
+                    tc_cp_sf(sfb_col + 4, make_sdesc(smem_u32(sh.sfb[1]), 0, 128));
+                    tc_commit(smem_u32(&sh.sfb_ready));
+                } else {
+                    sfb_ok = wait(smem_u32(&sh.sfb_ready), 0);
+                }
+            }
+            sfb_ok = __shfl_sync(0xffffffffu, sfb_ok, 0);
+            if (!sfb_ok) give_up();
+            tc_fence_after();
+        } else if (lane == 0) {
             for (int p = 0; p < 3; ++p) {
                 if (PAIR)
                     tc_cp_sf_pair(sfb_col + 4 * p, make_sdesc(smem_u32(sh.sfb[p]), 0, 128));
@@ -496,7 +548,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
-        for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
+        for (int j = r; j < ntiles && sfb_ok && !*abort; j += TC_PIPES) {
             const TcTile tt = tile_at(a, tile_of(j));
             const int buf = j % TC_ACC;
             const uint32_t use = (uint32_t)(j / TC_ACC);
@@ -521,8 +573,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
                         tc_cp_sf_pair(sfa, make_sdesc(sbase, 0, 128));
                     else
                         tc_cp_sf(sfa, make_sdesc(sbase, 0, 128));
+                    if (ATMEM) {
+                        // the stage's A into its TMEM slot, once for all six MMAs
+                        // (the slot is rewritten only after this stage's MMAs
+                        // have completed: the producer refills the stage after
+                        // their commit)
+                        const uint32_t at = a_col + 16 * stage;
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
+                        for (int ks = 0; ks < 2; ++ks)
+                            tc_cp_a(at + 8 * ks, make_sdesc(sbase + 512 + ks * 2 * 2048, 2048, 128));
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                            for (int p = 0; p < 3; ++p) {
+                                const uint64_t bdesc = make_sdesc(sbase + TC_A_BYTES + p * 512 + ks * 256, 128,
+                                                                  kPlaneGroupBytes);
+                                // planes 0 and 1: region X, bytes 0-1 / 2-3; plane 2: region Y
+                                tc_mma_mxf4_at(dcol, at + 8 * ks, bdesc,
+                                               make_idesc(tt.n_mma, 2 * ks, p == 1 ? 2 : 0), sfa,
+                                               sfb_col + (p == 2 ? 4 : 0), (g | ks | p) != 0);
+                            }
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < (ATMEM ? 0 : 2); ++ks) {
                         const uint64_t adesc = make_sdesc(sbase + 512 + ks * 2 * 2048, 2048, 128);
 #pragma unroll
                         for (int p = 0; p < 3; ++p) {
@@ -705,7 +778,9 @@ static int tc_grid() {
         int dev = 0, sms = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaFuncSetAttribute(k_tc_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_tc_gemm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(TcShared)) != cudaSuccess ||
+            cudaFuncSetAttribute(k_tc_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(TcShared)) != cudaSuccess)
             return -1;
         return sms;
@@ -720,7 +795,7 @@ static int tc_pair_grid() {
     return cache.get([] {
         const int single = tc_grid();
         if (single <= 0) return -1;
-        if (cudaFuncSetAttribute(k_tc_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(k_tc_gemm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(TcShared)) != cudaSuccess) {
             cudaGetLastError();
             return 0;
@@ -737,7 +812,7 @@ static int tc_pair_grid() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true>, &cfg) != cudaSuccess || clusters <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true, false>, &cfg) != cudaSuccess || clusters <= 0) {
             cudaGetLastError();
             return 0;
         }
@@ -762,11 +837,12 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
                            const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           uint64_t wait_ns, int withhold, cudaStream_t st) {
+                           bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st) {
     TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
              E, flag, row_scale, perm, k_div, out, wait_ns, withhold};
-    // the timeout test runs on the one-CTA form (withhold applies to it only)
-    if (withhold) pair = false;
+    // the timeout test runs on the one-CTA form (withhold applies to it only);
+    // the A-in-TMEM form is one CTA per SM
+    if (withhold || a_tmem) pair = false;
     cudaError_t e;
     // the pair takes two adjacent 128-row tiles of one expert: N % 256 == 0
     const int pgrid = (pair && N % (2 * TC_BM) == 0) ? tc_pair_grid() : 0;
@@ -785,11 +861,12 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<true>, a);
+        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<true, false>, a);
     } else {
         const int grid = tc_grid();
         if (grid <= 0) return cudaErrorInvalidConfiguration;
-        e = launch_pdl(k_tc_gemm<false>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a);
+        e = a_tmem ? launch_pdl(k_tc_gemm<false, true>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a)
+                   : launch_pdl(k_tc_gemm<false, false>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a);
     }
     count_launches(1);
     return e;

@@ -261,6 +261,11 @@ int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStre
  *   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
  *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
  *   multiple of 256); 0 one CTA per SM.  Same results.
+ *   MOE_OPT_TC_A_TMEM: 1 stages each pipeline stage's weight chunk in tensor
+ *   memory once (tcgen05.cp) and runs the six digit-plane MMAs of the stage
+ *   with A read from there, so shared memory feeds only the activation
+ *   operand; 0 reads both operands from shared memory.  One CTA per SM (it
+ *   takes precedence over MOE_OPT_TC_PAIR).  Same results.
  *   MOE_OPT_WAIT_LIMIT_US: limit, in microseconds, of every bounded wait inside
  *   the tensor-core GEMM (a pipeline stage normally lands in a few
  *   microseconds).  A wait that runs out raises MOE_FLAG_TIMEOUT in the call's
@@ -277,6 +282,7 @@ int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStre
 #define MOE_OPT_TC_PAIR 2
 #define MOE_OPT_WAIT_LIMIT_US 3
 #define MOE_OPT_TEST_TIMEOUT 4
+#define MOE_OPT_TC_A_TMEM 5
 int moe_set_option(int option, int value);
 int moe_get_option(int option);
 

@@ -1,12 +1,16 @@
-"""The tensor-core grouped GEMM in SM pairs (MOE_OPT_TC_PAIR = 1: clusters of
-two CTAs, tcgen05 cta_group::2, M = 256) against the one-CTA-per-SM path and
-the oracle.
+"""The tensor-core grouped GEMM's alternative forms against the plain
+one-CTA-per-SM form (both operands from shared memory) and the oracle:
 
-Both paths form the same exact sums, so y, hq and sh must be bit-identical
+* SM pairs (MOE_OPT_TC_PAIR = 1: clusters of two CTAs, tcgen05 cta_group::2,
+  M = 256), where the weight rows of a matrix are a multiple of 256 (W1
+  always, W2 when H is); other shapes fall back to one CTA per SM, which a
+  case here covers too;
+* the weight operand staged in tensor memory (MOE_OPT_TC_A_TMEM = 1: one
+  tcgen05.cp per stage, the digit-plane MMAs read A from TMEM).
+
+All forms compute the same exact sums, so y, hq and sh must be bit-identical
 between them; against the oracle the layer's usual bar applies (bit-exact
-INT8 codes and scales, y within tolerance).  The pair form applies where the
-weight rows of a matrix are a multiple of 256 (W1 always, W2 when H is); other
-shapes fall back to one CTA per SM, which a case here covers too.
+INT8 codes and scales, y within tolerance).
 """
 import numpy as np
 import pytest
@@ -33,11 +37,13 @@ def cu(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def _run(moe, d, w, pair):
+def _run(moe, d, w, pair, a_tmem=False):
     T, H, I, E, k = w.T, w.H, w.I, w.E, w.k
-    old = (moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS), moe.moe_get_option(moe.MOE_OPT_TC_PAIR))
+    old = (moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS), moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
+           moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM))
     moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
     moe.moe_set_option(moe.MOE_OPT_TC_PAIR, 1 if pair else 0)
+    moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, 1 if a_tmem else 0)
     try:
         packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]),
                                       cu(d["w2_scales"]))
@@ -56,6 +62,7 @@ def _run(moe, d, w, pair):
     finally:
         moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, old[0])
         moe.moe_set_option(moe.MOE_OPT_TC_PAIR, old[1])
+        moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, old[2])
 
 
 @pytest.mark.parametrize("T,H,E,k,I,seed", [
@@ -65,11 +72,12 @@ def _run(moe, d, w, pair):
     (13, 384, 9, 3, 256, 74),      # H = 384: W2 falls back to one CTA per SM, W1 in pairs
     (257, 256, 1, 1, 128, 75),     # E = 1, three token tiles, the last holds one row
 ])
-def test_pair_matches_single_and_oracle(moe, T, H, E, k, I, seed):
+@pytest.mark.parametrize("form", ["pair", "a_tmem"])
+def test_form_matches_single_and_oracle(moe, form, T, H, E, k, I, seed):
     w = synth.custom("pair", T, H, E, k, I, seed)
     d = synth.make(w)
     y1, d1 = _run(moe, d, w, pair=False)
-    y2, d2 = _run(moe, d, w, pair=True)
+    y2, d2 = _run(moe, d, w, pair=form == "pair", a_tmem=form == "a_tmem")
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(d1["hq"], d2["hq"])
     assert torch.equal(d1["sh"].view(torch.int32), d2["sh"].view(torch.int32))
@@ -84,7 +92,8 @@ def test_pair_matches_single_and_oracle(moe, T, H, E, k, I, seed):
     assert np.linalg.norm(yg - yo) / max(np.linalg.norm(yo), 1e-300) <= Y_FRO_REL
 
 
-def test_pair_option_validation(moe):
-    with pytest.raises(moe.MoeError):
-        moe.moe_set_option(moe.MOE_OPT_TC_PAIR, 2)
-    assert moe.moe_get_option(moe.MOE_OPT_TC_PAIR) in (0, 1)
+def test_form_option_validation(moe):
+    for opt in (moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM):
+        with pytest.raises(moe.MoeError):
+            moe.moe_set_option(opt, 2)
+        assert moe.moe_get_option(opt) in (0, 1)
