@@ -250,6 +250,25 @@ def run_gpu_workload(name: str, steps: int, warmup: int, dist: Dist, want_e2e: b
                alg_bytes_step=alg_bytes_step, alg_flop_step=alg_flop_step, gemm_ms=gemm_ms,
                w1_ms=w1_ms, w2_ms=w2_ms)
 
+    # the router projection in front of the path (not part of the metric's
+    # A1-A7 step): its own time per step, same tokens
+    wr = torch.from_numpy(synth.router_weight(w.seed, E, H)).cuda()
+    rb = synth.router_bias(E, w.bias_coef)
+    rb = None if rb is None else torch.from_numpy(rb.astype(np.float32)).cuda()
+    lg = torch.empty((T, E), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        moe.moe_router_logits(x, wr, rb, out=lg, stream=stream)
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    rsteps = max(3, min(steps, 200))
+    r0.record(stream)
+    for _ in range(rsteps):
+        moe.moe_router_logits(x, wr, rb, out=lg, stream=stream)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    res["router_ms"] = r0.elapsed_time(r1) / rsteps
+    res["router_flop"] = 2.0 * T * H * E
+    del wr, lg
+
     if want_e2e:
         xh = torch.from_numpy(d["x"]).view(torch.bfloat16).pin_memory()
         lh = torch.from_numpy(d["logits"]).pin_memory()
@@ -309,6 +328,14 @@ def cpu_baseline(name: str, seconds: float) -> dict:
     dt = time.time() - t0
     return {"value": toks / dt, "unit": "tokens/s", "cores": oracle.nthreads(), "kind": "oracle",
             "sample": sample, "seconds": round(dt, 2)}
+
+
+def router_line(r: dict) -> dict:
+    """The router projection (logits = x W_r^T, moe_router_logits) timed on its own:
+    the step in front of the layer, outside the A1-A7 metric."""
+    return {"ms_per_step": round(r["router_ms"], 5),
+            "tflops": round(r["router_flop"] / (r["router_ms"] * 1e-3) / 1e12, 3),
+            "kernel": "k_router_logits (fp32 CUDA-core contraction)", "in_metric": False}
 
 
 def roofline_hbm(r: dict, peaks: dict, traffic):
@@ -383,6 +410,7 @@ def main():
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "kernel_ms_per_step": {"w1": round(r["w1_ms"] / steps, 5), "w2": round(r["w2_ms"] / steps, 5)},
+        "router_projection": router_line(r),
     }
     if not a.no_decode_t64:
         # the larger decode batch (most experts get 1-3 rows): same HBM roofline
@@ -429,6 +457,7 @@ def main():
                              "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
                 "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
+                "router_projection": router_line(rp),
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
             }

@@ -24,7 +24,8 @@ FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_LAYOUT, FLAG_TIMEOUT, FLAG_BOUNDS = 1, 2, 
 # Exported symbols of include/moe.h, in declaration order.
 SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack_weights",
            "moe_router_logits", "moe_route", "moe_sort_workspace_bytes", "moe_sort", "moe_sort_static", "moe_workspace_bytes",
-           "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_tables",
+           "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_router_workspace_bytes",
+           "moe_layer_forward_with_router", "moe_layer_tables",
            "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
            "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
 
@@ -65,6 +66,8 @@ def _load():
         "moe_forward": ([D, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
         "moe_layer_workspace_bytes": ([D, i32], sz),
         "moe_layer_forward": ([D, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
+        "moe_layer_router_workspace_bytes": ([D, i32], sz),
+        "moe_layer_forward_with_router": ([D, vp, vp, vp, vp, vp, vp, sz, ctypes.POINTER(moe_debug), vp], i32),
         "moe_layer_tables": ([D, vp] + [ctypes.POINTER(vp)] * 5, i32),
         "moe_quant_rows_f32": ([vp, i32, i32, vp, vp, vp], i32),
         "moe_exp_f32": ([vp, vp, ctypes.c_int64, vp], i32),
@@ -270,6 +273,31 @@ def moe_layer_forward(logits, x, packed, H: int, I: int, E: int, k: int, ws=None
     _check(lib.moe_layer_forward(ctypes.byref(d), _ptr(logits), _ptr(x), _ptr(packed), _ptr(y),
                                  _ptr(ws), ws.numel(), ctypes.byref(dbg) if dbg is not None else None,
                                  _stream(stream)))
+    return y
+
+
+def moe_layer_router_workspace_bytes(T_max: int, H: int, I: int, E: int, k: int) -> int:
+    d = _dims(T_max, H, I, E, k)
+    n = lib.moe_layer_router_workspace_bytes(ctypes.byref(d), T_max)
+    if n == 0:
+        raise MoeError(-2, "unsupported dims")
+    return n
+
+
+def moe_layer_forward_with_router(x, w_router, bias, packed, H: int, I: int, E: int, k: int, ws=None, y=None,
+                                  dbg: moe_debug | None = None, stream=None):
+    """Router projection then the whole layer: x [T,H] bf16, w_router [E,H] fp32,
+    bias [E] fp32 or None -> y [T,H] bf16."""
+    T = x.shape[0]
+    dev = x.device
+    if ws is None:
+        ws = _empty_aligned(moe_layer_router_workspace_bytes(T, H, I, E, k), dev)
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    d = _dims(T, H, I, E, k)
+    _check(lib.moe_layer_forward_with_router(ctypes.byref(d), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(packed),
+                                             _ptr(y), _ptr(ws), ws.numel(),
+                                             ctypes.byref(dbg) if dbg is not None else None, _stream(stream)))
     return y
 
 

@@ -438,6 +438,36 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
                         L.total - L.fwd, (int32_t*)(w + L.flag), dbg, stream);
 }
 
+// moe_layer_forward preceded by the router projection: the logits go to a
+// region after the layer workspace.
+static size_t router_ws_offset(const moe_dims& d, long long T, int tc_min) {
+    return moe::align_up(layer_ws(d, T, tc_min).total, 256);
+}
+
+size_t moe_layer_router_workspace_bytes(const moe_dims* d, int T_max) {
+    if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
+    return router_ws_offset(*d, T_max, g_tc_min_rows.load()) + moe::align_up(4 * (size_t)T_max * d->E, 256);
+}
+
+int moe_layer_forward_with_router(const moe_dims* d, const void* x_bf16, const float* w_router,
+                                  const float* bias, const void* packed, void* y_bf16, void* ws,
+                                  size_t ws_bytes, const moe_debug* dbg, cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_dims(d, true)) return rc;
+    if (!ws || !packed || (d->T > 0 && (!x_bf16 || !w_router || !y_bf16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: NULL pointer");
+    if (!aligned(ws, 256))
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: ws must be 256-byte aligned");
+    const int tc_min = g_tc_min_rows.load();
+    const size_t lo = router_ws_offset(*d, d->T, tc_min);
+    const size_t need = lo + moe::align_up(4 * (size_t)d->T * d->E, 256);
+    if (ws_bytes < need)
+        return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: ws_bytes %zu < %zu", ws_bytes, need);
+    float* logits = (float*)((char*)ws + lo);
+    if (int rc = moe_router_logits(x_bf16, w_router, bias, d->T, d->H, d->E, logits, stream)) return rc;
+    return moe_layer_forward(d, logits, x_bf16, packed, y_bf16, ws, lo, dbg, stream);
+}
+
 int moe_layer_tables(const moe_dims* d, void* ws, int32_t** topk_idx, float** gates, int32_t** perm,
                      int32_t** pos, int32_t** offsets) {
     g_last_error.clear();

@@ -227,6 +227,19 @@ int moe_layer_forward(const moe_dims *d, const float *logits, const void *x_bf16
                       const void *packed, void *y_bf16, void *ws, size_t ws_bytes,
                       const moe_debug *dbg, cudaStream_t stream);
 
+/* The router projection followed by the whole layer: logits = x W_router^T
+ * (+ bias), as moe_router_logits computes them, then moe_layer_forward on
+ * those logits -- from x [T, H] bf16, w_router [E, H] fp32 and bias [E] fp32
+ * (or NULL) to y [T, H] bf16.  ws: moe_layer_router_workspace_bytes(d, T_max)
+ * bytes, 256-byte aligned, T <= T_max: the layer workspace (error word first;
+ * moe_layer_tables works on it) followed by the logits.  The results equal
+ * those of moe_router_logits followed by moe_layer_forward.  Asynchronous,
+ * graph-capturable; errors as for those two calls. */
+size_t moe_layer_router_workspace_bytes(const moe_dims *d, int T_max);
+int moe_layer_forward_with_router(const moe_dims *d, const void *x_bf16, const float *w_router,
+                                  const float *bias, const void *packed, void *y_bf16, void *ws,
+                                  size_t ws_bytes, const moe_debug *dbg, cudaStream_t stream);
+
 /* Device pointers to the routing tables moe_layer_forward leaves in its
  * workspace `ws` for dims d (d->T = the call's T): topk_idx [T, k] and gates
  * [T, k] as moe_route writes them, perm [T*k], pos [T*k] and offsets [E + 1]

@@ -79,3 +79,22 @@ def test_router_zero_tokens_and_bad_args(moe):
     with pytest.raises(moe.MoeError):
         moe.moe_router_logits(torch.empty((2, 100), dtype=torch.bfloat16, device="cuda"),
                               torch.zeros((4, 100), dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("T,H,E,k,I,seed", [(8, 4096, 256, 6, 2048, 1), (300, 512, 8, 2, 256, 81)])
+def test_layer_with_router_equals_the_two_calls(moe, T, H, E, k, I, seed):
+    # moe_layer_forward_with_router = moe_router_logits then moe_layer_forward,
+    # bit for bit (decode-size fused front, and a call with tensor-core experts)
+    w = synth.custom("lr", T, H, E, k, I, seed, 0.8 if T > 8 else 0.0)
+    d = synth.make(w)
+    wr = cu(synth.router_weight(seed, E, H))
+    bias = cu(synth.router_bias(E, w.bias_coef).astype(np.float32)) if w.bias_coef else None
+    packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]), cu(d["w2_scales"]))
+    x = cu(d["x"]).view(torch.bfloat16)
+    y1 = moe.moe_layer_forward_with_router(x, wr, bias, packed, H, I, E, k)
+    logits = moe.moe_router_logits(x, wr, bias)
+    ws = torch.empty(moe.moe_layer_workspace_bytes(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+    y2 = moe.moe_layer_forward(logits, x, packed, H, I, E, k, ws=ws)
+    torch.cuda.synchronize()
+    assert moe.moe_check_device_flag(ws) == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
