@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tc-pair", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_PAIR for the run (default: the library's default)")
+    ap.add_argument("--tc-min", type=int, default=None,
+                    help="MOE_OPT_TC_MIN_ROWS for the run (1: every expert on the tensor cores)")
     ap.add_argument("--tc-a-tmem", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_A_TMEM for the run (default: the library's default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -141,7 +143,7 @@ class Clocks:
         self.f.flush()
         rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, pw = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             r = [c.strip() for c in r]
@@ -150,13 +152,15 @@ class Clocks:
             try:
                 sm.append(float(r[1]))
                 mx = float(r[2])
+                pw.append(float(r[3]))
             except ValueError:
                 continue
             for n, v in zip(names, r[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w": statistics.median(pw) if pw else None}
 
 
 def measured_peaks() -> dict:
@@ -387,6 +391,8 @@ def main():
         moe.moe_set_option(moe.MOE_OPT_TC_PAIR, a.tc_pair)
     if a.tc_a_tmem is not None:
         moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, a.tc_a_tmem)
+    if a.tc_min is not None:
+        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, a.tc_min)
     rank0 = dist.rank == 0
     peaks = measured_peaks()
     r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
@@ -429,13 +435,16 @@ def main():
         # labelled milder variant (c = 1.25: empty experts, thousands of rows on
         # the top experts, many small experts on the streaming GEMM)
         fp8_peak = 2.0 * peaks["bf16_tflops"]
-        for key, pname, cap in (("prefill", a.prefill_workload, 20), ("prefill_skew", "prefill_skew_T16384", 5),
-                                ("prefill_skew1.25", "prefill_skew1.25_T16384", 5)):
+        # ~0.2 s of timed steps per line, so that the clocks sampled under load
+        # say whether the tensor-core GEMM ran at the burst or the power-capped
+        # sustained clock
+        for key, pname, cap in (("prefill", a.prefill_workload, 150), ("prefill_skew", "prefill_skew_T16384", 50),
+                                ("prefill_skew1.25", "prefill_skew1.25_T16384", 40)):
             if key.startswith("prefill_skew") and a.no_skew:
                 continue
             pw = synth.WORKLOADS[pname]
-            psteps = max(3, min(cap, steps // 100))
-            rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=False)
+            psteps = max(3, min(cap, steps // 10))
+            rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=rank0)
             ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
             out[key] = {
                 "workload": pw.name, "T": pw.T, "steps": psteps,
@@ -451,6 +460,10 @@ def main():
                              "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
                              # the INT8 operand enters the FP4 MMA as three exact digit planes,
                              # so the tensor pipe issues 3x the algorithmic work at the FP4 rate
+                             "frac_vs_sustained": round(ptf / (2.0 * peaks["bf16_tflops_sustained"]), 5)
+                             if peaks.get("bf16_tflops_sustained") else None,
+                             "peak_sustained": 2.0 * peaks["bf16_tflops_sustained"]
+                             if peaks.get("bf16_tflops_sustained") else None,
                              "mma_issued_tflops": round(3 * ptf, 2),
                              "mma_peak_fp4": 4.0 * peaks["bf16_tflops"],
                              "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
@@ -458,6 +471,7 @@ def main():
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
                 "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
                 "router_projection": router_line(rp),
+                "clocks": rp["clocks"],
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
             }

@@ -302,6 +302,12 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     const bool use_tc = !logits && T >= opt.tc_min_rows;
     // the timeout test applies to the first tensor-core launch after it is armed
     const int withhold = use_tc ? g_test_timeout.exchange(0) : 0;
+    // token tile of the tensor-core GEMM: the decode configuration when no
+    // expert can have more than kTcDecodeMaxT rows
+    const int tc_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
+    // with a threshold of 1 every expert with rows takes the tensor cores, so
+    // the streaming GEMM has nothing to do and is not launched
+    const bool use_gemv = !use_tc || opt.tc_min_rows > 1;
     // token rows per streaming-GEMM unit: 2 for small calls (nearly every expert
     // has one or two rows; the smaller ring slot fits more warps per SM), else 4
     const int group = T <= moe::kGemvSmallGroupMaxT ? moe::kGemvSmallGroup : moe::kGemvGroup;
@@ -327,7 +333,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
-        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? opt.tc_min_rows : 0x7fffffff,
+        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? opt.tc_min_rows : 0x7fffffff, tc_tile,
                                       group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
                                       stream),
                 "plan + row state");
@@ -336,11 +342,12 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         MOE_TRY(moe::launch_planes(xtp, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
-    MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                             uoff1, soff, E, gacc, flag, I, P, group, stream), "W1");
+    if (use_gemv)
+        MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
+                                 uoff1, soff, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns,
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns,
                                     withhold, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
@@ -348,11 +355,12 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                                hinit, dbg ? dbg->hq : nullptr, dbg ? dbg->sh : nullptr, flag, stream),
             "SwiGLU + h quant + h planes");
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
-    MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                             uoff2, soff, E, yacc, flag, 0, P, group, stream), "W2");
+    if (use_gemv)
+        MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
+                                 uoff2, soff, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns, 0,
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns, 0,
                                     stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
         __syncthreads();
         // no expert reaches the tensor-core threshold: plan with an unreachable one
         if (threadIdx.x < 32)
-            plan_warp(offs, a.E, P, 2 * a.I, a.H, 0x7fffffff, a.group, a.unit_off1, a.unit_off2, a.tile_off1,
+            plan_warp(offs, a.E, P, 2 * a.I, a.H, 0x7fffffff, kTcTokenTile, a.group, a.unit_off1, a.unit_off2, a.tile_off1,
                       a.tile_off2, a.plane_off, a.stream_off, a.expert_tc, a.flag, true, ps);
         // every row is a streaming row and every expert's streaming rows start
         // at its sorted offset, so sorted row i is streaming row i

@@ -71,12 +71,16 @@ constexpr int kGemvSmallGroupMaxT = 16;
 constexpr int kMaxExperts = 1024;   // the API's limit on E
 constexpr int kTcWeightTile = 128;
 constexpr int kTcTokenTile = 128;
+// Token tile of the tensor-core GEMM's decode configuration (calls with at
+// most kTcDecodeMaxT tokens, so at most that many rows per expert).
+constexpr int kTcDecodeTokenTile = 32;
+constexpr int kTcDecodeMaxT = 64;
 
 // Number of kernels this library has launched in the process (diagnostics).
 void count_launches(int n);
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
-                             int I, int H, int tc_min, int group, int32_t* unit_off1, int32_t* unit_off2,
+                             int I, int H, int tc_min, int tc_tile, int group, int32_t* unit_off1, int32_t* unit_off2,
                              int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off,
                              int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc, int32_t* flag,
                              cudaStream_t st);
@@ -170,8 +174,8 @@ cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, in
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
-                           const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st);
+                           const float* row_scale, const int32_t* perm, int k_div, float* out, int token_tile,
+                           bool pair, bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st);
 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,

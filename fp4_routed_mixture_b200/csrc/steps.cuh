@@ -308,8 +308,8 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 
 // ---- plan ----------------------------------------------------------------------------
 // Work split per expert: experts with at least tc_min rows go to the
-// tensor-core GEMM (tiles of kTcWeightTile weight rows x kTcTokenTile token
-// rows), the others to the streaming GEMM (units of kGemvTileRows weight rows
+// tensor-core GEMM (tiles of kTcWeightTile weight rows x tc_tile token rows,
+// the token tile of the configuration that GEMM is launched with), the others to the streaming GEMM (units of kGemvTileRows weight rows
 // x `group` tokens, the group size the streaming GEMM is launched with).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
@@ -334,7 +334,7 @@ struct PlanShared {
 constexpr int32_t kNoRow = INT32_MIN;
 
 static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
-                                 int group,
+                                 int tc_tile, int group,
                                  int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                                  int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                                  int32_t* __restrict__ plane_off, int32_t* __restrict__ stream_off,
@@ -353,7 +353,7 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
         const int m = any_bad ? 0 : offsets[e + 1] - offsets[e];
         const bool tc = m >= tc_min;
         const int g = tc ? 0 : (m + group - 1) / group;
-        const int nb = tc ? (m + kTcTokenTile - 1) / kTcTokenTile : 0;
+        const int nb = tc ? (m + tc_tile - 1) / tc_tile : 0;
         c[0] = g * (n1 / kGemvTileRows);
         c[1] = g * (n2 / kGemvTileRows);
         c[2] = nb * (n1 / kTcWeightTile);

@@ -55,50 +55,65 @@
 namespace moe {
 
 constexpr int TC_BM = kTcWeightTile;           // weight rows per tile (MMA M)
-constexpr int TC_BN = kTcTokenTile;            // token rows per tile (largest MMA N used)
 constexpr int TC_PIPES = 2;                    // producer + MMA-issuer pairs, alternating tiles
-constexpr int TC_STAGES = 3;                   // ring stages per pipe
 constexpr int TC_ACC = 3;                      // accumulator buffers shared by the pipes
 constexpr int TC_A_BYTES = 8704;               // one packed chunk: 128 rows x 128 inputs
-constexpr int TC_B_BYTES = TC_BN / 8 * kPlaneGroupBytes;  // 3 planes x TC_BN rows x 128 inputs
-constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
-constexpr int TC_CHUNKS = TC_BN / 32;          // 32-column chunks of a tile
-constexpr int TC_EPI_WARPS = 4 * TC_CHUNKS;    // one per (TMEM lane quadrant, column chunk)
 constexpr int TC_EPI_WARP0 = 2 * TC_PIPES;     // warps 0..: producers, then MMA issuers
-constexpr int TC_THREADS = 32 * (TC_EPI_WARP0 + TC_EPI_WARPS);
-constexpr int TC_TMEM_COLS = 512;
-// TMEM columns: accumulator b at b * TC_BN; then per pipe r, at TC_SF_COL + 24r,
-// the A scale factors (4 columns per stage) and the three constant B plane
-// scales (4 columns each).
-constexpr int TC_SF_COL = TC_ACC * TC_BN;
-constexpr int TC_SF_PIPE_COLS = 4 * TC_STAGES + 12;
-static_assert(TC_SF_COL + TC_PIPES * TC_SF_PIPE_COLS <= TC_TMEM_COLS, "accumulators and scale factors exceed TMEM");
-static_assert(TC_SF_COL % 4 == 0 && TC_SF_PIPE_COLS % 4 == 0, "scale-factor columns hold 4 bytes per lane");
-static_assert(TC_BN % 32 == 0 && TC_BN <= 256, "MMA N, whole column chunks");
-// The A-in-TMEM form (ATMEM): every stage's weight chunk is copied into TMEM
-// once (tcgen05.cp, two 128 x 256-bit halves, 16 columns) and the six plane
-// MMAs read A from there, so shared memory feeds only B.  Columns: the
-// accumulators, then per pipe r and stage s the A slot at TC_AT_A + 48r + 16s,
-// the A scale factors at TC_AT_SFA + 12r + 4s, and two constant B scale
-// regions shared by the pipes: X (bytes 2^6, 2^6, 2^3, 2^3 in every 4-byte
-// group) serves planes 0 and 1 through the scale-factor byte selector (0 and
-// 2), Y (all 2^0) plane 2.
-constexpr int TC_AT_A = TC_ACC * TC_BN;
-constexpr int TC_AT_SFA = TC_AT_A + TC_PIPES * TC_STAGES * 16;
-constexpr int TC_AT_SFB = TC_AT_SFA + TC_PIPES * TC_STAGES * 4;
-static_assert(TC_AT_SFB + 8 <= TC_TMEM_COLS, "A slots and scale factors exceed TMEM");
-static_assert(TC_AT_A % 16 == 0, "A slots on 16-column boundaries");
 
-struct TcShared {
-    uint8_t stage[TC_PIPES][TC_STAGES][TC_STAGE_BYTES];
-    uint8_t sfb[3][512];        // constant plane scales, copied to TMEM once per pipe
-    float col_scale[TC_EPI_WARPS][32];  // per epilogue warp: activation scale of its 32 columns
-    uint64_t full[TC_PIPES][TC_STAGES], empty[TC_PIPES][TC_STAGES], acc_full[TC_ACC], acc_empty[TC_ACC];
-    uint64_t drain[TC_PIPES];   // each issuer's last commit: all of its MMAs are done
-    uint64_t sfb_ready;         // ATMEM: the shared B scale regions are in TMEM
-    uint32_t tmem_base;
-    int32_t abort;
+constexpr int pow2_at_least(int v, int p = 32) { return p >= v ? p : pow2_at_least(v, 2 * p); }
+
+// A kernel configuration: BN token rows per tile (the largest MMA N used) and
+// STAGES ring stages per pipe.  The prefill form takes 128-row token tiles
+// with three 33 KB stages per pipe; the decode form (at most a few rows per
+// expert) takes 32-row tiles with six 14.5 KB stages per pipe, which keeps
+// twice the weight bytes in flight per SM -- at decode sizes the weights
+// stream from DRAM and every byte is used by one tile.
+template <int BN_, int STAGES_>
+struct TcCfg {
+    static constexpr int BN = BN_, STAGES = STAGES_;
+    static constexpr int B_BYTES = BN / 8 * kPlaneGroupBytes;  // 3 planes x BN rows x 128 inputs
+    static constexpr int STAGE_BYTES = TC_A_BYTES + B_BYTES;
+    static constexpr int CHUNKS = BN / 32;                      // 32-column chunks of a tile
+    static constexpr int EPI_WARPS = 4 * CHUNKS;                // one per (TMEM lane quadrant, column chunk)
+    static constexpr int THREADS = 32 * (TC_EPI_WARP0 + EPI_WARPS);
+    // TMEM columns: accumulator b at b * BN; then per pipe r, at SF_COL +
+    // SF_PIPE_COLS * r, the A scale factors (4 columns per stage) and the three
+    // constant B plane scales (4 columns each).
+    static constexpr int SF_COL = TC_ACC * BN;
+    static constexpr int SF_PIPE_COLS = 4 * STAGES + 12;
+    // The A-in-TMEM form (ATMEM): every stage's weight chunk is copied into
+    // TMEM once (tcgen05.cp, two 128 x 256-bit halves, 16 columns) and the six
+    // plane MMAs read A from there, so shared memory feeds only B.  Columns:
+    // the accumulators, then per pipe r and stage s the A slot at AT_A +
+    // 16 (STAGES r + s), the A scale factors at AT_SFA + 4 (STAGES r + s), and
+    // two constant B scale regions shared by the pipes: X (bytes 2^6, 2^6, 2^3,
+    // 2^3 in every 4-byte group) serves planes 0 and 1 through the
+    // scale-factor byte selector (0 and 2), Y (all 2^0) plane 2.
+    static constexpr int AT_A = TC_ACC * BN;
+    static constexpr int AT_SFA = AT_A + TC_PIPES * STAGES * 16;
+    static constexpr int AT_SFB = AT_SFA + TC_PIPES * STAGES * 4;
+    static constexpr int TMEM_COLS = pow2_at_least(
+        (SF_COL + TC_PIPES * SF_PIPE_COLS) > (AT_SFB + 8) ? (SF_COL + TC_PIPES * SF_PIPE_COLS) : (AT_SFB + 8));
+    static_assert(TMEM_COLS <= 512, "accumulators, A slots and scale factors exceed TMEM");
+    static_assert(SF_COL % 4 == 0 && SF_PIPE_COLS % 4 == 0, "scale-factor columns hold 4 bytes per lane");
+    static_assert(AT_A % 16 == 0, "A slots on 16-column boundaries");
+    static_assert(BN % 32 == 0 && BN <= 256, "MMA N, whole column chunks");
+
+    struct Shared {
+        uint8_t stage[TC_PIPES][STAGES][STAGE_BYTES];
+        uint8_t sfb[3][512];        // constant plane scales, copied to TMEM by the MMA issuers
+        float col_scale[EPI_WARPS][32];  // per epilogue warp: activation scale of its 32 columns
+        uint64_t full[TC_PIPES][STAGES], empty[TC_PIPES][STAGES], acc_full[TC_ACC], acc_empty[TC_ACC];
+        uint64_t drain[TC_PIPES];   // each issuer's last commit: all of its MMAs are done
+        uint64_t sfb_ready;         // ATMEM: the shared B scale regions are in TMEM
+        uint32_t tmem_base;
+        int32_t abort;
+    };
 };
+using TcPrefill = TcCfg<kTcTokenTile, 3>;
+using TcDecode = TcCfg<kTcDecodeTokenTile, 6>;
+static_assert(sizeof(TcPrefill::Shared) <= 227 * 1024 && sizeof(TcDecode::Shared) <= 227 * 1024,
+              "shared memory per CTA");
 
 struct TcArgs {
     const uint8_t* w;          // matrix region of the packed buffer
@@ -319,6 +334,7 @@ struct TcTile {
     int e, rb, i0, pr0, n_valid, n_mma;   // i0: first sorted row, pr0: its plane row
 };
 
+template <int TC_BN>
 __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
     int lo = 0, hi = a.E;  // last e with tile_off[e] <= t
     while (hi - lo > 1) {
@@ -349,9 +365,14 @@ __device__ __forceinline__ TcTile tile_at(const TcArgs& a, int t) {
 // barrier; a remote arrive joins the even CTA's), the even CTA's MMA commits
 // arrive on the barriers of both CTAs, and the odd CTA's epilogue warps release
 // accumulators with remote arrives.
-template <bool PAIR, bool ATMEM>
-__global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
+template <class Cfg, bool PAIR, bool ATMEM>
+__global__ void __launch_bounds__(Cfg::THREADS, 1) k_tc_gemm(TcArgs a) {
     static_assert(!(PAIR && ATMEM), "the A-in-TMEM form is one CTA per SM");
+    constexpr int TC_BN = Cfg::BN, TC_STAGES = Cfg::STAGES, TC_EPI_WARPS = Cfg::EPI_WARPS;
+    constexpr int TC_THREADS = Cfg::THREADS, TC_TMEM_COLS = Cfg::TMEM_COLS;
+    constexpr int TC_SF_COL = Cfg::SF_COL, TC_SF_PIPE_COLS = Cfg::SF_PIPE_COLS;
+    constexpr int TC_AT_A = Cfg::AT_A, TC_AT_SFA = Cfg::AT_SFA, TC_AT_SFB = Cfg::AT_SFB;
+    using TcShared = typename Cfg::Shared;
     pdl_begin();
     extern __shared__ __align__(1024) uint8_t tc_smem_raw[];
     TcShared& sh = *reinterpret_cast<TcShared*>(tc_smem_raw);
@@ -442,7 +463,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         bool filled[TC_STAGES] = {};
         uint32_t fill_parity[TC_STAGES] = {};
         for (int j = r; j < ntiles && !*abort; j += TC_PIPES) {
-            const TcTile tt = tile_at(a, tile_of(j));
+            const TcTile tt = tile_at<TC_BN>(a, tile_of(j));
             const uint8_t* wsrc = a.w + (size_t)tt.e * a.expert_bytes + (size_t)tt.rb * KG * TC_A_BYTES;
             // token rows this CTA supplies: all of them, or its half of the pair's
             const int nb_rows = PAIR ? tt.n_mma / 2 : tt.n_mma;
@@ -549,7 +570,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         uint32_t phase = 0;
         int issued = 0;
         for (int j = r; j < ntiles && sfb_ok && !*abort; j += TC_PIPES) {
-            const TcTile tt = tile_at(a, tile_of(j));
+            const TcTile tt = tile_at<TC_BN>(a, tile_of(j));
             const int buf = j % TC_ACC;
             const uint32_t use = (uint32_t)(j / TC_ACC);
             if (!wait(smem_u32(&sh.acc_empty[buf]), (use & 1u) ^ 1u)) {
@@ -673,7 +694,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_tc_gemm(TcArgs a) {
         const bool w1 = a.gate_up_half > 0;
         float* csc = sh.col_scale[ew];
         for (int j = 0; j < ntiles && !*abort; ++j) {
-            const TcTile tt = tile_at(a, tile_of(j));
+            const TcTile tt = tile_at<TC_BN>(a, tile_of(j));
             const int buf = j % TC_ACC;
             const uint32_t use = (uint32_t)(j / TC_ACC);
             const bool mine = n0 < tt.n_mma;
@@ -771,17 +792,23 @@ __global__ void __launch_bounds__(256)
         for (int p = 0; p < 3; ++p) *reinterpret_cast<uint4*>(dst + p * 512 + cc * 128) = v[3 * cc + p];
 }
 
-// One CTA per SM: it allocates all of the SM's TMEM.
+// One CTA per SM (it allocates the SM's TMEM) for every form of the kernel:
+// sets the dynamic shared-memory limit of each one-CTA instantiation.
+template <class Cfg>
+static cudaError_t set_smem(void (*k)(TcArgs)) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(typename Cfg::Shared));
+}
+
 static int tc_grid() {
     static PerContext cache;
     return cache.get([] {
         int dev = 0, sms = 0;
         if (cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaFuncSetAttribute(k_tc_gemm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(TcShared)) != cudaSuccess ||
-            cudaFuncSetAttribute(k_tc_gemm<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(TcShared)) != cudaSuccess)
+            set_smem<TcPrefill>(k_tc_gemm<TcPrefill, false, false>) != cudaSuccess ||
+            set_smem<TcPrefill>(k_tc_gemm<TcPrefill, false, true>) != cudaSuccess ||
+            set_smem<TcDecode>(k_tc_gemm<TcDecode, false, false>) != cudaSuccess ||
+            set_smem<TcDecode>(k_tc_gemm<TcDecode, false, true>) != cudaSuccess)
             return -1;
         return sms;
     });
@@ -789,21 +816,20 @@ static int tc_grid() {
 
 // Clusters of two CTAs that can be resident at once (0: the pair form is not
 // available); the grid is two CTAs per such cluster, so no cluster waits for
-// another to finish.
+// another to finish.  (The pair form is built for the prefill configuration.)
 static int tc_pair_grid() {
     static PerContext cache;
     return cache.get([] {
         const int single = tc_grid();
         if (single <= 0) return -1;
-        if (cudaFuncSetAttribute(k_tc_gemm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(TcShared)) != cudaSuccess) {
+        if (set_smem<TcPrefill>(k_tc_gemm<TcPrefill, true, false>) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * single);
-        cfg.blockDim = dim3(TC_THREADS);
-        cfg.dynamicSmemBytes = sizeof(TcShared);
+        cfg.blockDim = dim3(TcPrefill::THREADS);
+        cfg.dynamicSmemBytes = sizeof(TcPrefill::Shared);
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -812,7 +838,8 @@ static int tc_pair_grid() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<true, false>, &cfg) != cudaSuccess || clusters <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&clusters, k_tc_gemm<TcPrefill, true, false>, &cfg) != cudaSuccess ||
+            clusters <= 0) {
             cudaGetLastError();
             return 0;
         }
@@ -820,7 +847,7 @@ static int tc_pair_grid() {
     });
 }
 
-size_t tc_smem_bytes() { return sizeof(TcShared); }
+size_t tc_smem_bytes() { return sizeof(TcPrefill::Shared); }
 
 cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, int k_div, int rows,
                           const int32_t* plane_row, int plane_rows, uint8_t* planes, int32_t* flag,
@@ -836,21 +863,23 @@ cudaError_t launch_planes(const uint8_t* tplanes, int K, const int32_t* perm, in
 cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
                            const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
                            const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
-                           const float* row_scale, const int32_t* perm, int k_div, float* out, bool pair,
-                           bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st) {
+                           const float* row_scale, const int32_t* perm, int k_div, float* out, int token_tile,
+                           bool pair, bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st) {
     TcArgs a{w, expert_bytes, K, N, gate_up_half, planes, plane_rows, plane_off, P, offsets, tile_off,
              E, flag, row_scale, perm, k_div, out, wait_ns, withhold};
+    const bool decode = token_tile == TcDecode::BN;
+    if (!decode && token_tile != TcPrefill::BN) return cudaErrorInvalidValue;
     // the timeout test runs on the one-CTA form (withhold applies to it only);
-    // the A-in-TMEM form is one CTA per SM
-    if (withhold || a_tmem) pair = false;
+    // the A-in-TMEM and decode forms are one CTA per SM
+    if (withhold || a_tmem || decode) pair = false;
     cudaError_t e;
     // the pair takes two adjacent 128-row tiles of one expert: N % 256 == 0
     const int pgrid = (pair && N % (2 * TC_BM) == 0) ? tc_pair_grid() : 0;
     if (pgrid > 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(pgrid);
-        cfg.blockDim = dim3(TC_THREADS);
-        cfg.dynamicSmemBytes = sizeof(TcShared);
+        cfg.blockDim = dim3(TcPrefill::THREADS);
+        cfg.dynamicSmemBytes = sizeof(TcPrefill::Shared);
         cfg.stream = st;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -861,12 +890,20 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 2;
-        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<true, false>, a);
+        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<TcPrefill, true, false>, a);
     } else {
         const int grid = tc_grid();
         if (grid <= 0) return cudaErrorInvalidConfiguration;
-        e = a_tmem ? launch_pdl(k_tc_gemm<false, true>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a)
-                   : launch_pdl(k_tc_gemm<false, false>, dim3(grid), dim3(TC_THREADS), sizeof(TcShared), st, a);
+        if (decode)
+            e = a_tmem ? launch_pdl(k_tc_gemm<TcDecode, false, true>, dim3(grid), dim3(TcDecode::THREADS),
+                                    sizeof(TcDecode::Shared), st, a)
+                       : launch_pdl(k_tc_gemm<TcDecode, false, false>, dim3(grid), dim3(TcDecode::THREADS),
+                                    sizeof(TcDecode::Shared), st, a);
+        else
+            e = a_tmem ? launch_pdl(k_tc_gemm<TcPrefill, false, true>, dim3(grid), dim3(TcPrefill::THREADS),
+                                    sizeof(TcPrefill::Shared), st, a)
+                       : launch_pdl(k_tc_gemm<TcPrefill, false, false>, dim3(grid), dim3(TcPrefill::THREADS),
+                                    sizeof(TcPrefill::Shared), st, a);
     }
     count_launches(1);
     return e;
