@@ -14,6 +14,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.cpp")
+_SRCS = [_SRC, os.path.join(_HERE, "fp8_oracle.cpp")]
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "liboracle.so")
 
@@ -21,10 +22,10 @@ _LIB = os.path.join(_LIB_DIR, "liboracle.so")
 def build(force: bool = False) -> str:
     """Compile the oracle with g++ (-O2, IEEE arithmetic, no contraction)."""
     os.makedirs(_LIB_DIR, exist_ok=True)
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or any(os.path.getmtime(_LIB) < os.path.getmtime(f) for f in _SRCS):
         tmp = _LIB + ".tmp%d" % os.getpid()
         subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-ffp-contract=off",
-                               "-fno-fast-math", "-o", tmp, _SRC, "-lpthread"])
+                               "-fno-fast-math", "-o", tmp] + _SRCS + ["-lpthread"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -58,6 +59,10 @@ def _L():
         _lib.orc_forward_tokens.restype = i32
         _lib.orc_forward_dense.argtypes = [i32] * 5 + [vp] * 6 + [vp, vp, i32]
         _lib.orc_forward_dense.restype = i32
+        _lib.orc_e4m3.argtypes, _lib.orc_e4m3.restype = [i32], d
+        _lib.orc_e4m3_code.argtypes, _lib.orc_e4m3_code.restype = [d], i32
+        _lib.orc_fp8_quant_act.argtypes = [vp, i32, i32, vp, vp, i32]
+        _lib.orc_fp8_linear.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, i32]
     return _lib
 
 
@@ -250,3 +255,40 @@ def forward_dense(x, logits, w1_codes, w1_scales, w2_codes, w2_scales, k: int):
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return y64, y
+
+
+# ---- FP8 block-quantised dense projection (fp8_oracle.cpp) ---------------------
+
+def e4m3(code: int) -> float:
+    """Value of an OCP E4M3 code (NaN for 0x7F / 0xFF)."""
+    return _L().orc_e4m3(code)
+
+
+def e4m3_code(v: float) -> int:
+    """Nearest E4M3 code of v (|v| <= 448), ties to even."""
+    return int(_L().orc_e4m3_code(v))
+
+
+def fp8_quant_act(x_bits: np.ndarray):
+    """x raw bf16 bits [T, K] -> (q [T, K] E4M3 codes, s [T, K/128] UE8M0 bytes)."""
+    x = _c(x_bits, np.uint16)
+    T, K = x.shape
+    assert K % 128 == 0
+    q = np.empty((T, K), np.uint8)
+    s = np.empty((T, K // 128), np.uint8)
+    _L().orc_fp8_quant_act(_p(x), T, K, _p(q), _p(s), nthreads())
+    return q, s
+
+
+def fp8_linear(q: np.ndarray, s: np.ndarray, wq: np.ndarray, ws: np.ndarray, want_f64: bool = False):
+    """y[t, n] = bf16(sum_k dequant(q)[t,k] * dequant(wq)[n,k]); with want_f64 also
+    the fp64 sums and the sums of |terms|."""
+    q, s, wq, ws = _c(q, np.uint8), _c(s, np.uint8), _c(wq, np.uint8), _c(ws, np.uint8)
+    T, K = q.shape
+    N = wq.shape[0]
+    assert wq.shape[1] == K and s.shape == (T, K // 128) and ws.shape == (N // 128, K // 128)
+    y = np.empty((T, N), np.uint16)
+    y64 = np.empty((T, N), np.float64) if want_f64 else None
+    yabs = np.empty((T, N), np.float64) if want_f64 else None
+    _L().orc_fp8_linear(_p(q), _p(s), _p(wq), _p(ws), T, N, K, _p(y), _p(y64), _p(yabs), nthreads())
+    return (y, y64, yabs) if want_f64 else y
