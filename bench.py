@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-skew", action="store_true", help="skip the skewed prefill lines")
     ap.add_argument("--no-decode-t64", action="store_true", help="skip the decode_T64 line")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 dense projection lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tc-pair", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_PAIR for the run (default: the library's default)")
@@ -305,6 +306,58 @@ def run_gpu_workload(name: str, steps: int, warmup: int, dist: Dist, want_e2e: b
     return res
 
 
+def run_fp8_dense(name: str, steps: int, warmup: int, dist: Dist, peaks: dict, want_clocks: bool) -> dict:
+    """The FP8 block-quantised dense projection (moe_fp8_linear: activation
+    quantisation + tcgen05 kind::mxf8f6f4 GEMM), timed as whole calls."""
+    import torch
+
+    import fp4_routed_mixture_b200 as moe
+    w = synth.DENSE_WORKLOADS[name]
+    d = synth.make_dense(w)
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    packed = moe.moe_fp8_pack_weights(cu(d["w_codes"]), cu(d["w_scales"]))
+    x = cu(d["x"]).view(torch.bfloat16)
+    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(w.T, w.K), dtype=torch.uint8, device="cuda")
+    y = torch.empty((w.T, w.N), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        moe.moe_fp8_linear(x, packed, w.N, ws=ws, y=y, stream=stream)
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device()) if want_clocks else None
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        moe.moe_fp8_linear(x, packed, w.N, ws=ws, y=y, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop() if clocks else None
+    ms = dist.max(e0.elapsed_time(e1)) / steps
+    assert moe.moe_check_device_flag(ws) == 0
+    flop = 2.0 * w.T * w.N * w.K
+    wbytes = w.N * w.K + (w.N // 128) * (w.K // 128)
+    line = {"workload": name, "T": w.T, "N": w.N, "K": w.K, "steps": steps,
+            "value": round(whole_job_value(dist.world, w.T, steps, ms * steps), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 5), "clocks": clk,
+            "kernels": "k_fp8_quant_act + k_fp8_gemm (tcgen05 kind::mxf8f6f4 block-scaled); the step times both"}
+    if w.T >= 1024:
+        tf = flop / (ms * 1e-3) / 1e12
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        line["roofline"] = {"bound": "tensor", "achieved": round(tf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
+                            "frac": round(tf / fp8_peak, 5),
+                            "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)", "traffic": None}
+    else:
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                            "frac": round(gbs / peaks["hbm_gbs"], 4), "alg_bytes_per_launch": wbytes,
+                            "peak_source": peaks["source"] + " (hbm_gbs: stream copy)", "traffic": None}
+    del packed, ws
+    torch.cuda.empty_cache()
+    return line
+
+
 def cpu_baseline(name: str, seconds: float) -> dict:
     import oracle
     w = synth.WORKLOADS[name]
@@ -475,6 +528,9 @@ def main():
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
             }
+    if not a.no_fp8:
+        out["fp8_dense"] = [run_fp8_dense(n, max(3, min(cap, steps // 2)), 5, dist, peaks, want_clocks=rank0)
+                            for n, cap in (("dense_T4604", 400), ("dense_T8", 2000))]
     if rank0 and N == 1 and not a.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(a.workload, a.cpu_seconds)
     if rank0:

@@ -18,7 +18,8 @@ from .binding import (FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_BOUNDS, FLAG_LAYOUT,
                       moe_layer_workspace_bytes, make_debug, moe_launch_count,
                       moe_set_option, moe_get_option, MOE_OPT_TC_MIN_ROWS, MOE_OPT_TC_PAIR,
                       MOE_OPT_WAIT_LIMIT_US, MOE_OPT_TEST_TIMEOUT, MOE_OPT_TC_A_TMEM,
-                      moe_sort_static, moe_layer_forward_with_router, moe_layer_router_workspace_bytes)
+                      moe_sort_static, moe_layer_forward_with_router, moe_layer_router_workspace_bytes,
+                      moe_fp8_pack_weights, moe_fp8_unpack_weights, moe_fp8_linear)
 
 __all__ = ["moe_layer_forward", "moe_layer_tables", "moe_layer_workspace_bytes", "make_debug", "moe_pack_weights", "moe_unpack_weights", "moe_router_logits", "moe_route", "moe_sort", "moe_forward",
            "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32", "moe_check_device_flag", "moe_packed_bytes", "moe_workspace_bytes",

@@ -27,6 +27,8 @@ SYMBOLS = ["moe_last_error", "moe_packed_bytes", "moe_pack_weights", "moe_unpack
            "moe_forward", "moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_router_workspace_bytes",
            "moe_layer_forward_with_router", "moe_layer_tables",
            "moe_quant_rows_f32", "moe_exp_f32", "moe_swiglu_f32",
+           "moe_fp8_packed_bytes", "moe_fp8_pack_weights", "moe_fp8_unpack_weights", "moe_fp8_workspace_bytes",
+           "moe_fp8_linear",
            "moe_set_option", "moe_get_option", "moe_launch_count", "moe_check_device_flag"]
 
 
@@ -72,6 +74,11 @@ def _load():
         "moe_quant_rows_f32": ([vp, i32, i32, vp, vp, vp], i32),
         "moe_exp_f32": ([vp, vp, ctypes.c_int64, vp], i32),
         "moe_swiglu_f32": ([vp, vp, vp, ctypes.c_int64, vp], i32),
+        "moe_fp8_packed_bytes": ([i32, i32], sz),
+        "moe_fp8_pack_weights": ([i32, i32, vp, vp, vp, vp], i32),
+        "moe_fp8_unpack_weights": ([i32, i32, vp, vp, vp, vp], i32),
+        "moe_fp8_workspace_bytes": ([i32, i32], sz),
+        "moe_fp8_linear": ([vp, i32, i32, i32, vp, vp, vp, sz, vp, vp, vp], i32),
         "moe_set_option": ([i32, i32], i32),
         "moe_get_option": ([i32], i32),
         "moe_launch_count": ([], ctypes.c_ulonglong),
@@ -339,6 +346,40 @@ def moe_swiglu_f32(g, u, stream=None):
     h = torch.empty_like(g)
     _check(lib.moe_swiglu_f32(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream(stream)))
     return h
+
+
+def moe_fp8_pack_weights(w_codes, w_scales, stream=None) -> torch.Tensor:
+    """FP8 weights, canonical uint8 CUDA tensors [N, K] (E4M3 codes) and
+    [N/128, K/128] (UE8M0 bytes) -> packed device layout.  Synchronises."""
+    N, K = w_codes.shape
+    n = lib.moe_fp8_packed_bytes(N, K)
+    if n == 0:
+        raise MoeError(-2, "unsupported dims")
+    packed = _empty_aligned(n, w_codes.device)
+    _check(lib.moe_fp8_pack_weights(N, K, _ptr(w_codes), _ptr(w_scales), _ptr(packed), _stream(stream)))
+    return packed
+
+
+def moe_fp8_unpack_weights(packed, N: int, K: int, stream=None):
+    wq = torch.empty((N, K), dtype=torch.uint8, device=packed.device)
+    ws = torch.empty((N // 128, K // 128), dtype=torch.uint8, device=packed.device)
+    _check(lib.moe_fp8_unpack_weights(N, K, _ptr(packed), _ptr(wq), _ptr(ws), _stream(stream)))
+    return wq, ws
+
+
+def moe_fp8_linear(x, packed, N: int, ws=None, y=None, debug: dict | None = None, stream=None):
+    """x [T, K] bf16 -> y [T, N] bf16 through the FP8 packed weights.  `debug`
+    may hold uint8 CUDA tensors q [T, K] and s [T, K/128] for the quantised x."""
+    T, K = x.shape
+    if ws is None:
+        ws = _empty_aligned(lib.moe_fp8_workspace_bytes(T, K), x.device)
+    if y is None:
+        y = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
+    dq = (debug or {}).get("q")
+    ds = (debug or {}).get("s")
+    _check(lib.moe_fp8_linear(_ptr(x), T, N, K, _ptr(packed), _ptr(y), _ptr(ws), ws.numel(), _ptr(dq), _ptr(ds),
+                              _stream(stream)))
+    return y
 
 
 MOE_OPT_TC_MIN_ROWS = 1

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -325,7 +326,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (logits) {
         MOE_TRY(moe::launch_layer_front(logits, x_bf16, packed, T, H, I, E, k, group, topk_idx, gates, perm, pos,
                                         offsets,
-                                        uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, xq, sx, xinit,
+                                        uoff1, uoff2, prow, xq, sx, xinit,
                                         dbg ? dbg->xq : nullptr, dbg ? dbg->sx : nullptr, gacc, yacc, flag,
                                         stream),
                 "route + sort + x quant + plan");
@@ -342,9 +343,12 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         MOE_TRY(moe::launch_planes(xtp, H, perm, k, P, prow, L.plane_rows, px, flag, stream), "x planes");
     cudaEvent_t* ev = dbg ? const_cast<cudaEvent_t*>(dbg->events) : nullptr;
     if (ev && ev[0]) MOE_TRY(cudaEventRecord(ev[0], stream), "event");
+    // (with the fused front every row is a streaming row: its streaming rows
+    // are the sorted offsets)
+    const int32_t* gemv_soff = logits ? offsets : soff;
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                                 uoff1, soff, E, gacc, flag, I, P, group, stream), "W1");
+                                 uoff1, gemv_soff, E, gacc, flag, I, P, group, stream), "W1");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
                                     offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns,
@@ -357,7 +361,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                                 uoff2, soff, E, yacc, flag, 0, P, group, stream), "W2");
+                                 uoff2, gemv_soff, E, yacc, flag, 0, P, group, stream), "W2");
     if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
                                     offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns, 0,
@@ -512,6 +516,79 @@ int moe_swiglu_f32(const float* g, const float* u, float* h, int64_t n, cudaStre
     if (n < 0 || (n > 0 && (!g || !u || !h))) return fail(MOE_ERR_INVALID_ARG, "moe_swiglu_f32: bad arguments");
     cudaError_t e = moe::launch_swiglu(g, u, h, n, stream);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_swiglu_f32 launch");
+}
+
+// ---- FP8 block-quantised dense projection -----------------------------------
+
+static int check_fp8_dims(int N, int K, const char* who) {
+    if (N <= 0 || K <= 0 || N % 128 || K % 128)
+        return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: N and K must be positive multiples of 128 (N=%d K=%d)", who, N, K);
+    if ((long long)N * K >= (1LL << 40)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "%s: N*K too large", who);
+    return MOE_OK;
+}
+
+size_t moe_fp8_packed_bytes(int N, int K) {
+    if (N <= 0 || K <= 0 || N % 128 || K % 128) return 0;
+    return moe::fp8_packed_bytes(N, K);
+}
+
+int moe_fp8_pack_weights(int N, int K, const uint8_t* w_codes, const uint8_t* w_scales, void* packed,
+                         cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_fp8_dims(N, K, "moe_fp8_pack_weights")) return rc;
+    if (!w_codes || !w_scales || !packed) return fail(MOE_ERR_INVALID_ARG, "moe_fp8_pack_weights: NULL pointer");
+    if (!aligned(w_codes, 16) || !aligned(packed, 256))
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_pack_weights: codes need 16-byte, packed 256-byte alignment");
+    cudaError_t e = moe::launch_fp8_pack(N, K, w_codes, w_scales, packed, true, nullptr, nullptr, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_fp8_pack_weights launch");
+    int32_t flag = 0;
+    e = cudaMemcpyAsync(&flag, (const char*)packed + offsetof(moe::Fp8Header, flag), sizeof(flag),
+                        cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "moe_fp8_pack_weights");
+    if (flag & MOE_FLAG_BAD_SCALE)
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_pack_weights: scale byte 0xFF (E8M0 NaN) in the input");
+    return MOE_OK;
+}
+
+int moe_fp8_unpack_weights(int N, int K, const void* packed, uint8_t* w_codes, uint8_t* w_scales,
+                           cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_fp8_dims(N, K, "moe_fp8_unpack_weights")) return rc;
+    if (!w_codes || !w_scales || !packed) return fail(MOE_ERR_INVALID_ARG, "moe_fp8_unpack_weights: NULL pointer");
+    if (!aligned(w_codes, 16) || !aligned(packed, 256))
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_unpack_weights: codes need 16-byte, packed 256-byte alignment");
+    cudaError_t e = moe::launch_fp8_pack(N, K, nullptr, nullptr, const_cast<void*>(packed), false, w_codes, w_scales,
+                                         stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_fp8_unpack_weights launch");
+}
+
+size_t moe_fp8_workspace_bytes(int T_max, int K) {
+    if (T_max < 0 || K <= 0 || K % 128) return 0;
+    return moe::fp8_workspace_bytes(T_max, K);
+}
+
+int moe_fp8_linear(const void* x_bf16, int T, int N, int K, const void* packed, void* y_bf16, void* ws,
+                   size_t ws_bytes, uint8_t* dbg_q, uint8_t* dbg_s, cudaStream_t stream) {
+    g_last_error.clear();
+    if (int rc = check_fp8_dims(N, K, "moe_fp8_linear")) return rc;
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: T < 0");
+    if ((long long)T * (K > N ? K : N) >= (1LL << 40)) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "moe_fp8_linear: T too large");
+    if (!ws || !packed || (T > 0 && (!x_bf16 || !y_bf16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: NULL pointer");
+    if (!aligned(ws, 256) || !aligned(packed, 256) || !aligned(x_bf16, 16) || !aligned(y_bf16, 2) ||
+        (dbg_q && !aligned(dbg_q, 16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: ws/packed need 256-byte, x 16-byte alignment");
+    if (ws_bytes < moe::fp8_workspace_bytes(T, K))
+        return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: ws_bytes %zu < %zu", ws_bytes,
+                    moe::fp8_workspace_bytes(T, K));
+    if (T == 0) {
+        cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), stream);
+        return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_fp8_linear memset");
+    }
+    cudaError_t e = moe::launch_fp8_linear(x_bf16, T, N, K, packed, y_bf16, ws, dbg_q, dbg_s, load_options().wait_ns,
+                                           stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_fp8_linear launch");
 }
 
 unsigned long long moe_launch_count(void) { return moe::g_launches.load(); }

@@ -9,9 +9,10 @@
 // rows) and the pairs fit one sort chunk, one launch runs them all, with
 // roles by block:
 //   block 0      routes every token (a warp per token, route_token), sorts the
-//                pairs (sort_cta, expert ids from shared memory) and plans the
-//                streaming units (plan_warp); it also owns the call's error
-//                word (cleared, FLAG_LAYOUT on a packed-header mismatch);
+//                pairs (sort_cta, expert ids from shared memory) and forms the
+//                streaming-unit scans (front_plan_warp); it also owns the
+//                call's error word (cleared, FLAG_LAYOUT on a packed-header
+//                mismatch);
 //   blocks 1..T  x quant of token blockIdx.x - 1 (xquant_row);
 //   the rest     clear the fp64 accumulators of one sorted row each (every
 //                row is a streaming row here).
@@ -34,7 +35,7 @@ struct FrontArgs {
     int32_t* perm;              // [P]
     int32_t* pos;               // [P]
     int32_t* offsets;           // [E + 1]
-    int32_t *unit_off1, *unit_off2, *tile_off1, *tile_off2, *plane_off, *stream_off, *expert_tc, *plane_row;
+    int32_t *unit_off1, *unit_off2, *plane_row;
     int8_t* xq;
     float* sx;
     int32_t* xinit;
@@ -45,6 +46,35 @@ struct FrontArgs {
     int32_t* flag;
 };
 
+// The streaming-unit scans of a call in which every expert takes the
+// streaming GEMM: unit_off1[e] / unit_off2[e] = (token groups of the experts
+// before e) x (weight tiles of W1 / W2), [E] the totals.  One warp; lane l
+// owns a contiguous slice of experts.
+__device__ __forceinline__ void front_plan_warp(const int* offs, int E, int group, int tiles1, int tiles2,
+                                                int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2) {
+    const int lane = threadIdx.x & 31;
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int s = 0;
+    for (int e = e0; e < e1; ++e) s += (offs[e + 1] - offs[e] + group - 1) / group;
+    int x = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    int run = x - s;
+    for (int e = e0; e < e1; ++e) {
+        unit_off1[e] = run * tiles1;
+        unit_off2[e] = run * tiles2;
+        run += (offs[e + 1] - offs[e] + group - 1) / group;
+    }
+    if (lane == 31) {
+        unit_off1[E] = x * tiles1;
+        unit_off2[E] = x * tiles2;
+    }
+}
+
 template <int KMAX, int S>
 __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
     pdl_begin();
@@ -54,7 +84,6 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
         __shared__ int hist[kMaxExperts];
         __shared__ int tmp[kSortThreads + 1];
         __shared__ int offs[kMaxExperts + 1];
-        __shared__ PlanShared ps;
         if (threadIdx.x == 0) *a.flag = packed_header_ok(a.packed, a.H, a.I, a.E) ? 0 : FLAG_LAYOUT;
         const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
         for (int t = warp; t < a.T; t += nwarps)
@@ -63,10 +92,12 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
         __syncthreads();
         sort_cta([&](int p) { return s_idx[p]; }, P, a.E, a.perm, a.pos, a.offsets, hist, tmp, offs, a.flag);
         __syncthreads();
-        // no expert reaches the tensor-core threshold: plan with an unreachable one
-        if (threadIdx.x < 32)
-            plan_warp(offs, a.E, P, 2 * a.I, a.H, 0x7fffffff, kTcTokenTile, a.group, a.unit_off1, a.unit_off2, a.tile_off1,
-                      a.tile_off2, a.plane_off, a.stream_off, a.expert_tc, a.flag, true, ps);
+        // no expert reaches the tensor-core threshold, so the only tables the
+        // launches of this call read are the streaming units of W1 and W2
+        // (units of an expert: its token groups times the weight tiles) and
+        // the streaming rows, which are the sorted offsets themselves
+        if (threadIdx.x < 32) front_plan_warp(offs, a.E, a.group, 2 * a.I / kGemvTileRows, a.H / kGemvTileRows,
+                                              a.unit_off1, a.unit_off2);
         // every row is a streaming row and every expert's streaming rows start
         // at its sorted offset, so sorted row i is streaming row i
         for (int i = threadIdx.x; i < P; i += blockDim.x) a.plane_row[i] = ~i;
@@ -87,14 +118,12 @@ __global__ void __launch_bounds__(kSortThreads) k_layer_front(FrontArgs a) {
 
 cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
                                int E, int k, int group, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
-                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
-                               int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
-                               int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
+                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
                                float* dbg_sx, double* gacc, double* yacc, int32_t* flag, cudaStream_t st) {
     const int P = T * k;
     if (T < 1 || P > kFrontMaxPairs || E > kMaxExperts) return cudaErrorInvalidValue;
     FrontArgs a{logits, (const __nv_bfloat16*)x, packed, T, H, I, E, k, group, topk_idx, gates, perm, pos, offsets,
-                unit_off1, unit_off2, tile_off1, tile_off2, plane_off, stream_off, expert_tc, plane_row, xq, sx, xinit,
+                unit_off1, unit_off2, plane_row, xq, sx, xinit,
                 dbg_xq, dbg_sx, gacc, yacc, flag};
     const dim3 grid(1 + T + P), block(kSortThreads);
     cudaError_t e;

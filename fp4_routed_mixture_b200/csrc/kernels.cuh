@@ -121,9 +121,7 @@ cudaError_t launch_router_logits(const void* x, const float* wr, const float* bi
 constexpr int kFrontMaxPairs = 1024;
 cudaError_t launch_layer_front(const float* logits, const void* x, const void* packed, int T, int H, int I,
                                int E, int k, int group, int32_t* topk_idx, float* gates, int32_t* perm, int32_t* pos,
-                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
-                               int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
-                               int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
+                               int32_t* offsets, int32_t* unit_off1, int32_t* unit_off2, int32_t* plane_row, int8_t* xq, float* sx, int32_t* xinit, int8_t* dbg_xq,
                                float* dbg_sx, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
 
 size_t sort_workspace_bytes(int T_max, int k, int E);
@@ -180,5 +178,20 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,
                            int32_t* flag, cudaStream_t st);
+
+// ---- FP8 block-quantised dense projection (fp8_gemm.cu) ----
+constexpr int kFp8ChunkBytes = 512 + 128 * 128;   // scale atom + 128 x 128 E4M3 codes
+constexpr size_t kFp8HeaderBytes = 256;
+constexpr uint32_t kFp8Magic = 0x57385046u;      // "FP8W"
+struct Fp8Header {
+    uint32_t magic, N, K, reserved;
+    int32_t flag;  // device error word of the packing
+};
+size_t fp8_packed_bytes(int N, int K);
+size_t fp8_workspace_bytes(int T, int K);
+cudaError_t launch_fp8_pack(int N, int K, const uint8_t* wq, const uint8_t* ws, void* packed, bool fwd,
+                            uint8_t* out_wq, uint8_t* out_ws, cudaStream_t st);
+cudaError_t launch_fp8_linear(const void* x, int T, int N, int K, const void* packed, void* y, void* ws,
+                              uint8_t* dbg_q, uint8_t* dbg_s, uint64_t wait_ns, cudaStream_t st);
 
 }  // namespace moe

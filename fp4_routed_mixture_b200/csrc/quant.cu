@@ -80,8 +80,10 @@ __global__ void __launch_bounds__(kQThreads)
         int p = 0;
         if (row_ok) p = checked_index(perm[i], P, flag);
         float4* hr = reinterpret_cast<float4*>(hbuf + (size_t)(row_ok ? i : 0) * I);
+        // KEEP > 0 and the row fits: pass 1 leaves the row in registers
+        const bool use_keep = KEEP > 0 && steps <= KEEP;
         if (row_ok && tc) {
-            if (KEEP > 0) {
+            if (use_keep) {
 #pragma unroll
                 for (int g = 0; g < (KEEP > 0 ? KEEP : 1); ++g)
                     if (g < steps) {
@@ -109,7 +111,14 @@ __global__ void __launch_bounds__(kQThreads)
                     hv[u] = swiglu(gv, uv);
                     a = fmaxf(a, fabsf(hv[u]));
                 }
-                hr[g * R + l] = make_float4(hv[0], hv[1], hv[2], hv[3]);  // read back by this thread
+                const float4 h4 = make_float4(hv[0], hv[1], hv[2], hv[3]);
+                if (use_keep) {
+#pragma unroll
+                    for (int u = 0; u < (KEEP > 0 ? KEEP : 1); ++u)
+                        if (u == g) keep[u] = h4;
+                } else {
+                    hr[g * R + l] = h4;  // read back by this thread
+                }
             }
         }
         if (R == 32)
@@ -127,7 +136,7 @@ __global__ void __launch_bounds__(kQThreads)
         for (int g = 0; g < steps; ++g) {
             const int e0 = 4 * (g * R + l);
             float4 v;
-            if (KEEP > 0 && tc) {
+            if (use_keep) {
                 // (the loop is unrolled KEEP times, so the index is a constant)
 #pragma unroll
                 for (int u = 0; u < (KEEP > 0 ? KEEP : 1); ++u)
@@ -230,7 +239,8 @@ cudaError_t launch_hquant(const double* gacc, float* hbuf, const float* sx, cons
     // rows (prefill): a warp per row needs no block barriers
     cudaError_t e;
     if (P < 4096 && I % (4 * kQThreads) == 0) {
-        e = launch_pdl(k_hquant<kQThreads, 0>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf, sx,
+        // (a thread holds 4 * I / (4 * kQThreads) values: at most 4 float4 up to I = 4096)
+        e = launch_pdl(k_hquant<kQThreads, 4>, dim3(std::min(P, 148 * 8)), dim3(kQThreads), 0, st, gacc, hbuf, sx,
                        perm, plane_row, plane_rows, stream_rows, planes, P, k, I, hq, sh, hinit, dbg_hq, dbg_sh,
                        flag);
     } else {

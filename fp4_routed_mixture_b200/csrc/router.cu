@@ -85,9 +85,65 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Few tokens (decode): the tiled kernel above would run a handful of CTAs.
+// Instead a warp computes one expert's logits for all T <= kRouterSmallT
+// tokens: lane l walks h = 8 l, 8 l + 256, ... , loading 8 router weights
+// (two float4) and, for every token, 8 bf16 inputs (one uint4, from L1/L2:
+// the T rows are shared by every warp), accumulating per token with fused
+// multiply-adds; the per-lane partial sums are then added across the warp.
+// The same summation bound holds (any order).  The router weights, the
+// dominant bytes, are read once, coalesced.
+constexpr int kRouterSmallT = 16;
+
+template <int TMAX>
+__global__ void __launch_bounds__(256)
+    k_router_logits_small(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
+                          const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits) {
+    pdl_begin();
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (e >= E) return;
+    float acc[TMAX];
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) acc[t] = 0.0f;
+    const float* wrow = wr + (size_t)e * H;
+    for (int h = 8 * lane; h < H; h += 256) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(wrow + h));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(wrow + h + 4));
+        const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int t = 0; t < TMAX; ++t) {
+            if (t < T) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H + h));
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[t] = __fmaf_rn(__uint_as_float(xw[j] << 16), w[2 * j], acc[t]);          // bf16 -> fp32, exact
+                    acc[t] = __fmaf_rn(__uint_as_float(xw[j] & 0xffff0000u), w[2 * j + 1], acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TMAX; ++t) {
+        if (t < T) {
+            float v = acc[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) logits[(size_t)t * E + e] = bias ? __fadd_rn(v, __ldg(bias + e)) : v;
+        }
+    }
+}
+
 cudaError_t launch_router_logits(const void* x, const float* wr, const float* bias, int T, int H, int E,
                                  float* logits, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
+    if (T <= kRouterSmallT) {
+        const cudaError_t e = launch_pdl(k_router_logits_small<kRouterSmallT>, dim3((unsigned)((E + 7) / 8)),
+                                         dim3(256), 0, st, (const __nv_bfloat16*)x, wr, bias, T, H, E, logits);
+        count_launches(1);
+        return e;
+    }
     const dim3 grid((unsigned)((E + RT_E - 1) / RT_E), (unsigned)((T + RT_T - 1) / RT_T));
     const cudaError_t e = launch_pdl(k_router_logits, grid, dim3(256), 0, st, (const __nv_bfloat16*)x, wr, bias,
                                      T, H, E, logits);

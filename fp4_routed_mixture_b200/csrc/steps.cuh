@@ -23,9 +23,9 @@ __device__ __forceinline__ bool ranks_above(float a, int ia, float b, int ib) {
     return ia < ib;
 }
 
-// One warp routes one token: row holds its E logits (E <= 32*S); the k chosen
-// ids and gates go to idx_out[0..k) and gates_out[0..k), and the ids also to
-// idx_copy[0..k) when it is not NULL.  Lane l owns logits l, l+32, ... in
+// One warp routes one token: row holds its E logits (E <= 32*S), k <= KMAX
+// <= 32; the k chosen ids and gates go to idx_out[0..k) and gates_out[0..k),
+// and the ids also to idx_copy[0..k) when it is not NULL.  Lane l owns logits l, l+32, ... in
 // registers; each of the k rounds is a warp arg-max (ties to the lower id,
 // NaN last) followed by clearing the winner's bit in its owner's mask.
 template <int KMAX, int S>
@@ -42,11 +42,12 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
         if (id < E) avail |= 1u << s;
     }
 
-    float sel_val[KMAX];
-    int sel_id[KMAX];
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        if (j >= k) break;
+    // k rounds; round j's winner is kept by lane j (the loop body is emitted
+    // once: this code runs once per layer call, with a cold instruction cache)
+    float top = 0.0f, my_val = 0.0f;
+    int my_id = -1;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
         // lane-local best among still-available slots
         float bv = 0.0f;
         int bi = -1;
@@ -68,27 +69,23 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
                 bi = oi;
             }
         }
-        sel_val[j] = bv;
-        sel_id[j] = bi;
+        if (j == 0) top = bv;
+        if (lane == j) {
+            my_val = bv;
+            my_id = bi;
+        }
         if ((bi & 31) == lane) avail &= ~(1u << (bi >> 5));
     }
-    // gates: exp(l_j - l_0) / sum, fp32, slot order
-    if (lane == 0) {
-        float e[KMAX];
-        float den = 0.0f;
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j >= k) break;
-            e[j] = layer_exp(__fsub_rn(sel_val[j], sel_val[0]));
-            den = __fadd_rn(den, e[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            if (j >= k) break;
-            idx_out[j] = sel_id[j];
-            gates_out[j] = __fdiv_rn(e[j], den);
-            if (idx_copy) idx_copy[j] = sel_id[j];
-        }
+    // gates: lane j < k forms exp(l_j - l_0) (all lanes at once); the
+    // denominator is summed in slot order, then lane j divides
+    const float e = layer_exp(__fsub_rn(my_val, top));
+    float den = 0.0f;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) den = __fadd_rn(den, __shfl_sync(0xffffffffu, e, j));
+    if (lane < k) {
+        idx_out[lane] = my_id;
+        gates_out[lane] = __fdiv_rn(e, den);
+        if (idx_copy) idx_copy[lane] = my_id;
     }
 }
 
@@ -99,38 +96,33 @@ constexpr int kSortThreads = 256;
 __device__ __forceinline__ bool valid_expert(int e, int E) { return (unsigned)e < (unsigned)E; }
 
 // Exclusive scan of vals[0..E) in place (blockDim == kSortThreads, E <= 1024);
-// returns the total.  Uses `tmp` [kSortThreads + 1] of shared scratch.
+// returns the total.  Warp 0 scans (lane l owns a contiguous slice of at most
+// 32 entries); the other warps wait at the two barriers.  `tmp` [1] is shared
+// scratch for the total.
 static __device__ int block_exclusive_scan(int* vals, int E, int* tmp) {
-    const int tid = threadIdx.x;
-    const int per = (E + kSortThreads - 1) / kSortThreads;  // <= 4
-    int local[4];
-    int s = 0;
-    for (int j = 0; j < per; ++j) {
-        const int e = tid * per + j;
-        local[j] = (e < E) ? vals[e] : 0;
-        s += local[j];
-    }
-    tmp[tid] = s;
     __syncthreads();
-    // Hillis-Steele over kSortThreads partial sums
-    for (int o = 1; o < kSortThreads; o <<= 1) {
-        const int v = (tid >= o) ? tmp[tid - o] : 0;
-        __syncthreads();
-        tmp[tid] += v;
-        __syncthreads();
-    }
-    int run = (tid == 0) ? 0 : tmp[tid - 1];
-    const int total = tmp[kSortThreads - 1];
-    __syncthreads();
-    for (int j = 0; j < per; ++j) {
-        const int e = tid * per + j;
-        if (e < E) {
-            vals[e] = run;
-            run += local[j];
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (E + 31) / 32;
+        const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+        int s = 0;
+        for (int e = e0; e < e1; ++e) s += vals[e];
+        int x = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
         }
+        int run = x - s;
+        for (int e = e0; e < e1; ++e) {
+            const int v = vals[e];
+            vals[e] = run;
+            run += v;
+        }
+        if (lane == 31) tmp[0] = x;
     }
     __syncthreads();
-    return total;
+    return tmp[0];
 }
 
 // Stable scatter of pairs [p0, p1) (at most 32 x 32 of them) by one warp;

@@ -263,6 +263,51 @@ int moe_quant_rows_f32(const float *v, int rows, int cols, int8_t *q, float *s,
 int moe_exp_f32(const float *x, float *y, int64_t n, cudaStream_t stream);
 int moe_swiglu_f32(const float *g, const float *u, float *h, int64_t n, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * FP8 block-quantised dense projection ([A]: FP8 dense projections; [B]:
+ * "FP8 block quantization").  Readings: OCP E4M3 codes; one UE8M0 scale
+ * (value 2^(byte - 127)) per 128 x 128 weight block and per token x
+ * 128-input activation block;
+ *   xq, sx  per token and 128-input block of x: sx = the smallest power of two
+ *           2^e with max|x| <= 448 * 2^e (byte e + 127, 0 for an all-zero
+ *           block), xq = E4M3 codes of x / 2^e, round to nearest even;
+ *   y[t, n] = bf16( sum_k xq[t,k] 2^(sx[t,k/128]-127) * wq[n,k] 2^(sw[n/128,k/128]-127) )
+ * accumulated in fp32 by the tensor cores (tcgen05 kind::mxf8f6f4 with block
+ * scaling), rounded once to bf16.
+ * Weights, canonical (device memory): w_codes [N, K] uint8 E4M3 codes,
+ * w_scales [N/128, K/128] uint8 UE8M0 bytes; 0xFF (NaN) is rejected.
+ * N % 128 == 0, K % 128 == 0.
+ * ------------------------------------------------------------------------- */
+
+/* Size of the device layout built by moe_fp8_pack_weights (0 for bad dims). */
+size_t moe_fp8_packed_bytes(int N, int K);
+
+/* Canonical -> device layout (256-byte header, then 128 x 128 chunks).
+ * `packed`: moe_fp8_packed_bytes bytes, 256-byte aligned; w_codes 16-byte
+ * aligned.  Load-time call: SYNCHRONISES `stream`; MOE_ERR_INVALID_ARG on a
+ * scale byte 0xFF. */
+int moe_fp8_pack_weights(int N, int K, const uint8_t *w_codes, const uint8_t *w_scales, void *packed,
+                         cudaStream_t stream);
+
+/* Device layout -> canonical, the exact inverse (a round-trip check at load
+ * time catches any layout permutation).  Asynchronous. */
+int moe_fp8_unpack_weights(int N, int K, const void *packed, uint8_t *w_codes, uint8_t *w_scales,
+                           cudaStream_t stream);
+
+/* Workspace of moe_fp8_linear for up to T_max tokens of K inputs (the
+ * quantised activations in the GEMM's tile order; error word first). */
+size_t moe_fp8_workspace_bytes(int T_max, int K);
+
+/* y [T, N] bf16 = the projection of x [T, K] bf16 (16-byte aligned) by the
+ * packed weights.  ws: moe_fp8_workspace_bytes(T_max, K) bytes, 256-byte
+ * aligned, T <= T_max; its first int32 is the device error word (cleared by
+ * this call; MOE_FLAG_LAYOUT when `packed` was built for other N, K; the GEMM
+ * then leaves y untouched; MOE_FLAG_TIMEOUT as in moe_forward).  dbg_q
+ * [T, K] (16-byte aligned) and dbg_s [T, K/128], when not NULL, receive the
+ * E4M3 codes and UE8M0 bytes of x.  Asynchronous, graph-capturable. */
+int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, void *y_bf16, void *ws,
+                   size_t ws_bytes, uint8_t *dbg_q, uint8_t *dbg_s, cudaStream_t stream);
+
 /* Process-wide options.  Each call reads them once when it starts, so a call
  * sees one consistent set; a change made while calls are being enqueued on
  * other host threads applies from the next call that starts after it.

@@ -201,6 +201,46 @@ def custom(name: str, T: int, H: int, E: int, k: int, I: int, seed: int, bias_co
     return Workload(name, T, H, E, k, I, seed, bias_coef)
 
 
+# ---- FP8 block-quantised dense projection inputs --------------------------------
+# x [T, K] ~ N(0, 1) in bf16 (the activation generator above); weights as
+# uniform E4M3 code bytes (the two NaN bytes 0x7F / 0xFF replaced by their
+# neighbours 0x7E / 0xFE, 448 and -448) and one UE8M0 scale byte per 128 x 128
+# block, uniform in {118, ..., 122}.  Shapes use the layer's hidden size.
+TID_F8W, TID_F8S = 16, 17
+
+
+@dataclass(frozen=True)
+class DenseWorkload:
+    name: str
+    T: int
+    N: int
+    K: int
+    seed: int
+
+
+DENSE_WORKLOADS = {
+    w.name: w
+    for w in [
+        DenseWorkload("dense_T8", 8, 4096, 4096, 11),
+        DenseWorkload("dense_T4604", 4604, 4096, 4096, 13),
+    ]
+}
+
+
+def fp8_weights(seed: int, N: int, K: int) -> dict:
+    codes = code_bytes(seed, TID_F8W, (N, K))
+    nan = (codes & 0x7F) == 0x7F
+    codes[nan] -= 1
+    scales = scale_bytes(seed, TID_F8S, (N // 128, K // 128), 118, 5)
+    return dict(w_codes=codes, w_scales=scales)
+
+
+def make_dense(w: DenseWorkload) -> dict:
+    d = dict(x=x_bf16(w.seed, w.T, w.K))
+    d.update(fp8_weights(w.seed, w.N, w.K))
+    return d
+
+
 def bf16_to_f32(a: np.ndarray) -> np.ndarray:
     """Raw bf16 bits (uint16) -> float32 values (exact widening)."""
     return (a.astype(np.uint32) << 16).view(np.float32)

@@ -62,9 +62,11 @@ def test_router_with_bias_skewed_prefill_rows(moe):
     _check(moe, x, wr, bias)
 
 
-@pytest.mark.parametrize("T,H,E", [(1, 32, 1), (65, 160, 65), (3, 128, 1024), (130, 96, 7)])
+@pytest.mark.parametrize("T,H,E", [(1, 32, 1), (65, 160, 65), (3, 128, 1024), (130, 96, 7),
+                                   (16, 4096, 256), (17, 4096, 256), (5, 288, 9)])
 def test_router_ragged_shapes(moe, T, H, E):
-    # tiles of 64 tokens x 64 experts with ragged edges on both sides
+    # tiles of 64 tokens x 64 experts with ragged edges on both sides; up to
+    # 16 tokens the warp-per-expert kernel (E not a multiple of its 8 warps)
     rng = np.random.default_rng(T * 7 + E)
     x = synth.x_bf16(11 + T, T, H)
     wr = (0.02 * rng.standard_normal((E, H))).astype(np.float32)
