@@ -64,6 +64,10 @@ def parse():
                          "(the command profiled under ncu)")
     ap.add_argument("--experts", type=int, default=None,
                     help="with --profile-run: override E (a smaller capture of the same kernels)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="with --profile-run: override T (with --experts: keep the rows per expert)")
+    ap.add_argument("--fp8-workload", default=None,
+                    help="with --profile-run: run the FP8 dense projection of this workload instead")
     return ap.parse_args()
 
 
@@ -411,9 +415,24 @@ def profile_run(a):
     import torch
 
     import fp4_routed_mixture_b200 as moe
+    if a.fp8_workload:
+        fw = synth.DENSE_WORKLOADS[a.fp8_workload]
+        fd = synth.make_dense(fw)
+        cu = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        packed = moe.moe_fp8_pack_weights(cu(fd["w_codes"]), cu(fd["w_scales"]))
+        x = cu(fd["x"]).view(torch.bfloat16)
+        ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(fw.T, fw.K), dtype=torch.uint8, device="cuda")
+        for _ in range(a.steps or 3):
+            y = moe.moe_fp8_linear(x, packed, fw.N, ws=ws)
+        torch.cuda.synchronize()
+        assert moe.moe_check_device_flag(ws) == 0
+        print(f"profile run ok: {fw.name}, {a.steps or 3} steps, max|y| = {float(y.float().abs().max())}")
+        return
     w = synth.WORKLOADS[a.workload]
     if a.experts:
         w = dataclasses.replace(w, name=f"{w.name}_E{a.experts}", E=a.experts)
+    if a.tokens:
+        w = dataclasses.replace(w, name=f"{w.name}_T{a.tokens}", T=a.tokens)
     d = synth.make(w)
     cu = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     packed = moe.moe_pack_weights(*[cu(d[n]) for n in ("w1_codes", "w1_scales", "w2_codes", "w2_scales")])
@@ -491,14 +510,22 @@ def main():
         # ~0.2 s of timed steps per line, so that the clocks sampled under load
         # say whether the tensor-core GEMM ran at the burst or the power-capped
         # sustained clock
-        for key, pname, cap in (("prefill", a.prefill_workload, 150), ("prefill_skew", "prefill_skew_T16384", 50),
-                                ("prefill_skew1.25", "prefill_skew1.25_T16384", 40)):
+        # two regimes per line: a short run (20 / 5 / 5 steps) against the burst
+        # peak, and ~0.2 s of steps with clocks sampled against the sustained
+        # (power-capped) peak
+        for key, pname, cap, long_cap in (("prefill", a.prefill_workload, 20, 150),
+                                          ("prefill_skew", "prefill_skew_T16384", 5, 50),
+                                          ("prefill_skew1.25", "prefill_skew1.25_T16384", 5, 40)):
             if key.startswith("prefill_skew") and a.no_skew:
                 continue
             pw = synth.WORKLOADS[pname]
-            psteps = max(3, min(cap, steps // 10))
-            rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=rank0)
+            psteps = max(3, min(cap, steps // 100))
+            rp = run_gpu_workload(pw.name, psteps, 3, dist, want_e2e=False, want_clocks=False)
+            lsteps = max(3, min(long_cap, steps // 10))
+            rl = run_gpu_workload(pw.name, lsteps, 3, dist, want_e2e=False, want_clocks=rank0)
             ptf = rp["alg_flop_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e12
+            ltf = rl["alg_flop_step"] * lsteps / (rl["gemm_ms"] * 1e-3) / 1e12
+            sus = 2.0 * peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None
             out[key] = {
                 "workload": pw.name, "T": pw.T, "steps": psteps,
                 "value": round(whole_job_value(N, pw.T, psteps, rp["ms"]), 1), "unit": "tokens/s",
@@ -510,21 +537,22 @@ def main():
                                        "block-scaled, plus k_gemv for experts below the row threshold)",
                              "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
                              "frac": round(ptf / fp8_peak, 5),
-                             "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)",
+                             "peak_source": peaks["source"] + " bf16 burst x 2 (fp8/bf16 nominal ratio); "
+                                            "a short run of steps",
                              # the INT8 operand enters the FP4 MMA as three exact digit planes,
                              # so the tensor pipe issues 3x the algorithmic work at the FP4 rate
-                             "frac_vs_sustained": round(ptf / (2.0 * peaks["bf16_tflops_sustained"]), 5)
-                             if peaks.get("bf16_tflops_sustained") else None,
-                             "peak_sustained": 2.0 * peaks["bf16_tflops_sustained"]
-                             if peaks.get("bf16_tflops_sustained") else None,
                              "mma_issued_tflops": round(3 * ptf, 2),
                              "mma_peak_fp4": 4.0 * peaks["bf16_tflops"],
                              "mma_frac_fp4": round(3 * ptf / (4.0 * peaks["bf16_tflops"]), 5),
                              "hbm_achieved_gbs": round(rp["alg_bytes_step"] * psteps / (rp["gemm_ms"] * 1e-3) / 1e9, 1),
                              "traffic": profiled_traffic(f"k_tc_gemm_{pw.name}.md")},
                 "non_gemm_frac": round(1.0 - rp["gemm_ms"] / rp["ms"], 4),
+                "sustained": {"steps": lsteps, "ms_per_step": round(rl["ms"] / lsteps, 4),
+                              "value": round(whole_job_value(N, pw.T, lsteps, rl["ms"]), 1),
+                              "gemm_tflops": round(ltf, 2), "peak": sus,
+                              "frac": round(ltf / sus, 5) if sus else None,
+                              "peak_source": peaks["source"] + " bf16 sustained x 2", "clocks": rl["clocks"]},
                 "router_projection": router_line(rp),
-                "clocks": rp["clocks"],
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
             }
