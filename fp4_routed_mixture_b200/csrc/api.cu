@@ -56,7 +56,7 @@ int check_dims(const moe_dims* d, bool need_T) {
 // Process-wide options (moe_set_option).  Every public call reads them once
 // into an Options value, so a call sees one consistent set even while another
 // host thread changes them.
-std::atomic<int> g_tc_min_rows{32};        // experts with at least this many rows use the tensor-core GEMM
+std::atomic<int> g_tc_min_rows{0};         // tensor-core row threshold; 0 = automatic (see tc_threshold)
 std::atomic<int> g_tc_pair{0};             // tensor-core GEMM in SM pairs (cta_group::2) where the shape allows
 std::atomic<int> g_wait_limit_us{1000000}; // limit of the tensor-core GEMM's bounded waits
 std::atomic<int> g_test_timeout{0};        // one-shot: the next tensor-core launch withholds a stage
@@ -68,6 +68,19 @@ struct Options {
     bool tc_a_tmem;
     uint64_t wait_ns;
 };
+
+// The tensor-core row threshold of a call of T tokens.  Automatic (option 0):
+// calls of fewer than kAutoTcMinT tokens run every expert on the streaming
+// GEMM (with the fused front), larger calls put every expert with at least
+// two rows on the tensor cores -- measured faster than the streaming GEMM from
+// two rows up at decode_T64 and on the skewed prefill, while one-row experts
+// stream better.  An explicit option value is used as it is.
+constexpr int kAutoTcMinT = 32;
+constexpr int kAutoTcMinRows = 2;
+int tc_threshold(int option_value, long long T) {
+    if (option_value > 0) return option_value;
+    return T < kAutoTcMinT ? 0x7fffffff : kAutoTcMinRows;
+}
 
 Options load_options() {
     return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, g_tc_a_tmem.load() != 0,
@@ -246,7 +259,13 @@ int moe_sort_static(const int32_t* topk_idx, int T, int k, int E, int32_t* perm,
 
 size_t moe_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
-    return ws_layout(*d, T_max, g_tc_min_rows.load()).total;
+    const int v = g_tc_min_rows.load();
+    size_t total = ws_layout(*d, T_max, tc_threshold(v, T_max)).total;
+    // (automatic threshold: a call just below kAutoTcMinT tokens keeps every
+    // row on the streaming GEMM and may need more than the larger T_max)
+    if (v == 0 && T_max >= kAutoTcMinT)
+        total = std::max(total, ws_layout(*d, kAutoTcMinT - 1, tc_threshold(v, kAutoTcMinT - 1)).total);
+    return total;
 }
 
 }  // extern "C"
@@ -267,7 +286,8 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if (!aligned(ws, 256) || !aligned(packed, 256) || !aligned(x_bf16, 16) || !aligned(y_bf16, 16))
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: ws/packed need 256-byte, x/y 16-byte alignment");
-    const WsLayout L = ws_layout(*d, d->T, opt.tc_min_rows);
+    const int tc_min = tc_threshold(opt.tc_min_rows, d->T);
+    const WsLayout L = ws_layout(*d, d->T, tc_min);
     if (ws_bytes < L.total)
         return fail(MOE_ERR_INVALID_ARG,
                     "moe_forward: ws_bytes %zu < %zu (the size depends on MOE_OPT_TC_MIN_ROWS: size the "
@@ -300,7 +320,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     } while (0)
     // an expert has at most T rows, so the tensor-core path is skipped without
     // reading any count when T < tc_min (always so with the fused front)
-    const bool use_tc = !logits && T >= opt.tc_min_rows;
+    const bool use_tc = !logits && T >= tc_min;
     // the timeout test applies to the first tensor-core launch after it is armed
     const int withhold = use_tc ? g_test_timeout.exchange(0) : 0;
     // token tile of the tensor-core GEMM: the decode configuration when no
@@ -308,7 +328,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     const int tc_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
     // with a threshold of 1 every expert with rows takes the tensor cores, so
     // the streaming GEMM has nothing to do and is not launched
-    const bool use_gemv = !use_tc || opt.tc_min_rows > 1;
+    const bool use_gemv = !use_tc || tc_min > 1;
     // token rows per streaming-GEMM unit: 2 for small calls (nearly every expert
     // has one or two rows; the smaller ring slot fits more warps per SM), else 4
     const int group = T <= moe::kGemvSmallGroupMaxT ? moe::kGemvSmallGroup : moe::kGemvGroup;
@@ -334,7 +354,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
-        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? opt.tc_min_rows : 0x7fffffff, tc_tile,
+        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? tc_min : 0x7fffffff, tc_tile,
                                       group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
                                       stream),
                 "plan + row state");
@@ -368,7 +388,8 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                                     stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
-    MOE_TRY(moe::launch_combine(yacc, yf, prow, L.stream_rows, sh, gates, pos, T, k, H, y_bf16, flag, stream),
+    MOE_TRY(moe::launch_combine(yacc, yf, logits ? nullptr : etc, offsets, soff, topk_idx, E, L.stream_rows, sh, gates,
+                                pos, T, k, H, y_bf16, flag, stream),
             "combine");
 #undef MOE_TRY
     return MOE_OK;
@@ -417,7 +438,11 @@ static LayerWs layer_ws(const moe_dims& d, long long T, int tc_min) {
 
 size_t moe_layer_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
-    return layer_ws(*d, T_max, g_tc_min_rows.load()).total;
+    const int v = g_tc_min_rows.load();
+    size_t total = layer_ws(*d, T_max, tc_threshold(v, T_max)).total;
+    if (v == 0 && T_max >= kAutoTcMinT)
+        total = std::max(total, layer_ws(*d, kAutoTcMinT - 1, tc_threshold(v, kAutoTcMinT - 1)).total);
+    return total;
 }
 
 int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16, const void* packed,
@@ -429,7 +454,8 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: NULL pointer");
     if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward: ws must be 256-byte aligned");
     const Options opt = load_options();
-    const LayerWs L = layer_ws(*d, d->T, opt.tc_min_rows);
+    const int tc_min = tc_threshold(opt.tc_min_rows, d->T);
+    const LayerWs L = layer_ws(*d, d->T, tc_min);
     if (ws_bytes < L.total)
         return fail(MOE_ERR_INVALID_ARG,
                     "moe_layer_forward: ws_bytes %zu < %zu (the size depends on MOE_OPT_TC_MIN_ROWS: size the "
@@ -440,7 +466,7 @@ int moe_layer_forward(const moe_dims* d, const float* logits, const void* x_bf16
     int32_t* perm = (int32_t*)(w + L.perm);
     int32_t* pos = (int32_t*)(w + L.pos);
     int32_t* offsets = (int32_t*)(w + L.offsets);
-    if (d->T > 0 && d->T < opt.tc_min_rows && (long long)d->T * d->k <= moe::kFrontMaxPairs)
+    if (d->T > 0 && d->T < tc_min && (long long)d->T * d->k <= moe::kFrontMaxPairs)
         return forward_impl(opt, d, logits, x_bf16, idx, gates, perm, pos, offsets, packed, y_bf16, w + L.fwd,
                             L.total - L.fwd, (int32_t*)(w + L.flag), dbg, stream);
     if (int rc = moe_route(logits, d->T, d->E, d->k, idx, gates, stream)) return rc;
@@ -458,7 +484,7 @@ static size_t router_ws_offset(const moe_dims& d, long long T, int tc_min) {
 
 size_t moe_layer_router_workspace_bytes(const moe_dims* d, int T_max) {
     if (check_dims(d, false) != MOE_OK || T_max < 0) return 0;
-    return router_ws_offset(*d, T_max, g_tc_min_rows.load()) + moe::align_up(4 * (size_t)T_max * d->E, 256);
+    return moe::align_up(moe_layer_workspace_bytes(d, T_max), 256) + moe::align_up(4 * (size_t)T_max * d->E, 256);
 }
 
 int moe_layer_forward_with_router(const moe_dims* d, const void* x_bf16, const float* w_router,
@@ -470,8 +496,7 @@ int moe_layer_forward_with_router(const moe_dims* d, const void* x_bf16, const f
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: NULL pointer");
     if (!aligned(ws, 256))
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: ws must be 256-byte aligned");
-    const int tc_min = g_tc_min_rows.load();
-    const size_t lo = router_ws_offset(*d, d->T, tc_min);
+    const size_t lo = router_ws_offset(*d, d->T, tc_threshold(g_tc_min_rows.load(), d->T));
     const size_t need = lo + moe::align_up(4 * (size_t)d->T * d->E, 256);
     if (ws_bytes < need)
         return fail(MOE_ERR_INVALID_ARG, "moe_layer_forward_with_router: ws_bytes %zu < %zu", ws_bytes, need);
@@ -596,7 +621,7 @@ unsigned long long moe_launch_count(void) { return moe::g_launches.load(); }
 int moe_set_option(int option, int value) {
     g_last_error.clear();
     if (option == MOE_OPT_TC_MIN_ROWS) {
-        if (value < 1) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_MIN_ROWS must be >= 1");
+        if (value < 0) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_MIN_ROWS must be >= 0 (0: automatic)");
         g_tc_min_rows = value;
         return MOE_OK;
     }

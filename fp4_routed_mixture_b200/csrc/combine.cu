@@ -14,13 +14,18 @@ namespace moe {
 
 // One thread per 4 consecutive columns of one token (16-byte loads of Y).  The
 // k slots' row indices, gates and kernel choices are read first and all k rows
-// are then loaded before the sum, so the loads overlap.
+// are then loaded before the sum, so the loads overlap.  The kernel choice and
+// the compact streaming row come from per-expert tables (expert_tc, offsets,
+// stream_off: E entries, cache-resident), not from the per-row slot table, so
+// a slot costs no extra dependent miss.  With expert_tc == NULL every row is a
+// streaming row stored at its sorted row.
 template <int KMAX>
 __global__ void __launch_bounds__(256)
     k_combine(const double* __restrict__ yacc, const float* __restrict__ yf,
-              const int32_t* __restrict__ plane_row, int stream_rows, const float* __restrict__ sh,
-              const float* __restrict__ gates, const int32_t* __restrict__ pos, int P, int k, int H,
-              uint2* __restrict__ y, int32_t* flag) {
+              const int32_t* __restrict__ expert_tc, const int32_t* __restrict__ offsets,
+              const int32_t* __restrict__ stream_off, const int32_t* __restrict__ topk_idx, int E,
+              int stream_rows, const float* __restrict__ sh, const float* __restrict__ gates,
+              const int32_t* __restrict__ pos, int P, int k, int H, uint2* __restrict__ y, int32_t* flag) {
     pdl_begin();
     const int t = blockIdx.y;
     const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
@@ -34,9 +39,14 @@ __global__ void __launch_bounds__(256)
             const int p = t * k + j;
             row[j] = checked_index(__ldg(pos + p), P, flag);
             g[j] = __ldg(gates + p);
-            const int slot = __ldg(plane_row + row[j]);   // >= 0: tensor-core row; else ~streaming row
-            tc[j] = slot >= 0;
-            srow[j] = tc[j] ? 0 : checked_index(~slot, stream_rows, flag);
+            tc[j] = false;
+            srow[j] = row[j];
+            if (expert_tc) {
+                const int e = checked_index(__ldg(topk_idx + p), E, flag);
+                tc[j] = __ldg(expert_tc + e) != 0;
+                if (!tc[j])
+                    srow[j] = checked_index(__ldg(stream_off + e) + (row[j] - __ldg(offsets + e)), stream_rows, flag);
+            }
         }
     }
     float4 v[KMAX];
@@ -70,16 +80,17 @@ __global__ void __launch_bounds__(256)
                                              *reinterpret_cast<const uint32_t*>(&hi));
 }
 
-cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
+cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc, const int32_t* offsets,
+                           const int32_t* stream_off, const int32_t* topk_idx, int E, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,
                            int32_t* flag, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     dim3 grid((H / 4 + 255) / 256, T);
     const cudaError_t e =
-        k <= 8 ? launch_pdl(k_combine<8>, grid, dim3(256), 0, st, yacc, yf, plane_row, stream_rows, sh, gates, pos,
-                            T * k, k, H, (uint2*)y, flag)
-               : launch_pdl(k_combine<16>, grid, dim3(256), 0, st, yacc, yf, plane_row, stream_rows, sh, gates,
-                            pos, T * k, k, H, (uint2*)y, flag);
+        k <= 8 ? launch_pdl(k_combine<8>, grid, dim3(256), 0, st, yacc, yf, expert_tc, offsets, stream_off,
+                            topk_idx, E, stream_rows, sh, gates, pos, T * k, k, H, (uint2*)y, flag)
+               : launch_pdl(k_combine<16>, grid, dim3(256), 0, st, yacc, yf, expert_tc, offsets, stream_off,
+                            topk_idx, E, stream_rows, sh, gates, pos, T * k, k, H, (uint2*)y, flag);
     count_launches(1);
     return e;
 }

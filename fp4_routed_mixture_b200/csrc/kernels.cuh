@@ -175,7 +175,11 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
                            const float* row_scale, const int32_t* perm, int k_div, float* out, int token_tile,
                            bool pair, bool a_tmem, uint64_t wait_ns, int withhold, cudaStream_t st);
 
-cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* plane_row, int stream_rows,
+// expert_tc == NULL (the fused decode front): every row is a streaming row at
+// its sorted row; otherwise the kind and the compact streaming row come from
+// expert_tc / offsets / stream_off of the planner.
+cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc, const int32_t* offsets,
+                           const int32_t* stream_off, const int32_t* topk_idx, int E, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,
                            int32_t* flag, cudaStream_t st);
 

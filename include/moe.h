@@ -313,9 +313,14 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
  * other host threads applies from the next call that starts after it.
  *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
  *   run on the tensor-core grouped GEMM (tcgen05, tiles of 128 weight rows x
- *   128 token rows); experts with fewer rows run on the CUDA-core streaming
- *   GEMM.  Default 32; must be >= 1.  Both paths give the same results inside
- *   the exactness domains stated at moe_forward.
+ *   128 token rows, or 32 token rows in calls of at most 64 tokens); experts
+ *   with fewer rows run on the CUDA-core streaming GEMM.  Both paths give the
+ *   same results inside the exactness domains stated at moe_forward.
+ *   0 (the default) is automatic: calls of fewer than 32 tokens run every
+ *   expert on the streaming GEMM (and moe_layer_forward fuses their route,
+ *   sort, x quant and plan into one launch), larger calls use a threshold of
+ *   2.  A value >= 1 is used as it is.  The forward workspace depends on this
+ *   option: size it after setting the option.
  *   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
  *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
  *   multiple of 256); 0 one CTA per SM.  Same results.

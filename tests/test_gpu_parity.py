@@ -42,6 +42,15 @@ def cu(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
+def effective_tc_threshold(moe, T):
+    """The tensor-core row threshold a call of T tokens uses (MOE_OPT_TC_MIN_ROWS;
+    0 = automatic: every expert streams below 32 tokens, else 2)."""
+    v = moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS)
+    if v > 0:
+        return v
+    return 2 ** 31 - 1 if T < 32 else 2
+
+
 def y_check(y_gpu_bf16, y_orc_bits):
     yg = y_gpu_bf16.float().cpu().numpy().astype(np.float64)
     yo = synth.bf16_to_f32(y_orc_bits).astype(np.float64)
@@ -337,9 +346,9 @@ def chosen_tokens(offsets, perm, k, T, n_total=256, seed=7):
 
 @pytest.mark.parametrize("name", ["prefill_T4604", "prefill_skew_T16384", "prefill_skew1.25_T16384"])
 def test_forward_parity_sampled_full_size(moe, workload_data, name):
-    """Full-size prefill workloads in the default configuration (experts with
-    at least 32 rows on the tensor-core GEMM, the others on the streaming
-    GEMM): every routing/sort value is compared whole; the layer's outputs on
+    """Full-size prefill workloads in the default configuration (experts at or
+    above the automatic threshold on the tensor-core GEMM, the others on the
+    streaming GEMM): every routing/sort value is compared whole; the layer's outputs on
     chosen tokens (every touched expert, the largest expert's first, middle and
     last token tile) are compared with the oracle's per-token computation
     (INT8 codes bit-exact, y within tolerance)."""
@@ -358,8 +367,9 @@ def test_forward_parity_sampled_full_size(moe, workload_data, name):
     pairs = (tok[:, None] * w.k + np.arange(w.k)[None, :]).ravel()
     rows = opos[pairs]
     # both kernels are covered wherever the workload has both kinds of expert
-    tc_rows = counts[oi.ravel()[pairs]] >= moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS)
-    if ((counts > 0) & (counts < 32)).any():
+    thr = effective_tc_threshold(moe, w.T)
+    tc_rows = counts[oi.ravel()[pairs]] >= thr
+    if ((counts > 0) & (counts < thr)).any():
         assert (~tc_rows).any()
     assert tc_rows.any()
     assert np.array_equal(r["dbg"]["hq"].cpu().numpy()[rows], ot["hq"])
@@ -425,10 +435,10 @@ def test_tc_forward_parity_decode_T64(moe, workload_data, tc_everywhere):
 
 def test_tc_option_validation(moe):
     with pytest.raises(moe.MoeError):
-        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 0)
+        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, -1)
     with pytest.raises(moe.MoeError):
         moe.moe_set_option(99, 1)
-    assert moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS) >= 1
+    assert moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS) >= 0
 
 
 def test_forward_with_garbage_tables_raises_bounds_flag(moe):

@@ -14,6 +14,7 @@ import torch
 
 import oracle
 import synth
+from tests.test_gpu_parity import effective_tc_threshold
 
 pytestmark = pytest.mark.gpu
 
@@ -84,7 +85,7 @@ def _case(name, shape):
 @pytest.mark.parametrize("name,shape", FRONT_CASES, ids=[c[0] for c in FRONT_CASES])
 def test_fused_front_matches_oracle(moe, name, shape):
     w, d = _case(name, shape)
-    assert w.T < moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS) and w.T * w.k <= 1024
+    assert w.T < effective_tc_threshold(moe, w.T) and w.T * w.k <= 1024
     packed, logits, x = _inputs(moe, d)
     tabs, dbg, y, launches = _layer(moe, w, packed, logits, x)
     # one fused launch + W1, SwiGLU/h quant, W2, combine
