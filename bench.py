@@ -58,6 +58,8 @@ def parse():
                     help="MOE_OPT_TC_MIN_ROWS for the run (1: every expert on the tensor cores)")
     ap.add_argument("--tc-a-tmem", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_A_TMEM for the run (default: the library's default)")
+    ap.add_argument("--tc-weight-major", type=int, choices=[0, 1], default=None,
+                    help="MOE_OPT_TC_WEIGHT_MAJOR for the run (default: the library's default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
                     help="no timing, no JSON: pack the workload and run --steps layer calls "
@@ -446,9 +448,18 @@ def profile_run(a):
     print(f"profile run ok: {w.name}, {a.steps or 3} steps, max|y| = {float(y.float().abs().max())}")
 
 
+def apply_options(a):
+    import fp4_routed_mixture_b200 as moe
+    for value, opt in ((a.tc_pair, moe.MOE_OPT_TC_PAIR), (a.tc_a_tmem, moe.MOE_OPT_TC_A_TMEM),
+                       (a.tc_weight_major, moe.MOE_OPT_TC_WEIGHT_MAJOR), (a.tc_min, moe.MOE_OPT_TC_MIN_ROWS)):
+        if value is not None:
+            moe.moe_set_option(opt, value)
+
+
 def main():
     a = parse()
     if a.profile_run:
+        apply_options(a)
         return profile_run(a)
     if a.impl == "reference":
         return main_reference(a)
@@ -459,12 +470,7 @@ def main():
     import torch
 
     import fp4_routed_mixture_b200 as moe
-    if a.tc_pair is not None:
-        moe.moe_set_option(moe.MOE_OPT_TC_PAIR, a.tc_pair)
-    if a.tc_a_tmem is not None:
-        moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, a.tc_a_tmem)
-    if a.tc_min is not None:
-        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, a.tc_min)
+    apply_options(a)
     rank0 = dist.rank == 0
     peaks = measured_peaks()
     r = run_gpu_workload(a.workload, steps, warmup, dist, want_e2e=True, want_clocks=rank0)
@@ -555,6 +561,7 @@ def main():
                 "router_projection": router_line(rp),
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
+                "tc_weight_major": moe.moe_get_option(moe.MOE_OPT_TC_WEIGHT_MAJOR),
             }
     if not a.no_fp8:
         out["fp8_dense"] = [run_fp8_dense(n, max(3, min(cap, steps // 2)), 5, dist, peaks, want_clocks=rank0)

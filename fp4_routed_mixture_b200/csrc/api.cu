@@ -61,11 +61,13 @@ std::atomic<int> g_tc_pair{0};             // tensor-core GEMM in SM pairs (cta_
 std::atomic<int> g_wait_limit_us{1000000}; // limit of the tensor-core GEMM's bounded waits
 std::atomic<int> g_test_timeout{0};        // one-shot: the next tensor-core launch withholds a stage
 std::atomic<int> g_tc_a_tmem{0};           // tensor-core GEMM with the weight operand staged in TMEM
+std::atomic<int> g_tc_weight_major{0};     // prefill tensor-core GEMM in the weight-major form
 
 struct Options {
     int tc_min_rows;
     bool tc_pair;
     bool tc_a_tmem;
+    bool tc_weight_major;
     uint64_t wait_ns;
 };
 
@@ -84,7 +86,7 @@ int tc_threshold(int option_value, long long T) {
 
 Options load_options() {
     return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, g_tc_a_tmem.load() != 0,
-                   1000ull * (uint64_t)g_wait_limit_us.load()};
+                   g_tc_weight_major.load() != 0, 1000ull * (uint64_t)g_wait_limit_us.load()};
 }
 
 struct WsLayout {
@@ -326,6 +328,10 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     // token tile of the tensor-core GEMM: the decode configuration when no
     // expert can have more than kTcDecodeMaxT rows
     const int tc_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
+    // the prefill configuration runs the token-major form (128 token rows x 256
+    // weight rows per tile) unless a weight-major form is asked for
+    const bool tc_tn = tc_tile == moe::kTcTokenTile && !opt.tc_pair && !opt.tc_a_tmem && !opt.tc_weight_major;
+    const int tc_wtile = tc_tn ? moe::kTcTnWeightTile : moe::kTcWeightTile;
     // with a threshold of 1 every expert with rows takes the tensor cores, so
     // the streaming GEMM has nothing to do and is not launched
     const bool use_gemv = !use_tc || tc_min > 1;
@@ -355,7 +361,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
         MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? tc_min : 0x7fffffff, tc_tile,
-                                      group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
+                                      tc_wtile, group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
                                       stream),
                 "plan + row state");
     }
@@ -369,10 +375,14 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
                                  uoff1, gemv_soff, E, gacc, flag, I, P, group, stream), "W1");
-    if (use_tc)
+    if (use_tc && tc_tn)
+        MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
+                                       offsets, toff1, E, flag, sx, perm, k, hbuf, opt.wait_ns, withhold, stream),
+                "W1 tensor cores");
+    else if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns,
-                                    withhold, stream),
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile, opt.tc_pair, opt.tc_a_tmem,
+                                    opt.wait_ns, withhold, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
     MOE_TRY(moe::launch_hquant(gacc, hbuf, sx, perm, prow, L.plane_rows, L.stream_rows, ph, P, k, I, hq, sh,
@@ -382,10 +392,14 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
                                  uoff2, gemv_soff, E, yacc, flag, 0, P, group, stream), "W2");
-    if (use_tc)
+    if (use_tc && tc_tn)
+        MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
+                                       offsets, toff2, E, flag, sh, perm, 0, yf, opt.wait_ns, 0, stream),
+                "W2 tensor cores");
+    else if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile, opt.tc_pair, opt.tc_a_tmem, opt.wait_ns, 0,
-                                    stream),
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile, opt.tc_pair, opt.tc_a_tmem,
+                                    opt.wait_ns, 0, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");
     MOE_TRY(moe::launch_combine(yacc, yf, logits ? nullptr : etc, offsets, soff, topk_idx, E, L.stream_rows, sh, gates,
@@ -635,6 +649,12 @@ int moe_set_option(int option, int value) {
         g_tc_a_tmem = value;
         return MOE_OK;
     }
+    if (option == MOE_OPT_TC_WEIGHT_MAJOR) {
+        if (value != 0 && value != 1)
+            return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_WEIGHT_MAJOR must be 0 or 1");
+        g_tc_weight_major = value;
+        return MOE_OK;
+    }
     if (option == MOE_OPT_WAIT_LIMIT_US) {
         if (value < 1 || value > 10000000)
             return fail(MOE_ERR_INVALID_ARG, "moe_set_option: WAIT_LIMIT_US must be in [1, 10^7]");
@@ -654,6 +674,7 @@ int moe_get_option(int option) {
     if (option == MOE_OPT_TC_PAIR) return g_tc_pair;
     if (option == MOE_OPT_WAIT_LIMIT_US) return g_wait_limit_us;
     if (option == MOE_OPT_TC_A_TMEM) return g_tc_a_tmem;
+    if (option == MOE_OPT_TC_WEIGHT_MAJOR) return g_tc_weight_major;
     if (option == MOE_OPT_TEST_TIMEOUT) return g_test_timeout;
     return -1;
 }

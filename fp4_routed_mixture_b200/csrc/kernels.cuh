@@ -71,6 +71,9 @@ constexpr int kGemvSmallGroupMaxT = 16;
 constexpr int kMaxExperts = 1024;   // the API's limit on E
 constexpr int kTcWeightTile = 128;
 constexpr int kTcTokenTile = 128;
+// Weight rows per tile of the token-major form (tc_gemm_tn.cu): two packed
+// 128-row chunks.
+constexpr int kTcTnWeightTile = 256;
 // Token tile of the tensor-core GEMM's decode configuration (calls with at
 // most kTcDecodeMaxT tokens, so at most that many rows per expert).
 constexpr int kTcDecodeTokenTile = 32;
@@ -80,10 +83,10 @@ constexpr int kTcDecodeMaxT = 64;
 void count_launches(int n);
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
-                             int I, int H, int tc_min, int tc_tile, int group, int32_t* unit_off1, int32_t* unit_off2,
-                             int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off,
-                             int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc, int32_t* flag,
-                             cudaStream_t st);
+                             int I, int H, int tc_min, int tc_tile, int tc_wtile, int group, int32_t* unit_off1,
+                             int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off,
+                             int32_t* stream_off, int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc,
+                             int32_t* flag, cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may be
 // scheduled before the preceding kernel in the stream completes.  Every kernel
@@ -178,6 +181,14 @@ cudaError_t launch_tc_gemm(const uint8_t* w, size_t expert_bytes, int K, int N, 
 // expert_tc == NULL (the fused decode front): every row is a streaming row at
 // its sorted row; otherwise the kind and the compact streaming row come from
 // expert_tc / offsets / stream_off of the planner.
+// Token-major form (tc_gemm_tn.cu): 128 token rows x 256 weight rows per tile,
+// tile_off counting 256-row weight blocks; the same arguments otherwise.
+cudaError_t launch_tc_gemm_tn(const uint8_t* w, size_t expert_bytes, int K, int N, int gate_up_half,
+                              const uint8_t* planes, int plane_rows, const int32_t* plane_off, int P,
+                              const int32_t* offsets, const int32_t* tile_off, int E, int32_t* flag,
+                              const float* row_scale, const int32_t* perm, int k_div, float* out, uint64_t wait_ns,
+                              int withhold, cudaStream_t st);
+
 cudaError_t launch_combine(const double* yacc, const float* yf, const int32_t* expert_tc, const int32_t* offsets,
                            const int32_t* stream_off, const int32_t* topk_idx, int E, int stream_rows,
                            const float* sh, const float* gates, const int32_t* pos, int T, int k, int H, void* y,

@@ -312,23 +312,29 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
  * sees one consistent set; a change made while calls are being enqueued on
  * other host threads applies from the next call that starts after it.
  *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
- *   run on the tensor-core grouped GEMM (tcgen05, tiles of 128 weight rows x
- *   128 token rows, or 32 token rows in calls of at most 64 tokens); experts
- *   with fewer rows run on the CUDA-core streaming GEMM.  Both paths give the
+ *   run on the tensor-core grouped GEMM (tcgen05; tiles of 128 token rows x
+ *   256 weight rows, or 32 token rows x 128 weight rows in calls of at most 64
+ *   tokens); experts with fewer rows run on the CUDA-core streaming GEMM.  Both paths give the
  *   same results inside the exactness domains stated at moe_forward.
  *   0 (the default) is automatic: calls of fewer than 32 tokens run every
  *   expert on the streaming GEMM (and moe_layer_forward fuses their route,
  *   sort, x quant and plan into one launch), larger calls use a threshold of
  *   2.  A value >= 1 is used as it is.  The forward workspace depends on this
  *   option: size it after setting the option.
- *   MOE_OPT_TC_PAIR: 1 runs the tensor-core GEMM in SM pairs (clusters of two
- *   CTAs, tcgen05 cta_group::2, M = 256) where the weight rows allow it (a
- *   multiple of 256); 0 one CTA per SM.  Same results.
- *   MOE_OPT_TC_A_TMEM: 1 stages each pipeline stage's weight chunk in tensor
- *   memory once (tcgen05.cp) and runs the six digit-plane MMAs of the stage
- *   with A read from there, so shared memory feeds only the activation
- *   operand; 0 reads both operands from shared memory.  One CTA per SM (it
- *   takes precedence over MOE_OPT_TC_PAIR).  Same results.
+ *   MOE_OPT_TC_WEIGHT_MAJOR: 1 runs the tensor-core GEMM of calls of more than
+ *   64 tokens in its weight-major form (128 weight rows as the MMA's M, 128
+ *   token rows as its N) instead of the token-major form (128 token rows as
+ *   M, two 128-row weight chunks as N); 0 (default) the token-major form.
+ *   Same results.
+ *   MOE_OPT_TC_PAIR: 1 runs the weight-major tensor-core GEMM in SM pairs
+ *   (clusters of two CTAs, tcgen05 cta_group::2, M = 256) where the weight
+ *   rows allow it (a multiple of 256); 0 one CTA per SM.  Same results.
+ *   MOE_OPT_TC_A_TMEM: 1 runs the weight-major tensor-core GEMM with each
+ *   pipeline stage's weight chunk staged in tensor memory once (tcgen05.cp)
+ *   and the six digit-plane MMAs of the stage reading A from there, so shared
+ *   memory feeds only the activation operand; 0 reads both operands from
+ *   shared memory.  One CTA per SM (it takes precedence over
+ *   MOE_OPT_TC_PAIR).  Same results.
  *   MOE_OPT_WAIT_LIMIT_US: limit, in microseconds, of every bounded wait inside
  *   the tensor-core GEMM (a pipeline stage normally lands in a few
  *   microseconds).  A wait that runs out raises MOE_FLAG_TIMEOUT in the call's
@@ -346,6 +352,7 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
 #define MOE_OPT_WAIT_LIMIT_US 3
 #define MOE_OPT_TEST_TIMEOUT 4
 #define MOE_OPT_TC_A_TMEM 5
+#define MOE_OPT_TC_WEIGHT_MAJOR 6
 int moe_set_option(int option, int value);
 int moe_get_option(int option);
 

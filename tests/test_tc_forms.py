@@ -1,6 +1,9 @@
-"""The tensor-core grouped GEMM's alternative forms against the plain
-one-CTA-per-SM form (both operands from shared memory) and the oracle:
+"""The tensor-core grouped GEMM's alternative forms against the default form
+(token-major for calls of more than 64 tokens, the weight-major decode
+configuration below) and the oracle:
 
+* the weight-major form for every call size (MOE_OPT_TC_WEIGHT_MAJOR = 1:
+  128 weight rows as the MMA's M, 128 token rows as its N, one CTA per SM);
 * SM pairs (MOE_OPT_TC_PAIR = 1: clusters of two CTAs, tcgen05 cta_group::2,
   M = 256), where the weight rows of a matrix are a multiple of 256 (W1
   always, W2 when H is); other shapes fall back to one CTA per SM, which a
@@ -37,13 +40,14 @@ def cu(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def _run(moe, d, w, pair, a_tmem=False):
+def _run(moe, d, w, pair, a_tmem=False, weight_major=False):
     T, H, I, E, k = w.T, w.H, w.I, w.E, w.k
-    old = (moe.moe_get_option(moe.MOE_OPT_TC_MIN_ROWS), moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
-           moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM))
+    keys = (moe.MOE_OPT_TC_MIN_ROWS, moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM, moe.MOE_OPT_TC_WEIGHT_MAJOR)
+    old = tuple(moe.moe_get_option(k_) for k_ in keys)
     moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
     moe.moe_set_option(moe.MOE_OPT_TC_PAIR, 1 if pair else 0)
     moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, 1 if a_tmem else 0)
+    moe.moe_set_option(moe.MOE_OPT_TC_WEIGHT_MAJOR, 1 if weight_major else 0)
     try:
         packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]),
                                       cu(d["w2_scales"]))
@@ -60,9 +64,8 @@ def _run(moe, d, w, pair, a_tmem=False):
         assert moe.moe_check_device_flag(ws) == 0
         return y, dbg
     finally:
-        moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, old[0])
-        moe.moe_set_option(moe.MOE_OPT_TC_PAIR, old[1])
-        moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, old[2])
+        for k_, v in zip(keys, old):
+            moe.moe_set_option(k_, v)
 
 
 @pytest.mark.parametrize("T,H,E,k,I,seed", [
@@ -71,13 +74,14 @@ def _run(moe, d, w, pair, a_tmem=False):
     (9, 256, 16, 16, 128, 73),     # k = E: 16 experts, tiny token tiles (n_mma = 16)
     (13, 384, 9, 3, 256, 74),      # H = 384: W2 falls back to one CTA per SM, W1 in pairs
     (257, 256, 1, 1, 128, 75),     # E = 1, three token tiles, the last holds one row
+    (300, 384, 4, 2, 256, 76),     # token-major W2 with a ragged 128-row weight block
 ])
-@pytest.mark.parametrize("form", ["pair", "a_tmem"])
+@pytest.mark.parametrize("form", ["pair", "a_tmem", "weight_major"])
 def test_form_matches_single_and_oracle(moe, form, T, H, E, k, I, seed):
     w = synth.custom("pair", T, H, E, k, I, seed)
     d = synth.make(w)
     y1, d1 = _run(moe, d, w, pair=False)
-    y2, d2 = _run(moe, d, w, pair=form == "pair", a_tmem=form == "a_tmem")
+    y2, d2 = _run(moe, d, w, pair=form == "pair", a_tmem=form == "a_tmem", weight_major=form == "weight_major")
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(d1["hq"], d2["hq"])
     assert torch.equal(d1["sh"].view(torch.int32), d2["sh"].view(torch.int32))
@@ -93,7 +97,7 @@ def test_form_matches_single_and_oracle(moe, form, T, H, E, k, I, seed):
 
 
 def test_form_option_validation(moe):
-    for opt in (moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM):
+    for opt in (moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM, moe.MOE_OPT_TC_WEIGHT_MAJOR):
         with pytest.raises(moe.MoeError):
             moe.moe_set_option(opt, 2)
         assert moe.moe_get_option(opt) in (0, 1)

@@ -30,11 +30,13 @@ def moe():
     return m
 
 
-def test_withheld_stage_times_out_then_next_call_is_exact(moe):
+# 40 tokens: the weight-major decode configuration; 100 tokens: the token-major form
+@pytest.mark.parametrize("T", [40, 100])
+def test_withheld_stage_times_out_then_next_call_is_exact(moe, T):
     keys = [moe.MOE_OPT_TC_MIN_ROWS, moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_WAIT_LIMIT_US,
             moe.MOE_OPT_TEST_TIMEOUT]
     old = {k_: moe.moe_get_option(k_) for k_ in keys}
-    w = synth.custom("to", 40, 256, 2, 1, 128, 51)
+    w = synth.custom("to", T, 256, 2, 1, 128, 51)
     d = synth.make(w)
     try:
         moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
