@@ -43,12 +43,17 @@
 //                16-lane x 256-bit shape, in which four consecutive threads
 //                hold eight consecutive columns of one token row, so every
 //                store instruction writes whole 32-byte sectors of eight rows.
-// Three 128-column accumulators rotate over the (tile, half) sequence: half h
-// of the CTA's tile j uses accumulator (2j + h) mod 3.  At a tile boundary the
-// issuer of half 0 finds its accumulator long drained (it last held half 1 of
-// the tile two back), and only the issuer of half 1 waits for the epilogue to
-// read half 0 of the tile just finished, so the tensor core keeps working
-// while a tile drains.
+// Three 128-column accumulators rotate over the (tile, half) sequence: use
+// u = 2j + h (half h of the CTA's tile j) takes accumulator u mod 3.  At a
+// tile boundary the issuer of half 0 finds its accumulator long drained (it
+// last held half 1 of the tile two back), and only the issuer of half 1 waits
+// for the epilogue to read half 0 of the tile just finished, so the tensor
+// core keeps working while a tile drains.  Every epilogue warp waits for every
+// use in order and releases it (count 16), the warps of the other half without
+// reading it: each barrier's phases are then seen one after another by all of
+// its waiters, so no parity wait can mistake a phase two ahead or behind (an
+// issuer waits for the release of use u - 3 only after it has seen the release
+// of use u - 5, which every warp gave after that of u - 6).
 // Every wait is bounded in time; a wait that gives up raises FLAG_TIMEOUT and
 // the roles wind down (copies in flight are waited for, TMEM is freed).
 #include "kernels.cuh"
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(TN_THREADS, 1) k_tc_gemm_tn(TnArgs a) {
         }
         for (int b = 0; b < TN_ACC; ++b) {
             mbar_init(smem_u32(&sh.acc_full[b]), 1);                  // one issuer's commit
-            mbar_init(smem_u32(&sh.acc_empty[b]), TN_EPI_WARPS / 2);  // the warps of one half
+            mbar_init(smem_u32(&sh.acc_empty[b]), TN_EPI_WARPS);      // every epilogue warp
         }
         mbar_init(smem_u32(&sh.drain[0]), 1);
         mbar_init(smem_u32(&sh.drain[1]), 1);
@@ -356,11 +361,24 @@ __global__ void __launch_bounds__(TN_THREADS, 1) k_tc_gemm_tn(TnArgs a) {
         const int half = cg >> 1;
         const int t4 = lane >> 2, c2 = 2 * (lane & 3);
         const bool w1 = a.gate_up_half > 0;
+        // waits for use u and releases it (the caller reads it in between)
+        auto acquire = [&](int u) -> bool {
+            if (!wait(smem_u32(&sh.acc_full[u % TN_ACC]), (uint32_t)(u / TN_ACC) & 1u)) {
+                give_up();
+                return false;
+            }
+            tc_fence_after();
+            return true;
+        };
+        auto release = [&](int u) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[u % TN_ACC]));
+        };
         for (int j = 0; j < ntiles && !*abort; ++j) {
             const TnTile tt = tn_tile_at(a, tile_of(j));
             const bool mine = half < tt.halves;
             const int u = 2 * j + half, buf = u % TN_ACC;
-            const uint32_t use = (uint32_t)(u / TN_ACC);
             float s[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -372,11 +390,12 @@ __global__ void __launch_bounds__(TN_THREADS, 1) k_tc_gemm_tn(TnArgs a) {
                     s[k] = __ldg(a.row_scale + src);
                 }
             }
-            if (!wait(smem_u32(&sh.acc_full[buf]), use & 1u)) {
-                give_up();
-                break;
+            // the other half's use of this tile, when it comes first
+            if (half == 1) {
+                if (!acquire(u - 1)) break;
+                release(u - 1);
             }
-            tc_fence_after();
+            if (!acquire(u)) break;
             uint32_t v[64];   // v[32L + 4jj + 2hh + e]: row 32q + 16L + 8hh + t/4, column 8jj + c2 + e
             if (mine) {
                 const uint32_t taddr =
@@ -386,9 +405,12 @@ __global__ void __launch_bounds__(TN_THREADS, 1) k_tc_gemm_tn(TnArgs a) {
                 tn_wait_ld();
             }
             // the values are in registers: release the accumulator
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sh.acc_empty[buf]));
+            release(u);
+            // the other half's use of this tile, when it comes second
+            if (half == 0) {
+                if (!acquire(u + 1)) break;
+                release(u + 1);
+            }
             if (!mine) continue;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
