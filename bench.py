@@ -58,8 +58,8 @@ def parse():
                     help="MOE_OPT_TC_MIN_ROWS for the run (1: every expert on the tensor cores)")
     ap.add_argument("--tc-a-tmem", type=int, choices=[0, 1], default=None,
                     help="MOE_OPT_TC_A_TMEM for the run (default: the library's default)")
-    ap.add_argument("--tc-weight-major", type=int, choices=[0, 1], default=None,
-                    help="MOE_OPT_TC_WEIGHT_MAJOR for the run (default: the library's default)")
+    ap.add_argument("--tc-form", type=int, choices=[0, 1, 2], default=None,
+                    help="MOE_OPT_TC_FORM for the run (default: the library's default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--profile-run", action="store_true",
                     help="no timing, no JSON: pack the workload and run --steps layer calls "
@@ -182,20 +182,21 @@ def measured_peaks() -> dict:
 
 def profiled_traffic(summary: str):
     """DRAM bytes per launch (read + write) of a GEMM kernel, from a committed ncu
-    summary under profiles/; None unless the kernel source is unchanged since the
-    capture (the summary records the source file and its SHA-256)."""
+    summary under profiles/; None unless every kernel source is unchanged since
+    the capture (the summary records each source file and its SHA-256)."""
     p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
     text = open(p).read()
-    src = re.search(r"^\s*kernel_source:\s*(\S+)", text, re.M)
-    sha = re.search(r"^\s*kernel_source_sha256:\s*([0-9a-f]{64})", text, re.M)
+    srcs = re.findall(r"^\s*kernel_source:\s*(\S+)", text, re.M)
+    shas = re.findall(r"^\s*kernel_source_sha256:\s*([0-9a-f]{64})", text, re.M)
     val = re.search(r"^\s*dram_bytes_per_launch:\s*(\d+)", text, re.M)
-    if not (src and sha and val):
+    if not (srcs and len(srcs) == len(shas) and val):
         return None
-    path = os.path.join(ROOT, src.group(1))
-    if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest() != sha.group(1):
-        return None
+    for src, sha in zip(srcs, shas):   # every source the captured kernels were built from
+        path = os.path.join(ROOT, src)
+        if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest() != sha:
+            return None
     return int(val.group(1))
 
 
@@ -451,7 +452,7 @@ def profile_run(a):
 def apply_options(a):
     import fp4_routed_mixture_b200 as moe
     for value, opt in ((a.tc_pair, moe.MOE_OPT_TC_PAIR), (a.tc_a_tmem, moe.MOE_OPT_TC_A_TMEM),
-                       (a.tc_weight_major, moe.MOE_OPT_TC_WEIGHT_MAJOR), (a.tc_min, moe.MOE_OPT_TC_MIN_ROWS)):
+                       (a.tc_form, moe.MOE_OPT_TC_FORM), (a.tc_min, moe.MOE_OPT_TC_MIN_ROWS)):
         if value is not None:
             moe.moe_set_option(opt, value)
 
@@ -561,7 +562,7 @@ def main():
                 "router_projection": router_line(rp),
                 "tc_pair": moe.moe_get_option(moe.MOE_OPT_TC_PAIR),
                 "tc_a_tmem": moe.moe_get_option(moe.MOE_OPT_TC_A_TMEM),
-                "tc_weight_major": moe.moe_get_option(moe.MOE_OPT_TC_WEIGHT_MAJOR),
+                "tc_form": moe.moe_get_option(moe.MOE_OPT_TC_FORM),
             }
     if not a.no_fp8:
         out["fp8_dense"] = [run_fp8_dense(n, max(3, min(cap, steps // 2)), 5, dist, peaks, want_clocks=rank0)

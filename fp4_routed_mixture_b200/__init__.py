@@ -18,7 +18,7 @@ from .binding import (FLAG_BAD_EXPERT, FLAG_BAD_SCALE, FLAG_BOUNDS, FLAG_LAYOUT,
                       moe_layer_workspace_bytes, make_debug, moe_launch_count,
                       moe_set_option, moe_get_option, MOE_OPT_TC_MIN_ROWS, MOE_OPT_TC_PAIR,
                       MOE_OPT_WAIT_LIMIT_US, MOE_OPT_TEST_TIMEOUT, MOE_OPT_TC_A_TMEM,
-                      MOE_OPT_TC_WEIGHT_MAJOR,
+                      MOE_OPT_TC_FORM,
                       moe_sort_static, moe_layer_forward_with_router, moe_layer_router_workspace_bytes,
                       moe_fp8_pack_weights, moe_fp8_unpack_weights, moe_fp8_linear)
 

@@ -387,7 +387,7 @@ MOE_OPT_TC_PAIR = 2
 MOE_OPT_WAIT_LIMIT_US = 3
 MOE_OPT_TEST_TIMEOUT = 4
 MOE_OPT_TC_A_TMEM = 5
-MOE_OPT_TC_WEIGHT_MAJOR = 6
+MOE_OPT_TC_FORM = 6
 
 
 def moe_set_option(option: int, value: int):

@@ -61,13 +61,13 @@ std::atomic<int> g_tc_pair{0};             // tensor-core GEMM in SM pairs (cta_
 std::atomic<int> g_wait_limit_us{1000000}; // limit of the tensor-core GEMM's bounded waits
 std::atomic<int> g_test_timeout{0};        // one-shot: the next tensor-core launch withholds a stage
 std::atomic<int> g_tc_a_tmem{0};           // tensor-core GEMM with the weight operand staged in TMEM
-std::atomic<int> g_tc_weight_major{0};     // prefill tensor-core GEMM in the weight-major form
+std::atomic<int> g_tc_form{0};             // forms of the prefill tensor-core GEMMs (MOE_OPT_TC_FORM)
 
 struct Options {
     int tc_min_rows;
     bool tc_pair;
     bool tc_a_tmem;
-    bool tc_weight_major;
+    int tc_form;
     uint64_t wait_ns;
 };
 
@@ -86,7 +86,7 @@ int tc_threshold(int option_value, long long T) {
 
 Options load_options() {
     return Options{g_tc_min_rows.load(), g_tc_pair.load() != 0, g_tc_a_tmem.load() != 0,
-                   g_tc_weight_major.load() != 0, 1000ull * (uint64_t)g_wait_limit_us.load()};
+                   g_tc_form.load(), 1000ull * (uint64_t)g_wait_limit_us.load()};
 }
 
 struct WsLayout {
@@ -328,10 +328,16 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     // token tile of the tensor-core GEMM: the decode configuration when no
     // expert can have more than kTcDecodeMaxT rows
     const int tc_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
-    // the prefill configuration runs the token-major form (128 token rows x 256
-    // weight rows per tile) unless a weight-major form is asked for
-    const bool tc_tn = tc_tile == moe::kTcTokenTile && !opt.tc_pair && !opt.tc_a_tmem && !opt.tc_weight_major;
-    const int tc_wtile = tc_tn ? moe::kTcTnWeightTile : moe::kTcWeightTile;
+    // forms of the prefill configuration: W1 token-major (128 token rows x 256
+    // weight rows per tile: half the activation-operand traffic per MMA), W2
+    // weight-major (lanes are weight rows, so its fp32 Y rows are stored in
+    // whole 128-byte lines); MOE_OPT_TC_FORM and the weight-major variants
+    // (pair, A in TMEM) change that
+    const bool tc_prefill_tn = tc_tile == moe::kTcTokenTile && !opt.tc_pair && !opt.tc_a_tmem;
+    const bool tc_tn1 = tc_prefill_tn && opt.tc_form != 1;
+    const bool tc_tn2 = tc_prefill_tn && opt.tc_form == 2;
+    const int tc_wtile1 = tc_tn1 ? moe::kTcTnWeightTile : moe::kTcWeightTile;
+    const int tc_wtile2 = tc_tn2 ? moe::kTcTnWeightTile : moe::kTcWeightTile;
     // with a threshold of 1 every expert with rows takes the tensor cores, so
     // the streaming GEMM has nothing to do and is not launched
     const bool use_gemv = !use_tc || tc_min > 1;
@@ -361,7 +367,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
         MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? tc_min : 0x7fffffff, tc_tile,
-                                      tc_wtile, group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
+                                      tc_wtile1, tc_wtile2, group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
                                       stream),
                 "plan + row state");
     }
@@ -375,7 +381,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
                                  uoff1, gemv_soff, E, gacc, flag, I, P, group, stream), "W1");
-    if (use_tc && tc_tn)
+    if (use_tc && tc_tn1)
         MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
                                        offsets, toff1, E, flag, sx, perm, k, hbuf, opt.wait_ns, withhold, stream),
                 "W1 tensor cores");
@@ -392,7 +398,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
                                  uoff2, gemv_soff, E, yacc, flag, 0, P, group, stream), "W2");
-    if (use_tc && tc_tn)
+    if (use_tc && tc_tn2)
         MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
                                        offsets, toff2, E, flag, sh, perm, 0, yf, opt.wait_ns, 0, stream),
                 "W2 tensor cores");
@@ -649,10 +655,9 @@ int moe_set_option(int option, int value) {
         g_tc_a_tmem = value;
         return MOE_OK;
     }
-    if (option == MOE_OPT_TC_WEIGHT_MAJOR) {
-        if (value != 0 && value != 1)
-            return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_WEIGHT_MAJOR must be 0 or 1");
-        g_tc_weight_major = value;
+    if (option == MOE_OPT_TC_FORM) {
+        if (value < 0 || value > 2) return fail(MOE_ERR_INVALID_ARG, "moe_set_option: TC_FORM must be 0, 1 or 2");
+        g_tc_form = value;
         return MOE_OK;
     }
     if (option == MOE_OPT_WAIT_LIMIT_US) {
@@ -674,7 +679,7 @@ int moe_get_option(int option) {
     if (option == MOE_OPT_TC_PAIR) return g_tc_pair;
     if (option == MOE_OPT_WAIT_LIMIT_US) return g_wait_limit_us;
     if (option == MOE_OPT_TC_A_TMEM) return g_tc_a_tmem;
-    if (option == MOE_OPT_TC_WEIGHT_MAJOR) return g_tc_weight_major;
+    if (option == MOE_OPT_TC_FORM) return g_tc_form;
     if (option == MOE_OPT_TEST_TIMEOUT) return g_test_timeout;
     return -1;
 }

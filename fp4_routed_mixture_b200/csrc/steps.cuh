@@ -300,9 +300,9 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 
 // ---- plan ----------------------------------------------------------------------------
 // Work split per expert: experts with at least tc_min rows go to the
-// tensor-core GEMM (tiles of tc_wtile weight rows x tc_tile token rows, the
-// tile of the form and configuration that GEMM is launched with; a ragged last
-// weight block counts as a tile), the others to the streaming GEMM (units of kGemvTileRows weight rows
+// tensor-core GEMM (tiles of tc_wtile1 / tc_wtile2 weight rows of W1 / W2 x
+// tc_tile token rows, the tiles of the forms and configuration those GEMMs are
+// launched with; a ragged last weight block counts as a tile), the others to the streaming GEMM (units of kGemvTileRows weight rows
 // x `group` tokens, the group size the streaming GEMM is launched with).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
@@ -327,7 +327,7 @@ struct PlanShared {
 constexpr int32_t kNoRow = INT32_MIN;
 
 static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
-                                 int tc_tile, int tc_wtile, int group,
+                                 int tc_tile, int tc_wtile1, int tc_wtile2, int group,
                                  int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                                  int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                                  int32_t* __restrict__ plane_off, int32_t* __restrict__ stream_off,
@@ -349,8 +349,8 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
         const int nb = tc ? (m + tc_tile - 1) / tc_tile : 0;
         c[0] = g * (n1 / kGemvTileRows);
         c[1] = g * (n2 / kGemvTileRows);
-        c[2] = nb * ((n1 + tc_wtile - 1) / tc_wtile);
-        c[3] = nb * ((n2 + tc_wtile - 1) / tc_wtile);
+        c[2] = nb * ((n1 + tc_wtile1 - 1) / tc_wtile1);
+        c[3] = nb * ((n2 + tc_wtile2 - 1) / tc_wtile2);
         c[4] = tc ? (m + 15) & ~15 : 0;
         c[5] = tc ? 0 : m;
     };

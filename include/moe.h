@@ -321,15 +321,16 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
  *   sort, x quant and plan into one launch), larger calls use a threshold of
  *   2.  A value >= 1 is used as it is.  The forward workspace depends on this
  *   option: size it after setting the option.
- *   MOE_OPT_TC_WEIGHT_MAJOR: 1 runs the tensor-core GEMM of calls of more than
- *   64 tokens in its weight-major form (128 weight rows as the MMA's M, 128
- *   token rows as its N) instead of the token-major form (128 token rows as
- *   M, two 128-row weight chunks as N); 0 (default) the token-major form.
- *   Same results.
- *   MOE_OPT_TC_PAIR: 1 runs the weight-major tensor-core GEMM in SM pairs
+ *   MOE_OPT_TC_FORM: the forms of the tensor-core GEMMs of calls of more than
+ *   64 tokens.  0 (default): W1 token-major (128 token rows as the MMA's M,
+ *   two 128-row weight chunks as N: the activation operand is staged once for
+ *   256 weight rows), W2 weight-major (128 weight rows as M, 128 token rows as
+ *   N: its fp32 output rows are stored in whole lines); 1: both weight-major;
+ *   2: both token-major.  Same results.
+ *   MOE_OPT_TC_PAIR: 1 runs both tensor-core GEMMs weight-major in SM pairs
  *   (clusters of two CTAs, tcgen05 cta_group::2, M = 256) where the weight
  *   rows allow it (a multiple of 256); 0 one CTA per SM.  Same results.
- *   MOE_OPT_TC_A_TMEM: 1 runs the weight-major tensor-core GEMM with each
+ *   MOE_OPT_TC_A_TMEM: 1 runs both tensor-core GEMMs weight-major with each
  *   pipeline stage's weight chunk staged in tensor memory once (tcgen05.cp)
  *   and the six digit-plane MMAs of the stage reading A from there, so shared
  *   memory feeds only the activation operand; 0 reads both operands from
@@ -352,7 +353,7 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
 #define MOE_OPT_WAIT_LIMIT_US 3
 #define MOE_OPT_TEST_TIMEOUT 4
 #define MOE_OPT_TC_A_TMEM 5
-#define MOE_OPT_TC_WEIGHT_MAJOR 6
+#define MOE_OPT_TC_FORM 6
 int moe_set_option(int option, int value);
 int moe_get_option(int option);
 

@@ -417,9 +417,10 @@ def tc_everywhere(moe):
     (13, 384, 9, 3, 256, 42),      # tiny experts: n_mma = 16
     (9, 256, 16, 16, 128, 43),     # k = E
     (257, 128, 1, 1, 128, 53),     # E = 1, 257 rows: three n-blocks, last holds one row
-    # token-major form (calls of more than 64 tokens): 256-row weight blocks
-    (300, 384, 4, 2, 256, 54),     # W2 with H = 384: a ragged last weight block of 128 rows
-    (130, 640, 3, 3, 384, 56),     # W1 N = 768 (three blocks), W2 N = 640 (two and a half)
+    # calls of more than 64 tokens: W1 token-major (256-row weight blocks), W2
+    # weight-major; both token-major in tests/test_tc_forms.py
+    (300, 384, 4, 2, 256, 54),     # H = 384: W2 with three 128-row weight blocks
+    (130, 640, 3, 3, 384, 56),     # W1 N = 768 (three 256-row blocks), W2 N = 640
     (65, 256, 64, 2, 128, 57),     # one token row more than the decode configuration takes
 ])
 def test_tc_forward_parity_shapes(moe, tc_everywhere, T, H, E, k, I, seed):

@@ -1,9 +1,10 @@
-"""The tensor-core grouped GEMM's alternative forms against the default form
-(token-major for calls of more than 64 tokens, the weight-major decode
-configuration below) and the oracle:
+"""The tensor-core grouped GEMM's alternative forms against the default forms
+(for calls of more than 64 tokens W1 token-major and W2 weight-major; the
+weight-major decode configuration below) and the oracle:
 
-* the weight-major form for every call size (MOE_OPT_TC_WEIGHT_MAJOR = 1:
-  128 weight rows as the MMA's M, 128 token rows as its N, one CTA per SM);
+* both GEMMs weight-major (MOE_OPT_TC_FORM = 1: 128 weight rows as the MMA's
+  M, 128 token rows as its N, one CTA per SM) or both token-major
+  (MOE_OPT_TC_FORM = 2: 128 token rows as M, two 128-row weight chunks as N);
 * SM pairs (MOE_OPT_TC_PAIR = 1: clusters of two CTAs, tcgen05 cta_group::2,
   M = 256), where the weight rows of a matrix are a multiple of 256 (W1
   always, W2 when H is); other shapes fall back to one CTA per SM, which a
@@ -40,14 +41,14 @@ def cu(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def _run(moe, d, w, pair, a_tmem=False, weight_major=False):
+def _run(moe, d, w, pair, a_tmem=False, form=0):
     T, H, I, E, k = w.T, w.H, w.I, w.E, w.k
-    keys = (moe.MOE_OPT_TC_MIN_ROWS, moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM, moe.MOE_OPT_TC_WEIGHT_MAJOR)
+    keys = (moe.MOE_OPT_TC_MIN_ROWS, moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM, moe.MOE_OPT_TC_FORM)
     old = tuple(moe.moe_get_option(k_) for k_ in keys)
     moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
     moe.moe_set_option(moe.MOE_OPT_TC_PAIR, 1 if pair else 0)
     moe.moe_set_option(moe.MOE_OPT_TC_A_TMEM, 1 if a_tmem else 0)
-    moe.moe_set_option(moe.MOE_OPT_TC_WEIGHT_MAJOR, 1 if weight_major else 0)
+    moe.moe_set_option(moe.MOE_OPT_TC_FORM, form)
     try:
         packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]),
                                       cu(d["w2_scales"]))
@@ -76,12 +77,13 @@ def _run(moe, d, w, pair, a_tmem=False, weight_major=False):
     (257, 256, 1, 1, 128, 75),     # E = 1, three token tiles, the last holds one row
     (300, 384, 4, 2, 256, 76),     # token-major W2 with a ragged 128-row weight block
 ])
-@pytest.mark.parametrize("form", ["pair", "a_tmem", "weight_major"])
+@pytest.mark.parametrize("form", ["pair", "a_tmem", "weight_major", "token_major"])
 def test_form_matches_single_and_oracle(moe, form, T, H, E, k, I, seed):
     w = synth.custom("pair", T, H, E, k, I, seed)
     d = synth.make(w)
     y1, d1 = _run(moe, d, w, pair=False)
-    y2, d2 = _run(moe, d, w, pair=form == "pair", a_tmem=form == "a_tmem", weight_major=form == "weight_major")
+    y2, d2 = _run(moe, d, w, pair=form == "pair", a_tmem=form == "a_tmem",
+                  form={"weight_major": 1, "token_major": 2}.get(form, 0))
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(d1["hq"], d2["hq"])
     assert torch.equal(d1["sh"].view(torch.int32), d2["sh"].view(torch.int32))
@@ -97,7 +99,11 @@ def test_form_matches_single_and_oracle(moe, form, T, H, E, k, I, seed):
 
 
 def test_form_option_validation(moe):
-    for opt in (moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM, moe.MOE_OPT_TC_WEIGHT_MAJOR):
+    for opt in (moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_TC_A_TMEM):
         with pytest.raises(moe.MoeError):
             moe.moe_set_option(opt, 2)
         assert moe.moe_get_option(opt) in (0, 1)
+    for bad in (-1, 3):
+        with pytest.raises(moe.MoeError):
+            moe.moe_set_option(moe.MOE_OPT_TC_FORM, bad)
+    assert moe.moe_get_option(moe.MOE_OPT_TC_FORM) in (0, 1, 2)
