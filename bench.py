@@ -402,11 +402,14 @@ def router_line(r: dict) -> dict:
             "kernel": "k_router_logits (fp32 CUDA-core contraction)", "in_metric": False}
 
 
-def roofline_hbm(r: dict, peaks: dict, traffic):
-    n_launch = 2 * r["steps"]
+def roofline_hbm(r: dict, peaks: dict, traffic, kernel="k_gemv (W1 and W2 launches)", per_step=2):
+    """HBM roofline of the W1 + W2 GEMM phases (events around each phase);
+    per_step = GEMM launches per step, alg_bytes_per_launch = the step's weight
+    bytes split over the two phases."""
+    n_launch = per_step * r["steps"]
     bytes_per_launch = r["alg_bytes_step"] / 2.0
     achieved = (r["alg_bytes_step"] * r["steps"]) / (r["gemm_ms"] * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": "k_gemv (W1 and W2 launches)", "achieved": round(achieved, 1),
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": traffic, "launches": n_launch, "alg_bytes_per_launch": bytes_per_launch,
             "peak_source": peaks["source"] + " (hbm_gbs: stream copy)"}
@@ -506,7 +509,11 @@ def main():
             "workload": dw.name, "T": dw.T, "steps": dsteps,
             "value": round(whole_job_value(N, dw.T, dsteps, rd["ms"]), 1), "unit": "tokens/s",
             "ms_per_step": round(rd["ms"] / dsteps, 5), "touched_experts": rd["touched"],
-            "roofline": roofline_hbm(rd, peaks, profiled_traffic(f"k_gemv_{dw.name}.md")),
+            # (at 64 tokens experts with two or more rows take the tensor cores)
+            "roofline": roofline_hbm(rd, peaks, profiled_traffic(f"k_tc_gemm_{dw.name}.md"),
+                                     kernel="W1 and W2 phases: k_tc_gemm (decode configuration) for experts "
+                                            "with two or more rows, k_gemv for one-row experts",
+                                     per_step=4),
         }
     if not a.no_prefill:
         # prefill lines (tensor-core path): the prefill chunk, the skewed
@@ -540,8 +547,9 @@ def main():
                 "gemm_ms_per_step": round(rp["gemm_ms"] / psteps, 4),
                 "touched_experts": rp["touched"],
                 "roofline": {"bound": "tensor",
-                             "kernel": "W1 and W2 grouped GEMM launches (k_tc_gemm tcgen05 kind::mxf4 "
-                                       "block-scaled, plus k_gemv for experts below the row threshold)",
+                             "kernel": "W1 and W2 grouped GEMM launches (tcgen05 kind::mxf4 block-scaled: "
+                                       "k_tc_gemm_tn token-major for W1, k_tc_gemm weight-major for W2; "
+                                       "k_gemv for one-row experts)",
                              "achieved": round(ptf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
                              "frac": round(ptf / fp8_peak, 5),
                              "peak_source": peaks["source"] + " bf16 burst x 2 (fp8/bf16 nominal ratio); "

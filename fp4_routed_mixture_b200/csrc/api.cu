@@ -325,17 +325,19 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     const bool use_tc = !logits && T >= tc_min;
     // the timeout test applies to the first tensor-core launch after it is armed
     const int withhold = use_tc ? g_test_timeout.exchange(0) : 0;
-    // token tile of the tensor-core GEMM: the decode configuration when no
-    // expert can have more than kTcDecodeMaxT rows
-    const int tc_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
-    // forms of the prefill configuration: W1 token-major (128 token rows x 256
+    // Forms of the tensor-core GEMMs: W1 token-major (128 token rows x 256
     // weight rows per tile: half the activation-operand traffic per MMA), W2
     // weight-major (lanes are weight rows, so its fp32 Y rows are stored in
-    // whole 128-byte lines); MOE_OPT_TC_FORM and the weight-major variants
-    // (pair, A in TMEM) change that
-    const bool tc_prefill_tn = tc_tile == moe::kTcTokenTile && !opt.tc_pair && !opt.tc_a_tmem;
-    const bool tc_tn1 = tc_prefill_tn && opt.tc_form != 1;
-    const bool tc_tn2 = tc_prefill_tn && opt.tc_form == 2;
+    // whole 128-byte lines) with 128-row token tiles, or 32-row ones (the
+    // decode configuration) when no expert can have more than kTcDecodeMaxT
+    // rows.  MOE_OPT_TC_FORM 1 / 2 take both weight-major / both token-major;
+    // the weight-major variants (pair, A in TMEM) take both weight-major.
+    const int wm_tile = T <= moe::kTcDecodeMaxT ? moe::kTcDecodeTokenTile : moe::kTcTokenTile;
+    const bool wm_variant = opt.tc_pair || opt.tc_a_tmem;
+    const bool tc_tn1 = !wm_variant && opt.tc_form != 1;
+    const bool tc_tn2 = !wm_variant && opt.tc_form == 2;
+    const int tc_tile1 = tc_tn1 ? moe::kTcTokenTile : wm_tile;
+    const int tc_tile2 = tc_tn2 ? moe::kTcTokenTile : wm_tile;
     const int tc_wtile1 = tc_tn1 ? moe::kTcTnWeightTile : moe::kTcWeightTile;
     const int tc_wtile2 = tc_tn2 ? moe::kTcTnWeightTile : moe::kTcWeightTile;
     // with a threshold of 1 every expert with rows takes the tensor cores, so
@@ -366,9 +368,9 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
         MOE_TRY(moe::launch_xquant(x_bf16, T, H, xq, sx, xinit, use_tc ? xtp : nullptr, dbg ? dbg->xq : nullptr,
                                    dbg ? dbg->sx : nullptr, packed, I, E, flag, stream),
                 "x quant + header check");
-        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? tc_min : 0x7fffffff, tc_tile,
-                                      tc_wtile1, tc_wtile2, group, uoff1, uoff2, toff1, toff2, poff, soff, etc, prow, gacc, yacc, flag,
-                                      stream),
+        MOE_TRY(moe::launch_plan_rows(offsets, topk_idx, perm, E, P, I, H, use_tc ? tc_min : 0x7fffffff, tc_tile1,
+                                      tc_tile2, tc_wtile1, tc_wtile2, group, uoff1, uoff2, toff1, toff2, poff, soff,
+                                      etc, prow, gacc, yacc, flag, stream),
                 "plan + row state");
     }
     if (use_tc)
@@ -387,7 +389,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                 "W1 tensor cores");
     else if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
-                                    offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile, opt.tc_pair, opt.tc_a_tmem,
+                                    offsets, toff1, E, flag, sx, perm, k, hbuf, tc_tile1, opt.tc_pair, opt.tc_a_tmem,
                                     opt.wait_ns, withhold, stream),
                 "W1 tensor cores");
     if (ev && ev[1]) MOE_TRY(cudaEventRecord(ev[1], stream), "event");
@@ -404,7 +406,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
                 "W2 tensor cores");
     else if (use_tc)
         MOE_TRY(moe::launch_tc_gemm(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
-                                    offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile, opt.tc_pair, opt.tc_a_tmem,
+                                    offsets, toff2, E, flag, sh, perm, 0, yf, tc_tile2, opt.tc_pair, opt.tc_a_tmem,
                                     opt.wait_ns, 0, stream),
                 "W2 tensor cores");
     if (ev && ev[3]) MOE_TRY(cudaEventRecord(ev[3], stream), "event");

@@ -83,11 +83,10 @@ constexpr int kTcDecodeMaxT = 64;
 void count_launches(int n);
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
-                             int I, int H, int tc_min, int tc_tile, int tc_wtile1, int tc_wtile2, int group,
-                             int32_t* unit_off1,
-                             int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off,
-                             int32_t* stream_off, int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc,
-                             int32_t* flag, cudaStream_t st);
+                             int I, int H, int tc_min, int tc_tile1, int tc_tile2, int tc_wtile1, int tc_wtile2,
+                             int group, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
+                             int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
+                             int32_t* plane_row, double* gacc, double* yacc, int32_t* flag, cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may be
 // scheduled before the preceding kernel in the stream completes.  Every kernel

@@ -22,8 +22,8 @@ namespace moe {
 // Rows of tensor-core experts are written whole by that GEMM.
 __global__ void __launch_bounds__(256)
     k_plan_rows(const int32_t* __restrict__ offsets, const int32_t* __restrict__ topk_idx,
-                const int32_t* __restrict__ perm, int E, int P, int I, int H, int tc_min, int tc_tile, int tc_wtile1,
-                int tc_wtile2, int group,
+                const int32_t* __restrict__ perm, int E, int P, int I, int H, int tc_min, int tc_tile1, int tc_tile2,
+                int tc_wtile1, int tc_wtile2, int group,
                 int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                 int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                 int32_t* __restrict__ plane_off, int32_t* __restrict__ stream_off,
@@ -32,8 +32,8 @@ __global__ void __launch_bounds__(256)
     pdl_begin();
     __shared__ PlanShared ps;
     if (threadIdx.x < 32)
-        plan_warp(offsets, E, P, 2 * I, H, tc_min, tc_tile, tc_wtile1, tc_wtile2, group, unit_off1, unit_off2, tile_off1,
-                  tile_off2, plane_off, stream_off, expert_tc, flag, blockIdx.x == 0, ps);
+        plan_warp(offsets, E, P, 2 * I, H, tc_min, tc_tile1, tc_tile2, tc_wtile1, tc_wtile2, group, unit_off1,
+                  unit_off2, tile_off1, tile_off2, plane_off, stream_off, expert_tc, flag, blockIdx.x == 0, ps);
     __syncthreads();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P; i += gridDim.x * blockDim.x) {
         const int e = checked_index(topk_idx[checked_index(perm[i], P, flag)], E, flag);
@@ -59,15 +59,15 @@ __global__ void __launch_bounds__(256)
 }
 
 cudaError_t launch_plan_rows(const int32_t* offsets, const int32_t* topk_idx, const int32_t* perm, int E, int P,
-                             int I, int H, int tc_min, int tc_tile, int tc_wtile1, int tc_wtile2, int group,
-                             int32_t* unit_off1,
-                             int32_t* unit_off2, int32_t* tile_off1, int32_t* tile_off2, int32_t* plane_off,
-                             int32_t* stream_off, int32_t* expert_tc, int32_t* plane_row, double* gacc, double* yacc,
-                             int32_t* flag, cudaStream_t st) {
+                             int I, int H, int tc_min, int tc_tile1, int tc_tile2, int tc_wtile1, int tc_wtile2,
+                             int group, int32_t* unit_off1, int32_t* unit_off2, int32_t* tile_off1,
+                             int32_t* tile_off2, int32_t* plane_off, int32_t* stream_off, int32_t* expert_tc,
+                             int32_t* plane_row, double* gacc, double* yacc, int32_t* flag, cudaStream_t st) {
     const int grid = std::max(1, std::min(P, 148 * 8));
     const cudaError_t e = launch_pdl(k_plan_rows, dim3(grid), dim3(256), 0, st, offsets, topk_idx, perm, E, P, I,
-                                     H, tc_min, tc_tile, tc_wtile1, tc_wtile2, group, unit_off1, unit_off2, tile_off1, tile_off2,
-                                     plane_off, stream_off, expert_tc, plane_row, gacc, yacc, flag);
+                                     H, tc_min, tc_tile1, tc_tile2, tc_wtile1, tc_wtile2, group, unit_off1, unit_off2,
+                                     tile_off1, tile_off2, plane_off, stream_off, expert_tc, plane_row, gacc, yacc,
+                                     flag);
     count_launches(1);
     return e;
 }

@@ -300,9 +300,10 @@ __device__ __forceinline__ void xquant_row(const __nv_bfloat16* __restrict__ x, 
 
 // ---- plan ----------------------------------------------------------------------------
 // Work split per expert: experts with at least tc_min rows go to the
-// tensor-core GEMM (tiles of tc_wtile1 / tc_wtile2 weight rows of W1 / W2 x
-// tc_tile token rows, the tiles of the forms and configuration those GEMMs are
-// launched with; a ragged last weight block counts as a tile), the others to the streaming GEMM (units of kGemvTileRows weight rows
+// tensor-core GEMM (tiles of tc_tile1 / tc_tile2 token rows x tc_wtile1 /
+// tc_wtile2 weight rows of W1 / W2, the tiles of the forms and configurations
+// those GEMMs are launched with; a ragged last weight block counts as a tile),
+// the others to the streaming GEMM (units of kGemvTileRows weight rows
 // x `group` tokens, the group size the streaming GEMM is launched with).  Forms the exclusive scans over experts of the streaming
 // units of W1/W2, of the tensor-core tiles of W1/W2 and of the digit-plane rows
 // (each tensor-core expert's rows padded to a multiple of 16, so that every
@@ -327,7 +328,7 @@ struct PlanShared {
 constexpr int32_t kNoRow = INT32_MIN;
 
 static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int P, int n1, int n2, int tc_min,
-                                 int tc_tile, int tc_wtile1, int tc_wtile2, int group,
+                                 int tc_tile1, int tc_tile2, int tc_wtile1, int tc_wtile2, int group,
                                  int32_t* __restrict__ unit_off1, int32_t* __restrict__ unit_off2,
                                  int32_t* __restrict__ tile_off1, int32_t* __restrict__ tile_off2,
                                  int32_t* __restrict__ plane_off, int32_t* __restrict__ stream_off,
@@ -346,11 +347,12 @@ static __device__ void plan_warp(const int32_t* __restrict__ offsets, int E, int
         const int m = any_bad ? 0 : offsets[e + 1] - offsets[e];
         const bool tc = m >= tc_min;
         const int g = tc ? 0 : (m + group - 1) / group;
-        const int nb = tc ? (m + tc_tile - 1) / tc_tile : 0;
+        const int nb1 = tc ? (m + tc_tile1 - 1) / tc_tile1 : 0;
+        const int nb2 = tc ? (m + tc_tile2 - 1) / tc_tile2 : 0;
         c[0] = g * (n1 / kGemvTileRows);
         c[1] = g * (n2 / kGemvTileRows);
-        c[2] = nb * ((n1 + tc_wtile1 - 1) / tc_wtile1);
-        c[3] = nb * ((n2 + tc_wtile2 - 1) / tc_wtile2);
+        c[2] = nb1 * ((n1 + tc_wtile1 - 1) / tc_wtile1);
+        c[3] = nb2 * ((n2 + tc_wtile2 - 1) / tc_wtile2);
         c[4] = tc ? (m + 15) & ~15 : 0;
         c[5] = tc ? 0 : m;
     };

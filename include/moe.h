@@ -312,21 +312,21 @@ int moe_fp8_linear(const void *x_bf16, int T, int N, int K, const void *packed, 
  * sees one consistent set; a change made while calls are being enqueued on
  * other host threads applies from the next call that starts after it.
  *   MOE_OPT_TC_MIN_ROWS: experts with at least this many token rows in a call
- *   run on the tensor-core grouped GEMM (tcgen05; tiles of 128 token rows x
- *   256 weight rows, or 32 token rows x 128 weight rows in calls of at most 64
- *   tokens); experts with fewer rows run on the CUDA-core streaming GEMM.  Both paths give the
+ *   run on the tensor-core grouped GEMMs (tcgen05, forms: MOE_OPT_TC_FORM);
+ *   experts with fewer rows run on the CUDA-core streaming GEMM.  Both paths give the
  *   same results inside the exactness domains stated at moe_forward.
  *   0 (the default) is automatic: calls of fewer than 32 tokens run every
  *   expert on the streaming GEMM (and moe_layer_forward fuses their route,
  *   sort, x quant and plan into one launch), larger calls use a threshold of
  *   2.  A value >= 1 is used as it is.  The forward workspace depends on this
  *   option: size it after setting the option.
- *   MOE_OPT_TC_FORM: the forms of the tensor-core GEMMs of calls of more than
- *   64 tokens.  0 (default): W1 token-major (128 token rows as the MMA's M,
- *   two 128-row weight chunks as N: the activation operand is staged once for
- *   256 weight rows), W2 weight-major (128 weight rows as M, 128 token rows as
- *   N: its fp32 output rows are stored in whole lines); 1: both weight-major;
- *   2: both token-major.  Same results.
+ *   MOE_OPT_TC_FORM: the forms of the tensor-core GEMMs.  0 (default): W1
+ *   token-major (128 token rows as the MMA's M, two 128-row weight chunks as
+ *   N: the activation operand is staged once for 256 weight rows), W2
+ *   weight-major (128 weight rows as M, token rows as N: its fp32 output rows
+ *   are stored in whole lines; 128-row token tiles, or 32-row ones in calls of
+ *   at most 64 tokens); 1: both weight-major; 2: both token-major.  Same
+ *   results.
  *   MOE_OPT_TC_PAIR: 1 runs both tensor-core GEMMs weight-major in SM pairs
  *   (clusters of two CTAs, tcgen05 cta_group::2, M = 256) where the weight
  *   rows allow it (a multiple of 256); 0 one CTA per SM.  Same results.

@@ -30,17 +30,20 @@ def moe():
     return m
 
 
-# 40 tokens: the weight-major decode configuration; 100 tokens: the token-major form
-@pytest.mark.parametrize("T", [40, 100])
-def test_withheld_stage_times_out_then_next_call_is_exact(moe, T):
+# the W1 kernel whose stage is withheld: weight-major decode configuration
+# (40 tokens, form 1), weight-major prefill configuration (100 tokens, form 1),
+# token-major (form 0)
+@pytest.mark.parametrize("T,form", [(40, 1), (100, 1), (100, 0)])
+def test_withheld_stage_times_out_then_next_call_is_exact(moe, T, form):
     keys = [moe.MOE_OPT_TC_MIN_ROWS, moe.MOE_OPT_TC_PAIR, moe.MOE_OPT_WAIT_LIMIT_US,
-            moe.MOE_OPT_TEST_TIMEOUT]
+            moe.MOE_OPT_TEST_TIMEOUT, moe.MOE_OPT_TC_FORM]
     old = {k_: moe.moe_get_option(k_) for k_ in keys}
     w = synth.custom("to", T, 256, 2, 1, 128, 51)
     d = synth.make(w)
     try:
         moe.moe_set_option(moe.MOE_OPT_TC_MIN_ROWS, 1)
         moe.moe_set_option(moe.MOE_OPT_TC_PAIR, 0)
+        moe.moe_set_option(moe.MOE_OPT_TC_FORM, form)
         moe.moe_set_option(moe.MOE_OPT_WAIT_LIMIT_US, 20000)   # 20 ms
         packed = moe.moe_pack_weights(cu(d["w1_codes"]), cu(d["w1_scales"]), cu(d["w2_codes"]),
                                       cu(d["w2_scales"]))
