@@ -402,16 +402,19 @@ def router_line(r: dict) -> dict:
             "kernel": "k_router_logits (fp32 CUDA-core contraction)", "in_metric": False}
 
 
-def roofline_hbm(r: dict, peaks: dict, traffic, kernel="k_gemv (W1 and W2 launches)", per_step=2):
-    """HBM roofline of the W1 + W2 GEMM phases (events around each phase);
-    per_step = GEMM launches per step, alg_bytes_per_launch = the step's weight
-    bytes split over the two phases."""
-    n_launch = per_step * r["steps"]
-    bytes_per_launch = r["alg_bytes_step"] / 2.0
+def roofline_hbm(r: dict, peaks: dict, traffic, kernel="k_gemv (W1 and W2 launches)", per_phase=1):
+    """HBM roofline of the W1 + W2 GEMM phases (events around each phase, one or
+    more launches each).  The step's weight bytes are split over the two
+    phases; with one launch per phase they are the bytes per launch, and the
+    traffic (DRAM bytes, from a committed ncu summary) is per phase."""
+    n_launch = 2 * per_phase * r["steps"]
+    bytes_per_phase = r["alg_bytes_step"] / 2.0
     achieved = (r["alg_bytes_step"] * r["steps"]) / (r["gemm_ms"] * 1e-3) / 1e9
+    per = {"alg_bytes_per_launch": bytes_per_phase} if per_phase == 1 else \
+          {"alg_bytes_per_phase": bytes_per_phase, "traffic_is": "DRAM bytes per phase"}
     return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic, "launches": n_launch, "alg_bytes_per_launch": bytes_per_launch,
+            "traffic": traffic, "launches": n_launch, **per,
             "peak_source": peaks["source"] + " (hbm_gbs: stream copy)"}
 
 
@@ -511,9 +514,10 @@ def main():
             "ms_per_step": round(rd["ms"] / dsteps, 5), "touched_experts": rd["touched"],
             # (at 64 tokens experts with two or more rows take the tensor cores)
             "roofline": roofline_hbm(rd, peaks, profiled_traffic(f"k_tc_gemm_{dw.name}.md"),
-                                     kernel="W1 and W2 phases: k_tc_gemm (decode configuration) for experts "
-                                            "with two or more rows, k_gemv for one-row experts",
-                                     per_step=4),
+                                     kernel="W1 and W2 phases, two launches each: k_gemv for one-row experts, "
+                                            "then the tensor cores for experts with two or more rows "
+                                            "(W1 k_tc_gemm_tn, W2 k_tc_gemm decode configuration)",
+                                     per_phase=2),
         }
     if not a.no_prefill:
         # prefill lines (tensor-core path): the prefill chunk, the skewed
