@@ -324,7 +324,7 @@ def run_fp8_dense(name: str, steps: int, warmup: int, dist: Dist, peaks: dict, w
     cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     packed = moe.moe_fp8_pack_weights(cu(d["w_codes"]), cu(d["w_scales"]))
     x = cu(d["x"]).view(torch.bfloat16)
-    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(w.T, w.K), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(w.T, w.N, w.K), dtype=torch.uint8, device="cuda")
     y = torch.empty((w.T, w.N), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
@@ -430,7 +430,7 @@ def profile_run(a):
         cu = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
         packed = moe.moe_fp8_pack_weights(cu(fd["w_codes"]), cu(fd["w_scales"]))
         x = cu(fd["x"]).view(torch.bfloat16)
-        ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(fw.T, fw.K), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(fw.T, fw.N, fw.K), dtype=torch.uint8, device="cuda")
         for _ in range(a.steps or 3):
             y = moe.moe_fp8_linear(x, packed, fw.N, ws=ws)
         torch.cuda.synchronize()

@@ -77,7 +77,7 @@ def _load():
         "moe_fp8_packed_bytes": ([i32, i32], sz),
         "moe_fp8_pack_weights": ([i32, i32, vp, vp, vp, vp], i32),
         "moe_fp8_unpack_weights": ([i32, i32, vp, vp, vp, vp], i32),
-        "moe_fp8_workspace_bytes": ([i32, i32], sz),
+        "moe_fp8_workspace_bytes": ([i32, i32, i32], sz),
         "moe_fp8_linear": ([vp, i32, i32, i32, vp, vp, vp, sz, vp, vp, vp], i32),
         "moe_set_option": ([i32, i32], i32),
         "moe_get_option": ([i32], i32),
@@ -372,7 +372,7 @@ def moe_fp8_linear(x, packed, N: int, ws=None, y=None, debug: dict | None = None
     may hold uint8 CUDA tensors q [T, K] and s [T, K/128] for the quantised x."""
     T, K = x.shape
     if ws is None:
-        ws = _empty_aligned(lib.moe_fp8_workspace_bytes(T, K), x.device)
+        ws = _empty_aligned(lib.moe_fp8_workspace_bytes(T, N, K), x.device)
     if y is None:
         y = torch.empty((T, N), dtype=torch.bfloat16, device=x.device)
     dq = (debug or {}).get("q")

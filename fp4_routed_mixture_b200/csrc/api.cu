@@ -610,9 +610,9 @@ int moe_fp8_unpack_weights(int N, int K, const void* packed, uint8_t* w_codes, u
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_fp8_unpack_weights launch");
 }
 
-size_t moe_fp8_workspace_bytes(int T_max, int K) {
-    if (T_max < 0 || K <= 0 || K % 128) return 0;
-    return moe::fp8_workspace_bytes(T_max, K);
+size_t moe_fp8_workspace_bytes(int T_max, int N, int K) {
+    if (T_max < 0 || K <= 0 || K % 128 || N <= 0 || N % 128) return 0;
+    return moe::fp8_workspace_bytes(T_max, N, K);
 }
 
 int moe_fp8_linear(const void* x_bf16, int T, int N, int K, const void* packed, void* y_bf16, void* ws,
@@ -626,9 +626,9 @@ int moe_fp8_linear(const void* x_bf16, int T, int N, int K, const void* packed, 
     if (!aligned(ws, 256) || !aligned(packed, 256) || !aligned(x_bf16, 16) || !aligned(y_bf16, 2) ||
         (dbg_q && !aligned(dbg_q, 16)))
         return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: ws/packed need 256-byte, x 16-byte alignment");
-    if (ws_bytes < moe::fp8_workspace_bytes(T, K))
+    if (ws_bytes < moe::fp8_workspace_bytes(T, N, K))
         return fail(MOE_ERR_INVALID_ARG, "moe_fp8_linear: ws_bytes %zu < %zu", ws_bytes,
-                    moe::fp8_workspace_bytes(T, K));
+                    moe::fp8_workspace_bytes(T, N, K));
     if (T == 0) {
         cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), stream);
         return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_fp8_linear memset");

@@ -34,6 +34,11 @@
 // token-tile-major so that consecutive tiles share the activations in L2.
 // The epilogue writes bf16 y.  Every wait is bounded and raises
 // MOE_FLAG_TIMEOUT.
+// Decode sizes (T <= kFp8SplitMaxT: one token tile, N/128 tiles for 148 SMs):
+// the K range of every tile is split over S CTAs (S <= 8, about SMs / tiles),
+// each writes its fp32 partial sums to the workspace, and k_fp8_reduce adds
+// the S partials in a fixed order and rounds to bf16 -- deterministic, and the
+// weight stream is spread over S times as many SMs.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -74,6 +79,8 @@ struct F8Args {
     __nv_bfloat16* y;          // [T, N]
     int32_t* flag;
     uint64_t wait_ns;
+    int splits;                // S > 1: K split S ways, fp32 partials to `part`
+    float* part;               // [S][T][N]
 };
 
 // kind::mxf8f6f4 instruction descriptor: E4M3 x E4M3, UE8M0 scales, fp32
@@ -107,14 +114,19 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
     extern __shared__ __align__(1024) uint8_t f8_smem_raw[];
     F8Shared& sh = *reinterpret_cast<F8Shared*>(f8_smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int KG = a.K / 128, RB = a.N / F8_BM, NB = (a.T + F8_BN - 1) / F8_BN;
-    const int total = RB * NB;
+    const int KG = a.K / 128, RB = a.N / F8_BM, NB = (a.T + F8_BN - 1) / F8_BN, S = a.splits;
+    const int total = RB * NB * S;
     if (total == 0) return;
     const int ntiles = ((int)blockIdx.x < total) ? (total - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-    auto tile = [&](int j, int& rb, int& nb) {
+    // work item j of this CTA: tile (rb, nb) and its K range [g0, g1)
+    auto tile = [&](int j, int& rb, int& nb, int& g0, int& g1, int& s) {
         const int t = (int)blockIdx.x + j * (int)gridDim.x;
-        nb = t / RB;
-        rb = t % RB;
+        const int tt = t / S;
+        s = t % S;
+        nb = tt / RB;
+        rb = tt % RB;
+        g0 = s * KG / S;
+        g1 = (s + 1) * KG / S;
     };
 
     if (threadIdx.x == 0) {
@@ -159,14 +171,14 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
         bool filled[F8_STAGES] = {};
         uint32_t fill_parity[F8_STAGES] = {};
         for (int j = r; j < ntiles && !*abort; j += F8_PIPES) {
-            int rb, nb;
-            tile(j, rb, nb);
+            int rb, nb, g0, g1, sp;
+            tile(j, rb, nb, g0, g1, sp);
             const uint8_t* wsrc = a.w + (size_t)rb * KG * F8_A_BYTES;
             const uint8_t* bsrc = a.xb + (size_t)nb * KG * F8_B_BYTES;
             const uint8_t* ssrc = a.xs + (size_t)nb * KG * F8_SF_BYTES;
             const int n_mma = (min(F8_BN, a.T - nb * F8_BN) + 15) & ~15;
             const uint32_t bbytes = (uint32_t)n_mma * 128;   // the tile's token rows
-            for (int g = 0; g < KG; ++g) {
+            for (int g = g0; g < g1; ++g) {
                 const uint32_t fb = smem_u32(&sh.full[r][stage]), eb = smem_u32(&sh.empty[r][stage]);
                 if (!wait(eb, phase ^ 1u)) {
                     give_up();
@@ -197,8 +209,8 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
         int stage = 0;
         uint32_t phase = 0;
         for (int j = r; j < ntiles && !*abort; j += F8_PIPES) {
-            int rb, nb;
-            tile(j, rb, nb);
+            int rb, nb, g0, g1, sp;
+            tile(j, rb, nb, g0, g1, sp);
             const int n_valid = min(F8_BN, a.T - nb * F8_BN);
             const int n_mma = (n_valid + 15) & ~15;
             const int buf = j % F8_ACC;
@@ -210,7 +222,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
             tc_fence_after();
             const uint32_t dcol = tmem + buf * F8_BN;
             bool ok = true;
-            for (int g = 0; g < KG; ++g) {
+            for (int g = g0; g < g1; ++g) {
                 if (!wait(smem_u32(&sh.full[r][stage]), phase)) {
                     give_up();
                     ok = false;
@@ -231,7 +243,7 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
                         // tokens: columns 128 B apart, 8-row groups 1 KB apart)
                         const uint64_t adesc = make_sdesc(sa + 512 + mi * 2 * 2048, 2048, 128);
                         const uint64_t bdesc = make_sdesc(sb + mi * 2 * 128, 128, 1024);
-                        tc_mma_mxf8(dcol, adesc, bdesc, f8_idesc(n_mma, mi), sfa, sfb, (g | mi) != 0);
+                        tc_mma_mxf8(dcol, adesc, bdesc, f8_idesc(n_mma, mi), sfa, sfb, (g > g0) || mi != 0);
                     }
                     tc_commit(smem_u32(&sh.empty[r][stage]));
                 }
@@ -259,8 +271,8 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
         const int q = warp & 3;
         const int n0 = 32 * (ew >> 2);
         for (int j = 0; j < ntiles && !*abort; ++j) {
-            int rb, nb;
-            tile(j, rb, nb);
+            int rb, nb, g0, g1, sp;
+            tile(j, rb, nb, g0, g1, sp);
             const int n_valid = min(F8_BN, a.T - nb * F8_BN);
             const int buf = j % F8_ACC;
             const uint32_t use = (uint32_t)(j / F8_ACC);
@@ -273,10 +285,17 @@ __global__ void __launch_bounds__(F8_THREADS, 1) k_fp8_gemm(F8Args a) {
                 uint32_t v[32];
                 tc_ld32(tmem + ((uint32_t)(q * 32) << 16) + buf * F8_BN + n0, v);
                 const int n = rb * F8_BM + q * 32 + lane;
-                __nv_bfloat16* out = a.y + (size_t)(nb * F8_BN + n0) * a.N + n;
+                if (S == 1) {
+                    __nv_bfloat16* out = a.y + (size_t)(nb * F8_BN + n0) * a.N + n;
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    if (n0 + c < n_valid) out[(size_t)c * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                    for (int c = 0; c < 32; ++c)
+                        if (n0 + c < n_valid) out[(size_t)c * a.N] = __float2bfloat16_rn(__uint_as_float(v[c]));
+                } else {
+                    float* out = a.part + ((size_t)sp * a.T + nb * F8_BN + n0) * a.N + n;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (n0 + c < n_valid) out[(size_t)c * a.N] = __uint_as_float(v[c]);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -305,10 +324,17 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// The first kernel of a call: thread 0 of CTA 0 also clears the call's error
+// word, or sets FLAG_LAYOUT when the packed weights were built for other dims.
 __global__ void __launch_bounds__(256)
     k_fp8_quant_act(const __nv_bfloat16* __restrict__ x, int T, int K, uint8_t* __restrict__ xb,
-                    uint8_t* __restrict__ xs, uint8_t* __restrict__ dbg_q, uint8_t* __restrict__ dbg_s) {
+                    uint8_t* __restrict__ xs, uint8_t* __restrict__ dbg_q, uint8_t* __restrict__ dbg_s,
+                    const uint8_t* __restrict__ packed, int N, int32_t* flag) {
     pdl_begin();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const Fp8Header* h = reinterpret_cast<const Fp8Header*>(packed);
+        *flag = (h->magic == kFp8Magic && (int)h->N == N && (int)h->K == K) ? 0 : FLAG_LAYOUT;
+    }
     const int t = blockIdx.x;
     const int KG = K / 128, nb = t / F8_BN, row = t % F8_BN;
     const int nchunk = K / 16;
@@ -406,16 +432,46 @@ __global__ void k_fp8_header(uint8_t* packed, int N, int K) {
     h->flag = 0;
 }
 
-__global__ void k_fp8_check_header(const uint8_t* packed, int N, int K, int32_t* flag) {
-    const Fp8Header* h = reinterpret_cast<const Fp8Header*>(packed);
-    *flag = (h->magic == kFp8Magic && (int)h->N == N && (int)h->K == K) ? 0 : FLAG_LAYOUT;
-}
 
 size_t fp8_packed_bytes(int N, int K) { return kFp8HeaderBytes + (size_t)(N / 128) * (K / 128) * kFp8ChunkBytes; }
 
-size_t fp8_workspace_bytes(int T, int K) {
+// Workspace: the error word (256 bytes), the activation tiles, then (calls of
+// at most kFp8SplitMaxT tokens) the fp32 partial sums of the split K ranges.
+static size_t fp8_act_bytes(int T, int K) {
     const size_t nb = (size_t)(T + F8_BN - 1) / F8_BN;
-    return 256 + nb * (K / 128) * (F8_B_BYTES + F8_SF_BYTES);
+    return nb * (K / 128) * (F8_B_BYTES + F8_SF_BYTES);
+}
+static size_t fp8_part_offset(int T, int K) { return 256 + ((fp8_act_bytes(T, K) + 255) & ~(size_t)255); }
+
+size_t fp8_workspace_bytes(int T, int N, int K) {
+    // (a call with fewer tokens than T lays its partials out at a lower offset)
+    const int tp = std::min(T, kFp8SplitMaxT);
+    return fp8_part_offset(T, K) + (size_t)kFp8MaxSplits * tp * N * sizeof(float);
+}
+
+// y = bf16(sum over s of the partial sums, s = 0, 1, ... in order).
+__global__ void __launch_bounds__(256)
+    k_fp8_reduce(const float* __restrict__ part, int S, int T, int N, __nv_bfloat16* __restrict__ y,
+                 const int32_t* flag) {
+    pdl_begin();
+    // weights packed for other dims: the GEMM wrote no partials and y stays untouched
+    if (*(volatile const int32_t*)flag & FLAG_LAYOUT) return;
+    const size_t tn = (size_t)T * N, n4 = tn / 4;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        float4 acc = reinterpret_cast<const float4*>(part)[i];
+        for (int s = 1; s < S; ++s) {
+            const float4 v = reinterpret_cast<const float4*>(part + (size_t)s * tn)[i];
+            acc.x = __fadd_rn(acc.x, v.x);
+            acc.y = __fadd_rn(acc.y, v.y);
+            acc.z = __fadd_rn(acc.z, v.z);
+            acc.w = __fadd_rn(acc.w, v.w);
+        }
+        __nv_bfloat16* o = y + 4 * i;
+        o[0] = __float2bfloat16_rn(acc.x);
+        o[1] = __float2bfloat16_rn(acc.y);
+        o[2] = __float2bfloat16_rn(acc.z);
+        o[3] = __float2bfloat16_rn(acc.w);
+    }
 }
 
 cudaError_t launch_fp8_pack(int N, int K, const uint8_t* wq, const uint8_t* ws, void* packed, bool fwd,
@@ -452,17 +508,25 @@ cudaError_t launch_fp8_linear(const void* x, int T, int N, int K, const void* pa
     uint8_t* xb = (uint8_t*)ws + 256;
     const size_t nb = (size_t)(T + F8_BN - 1) / F8_BN;
     uint8_t* xs = xb + nb * (K / 128) * F8_B_BYTES;
-    k_fp8_check_header<<<1, 1, 0, st>>>((const uint8_t*)packed, N, K, flag);
-    count_launches(1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(k_fp8_quant_act, dim3(T), dim3(256), 0, st, (const __nv_bfloat16*)x, T, K, xb, xs, dbg_q, dbg_s);
+    cudaError_t e = launch_pdl(k_fp8_quant_act, dim3(T), dim3(256), 0, st, (const __nv_bfloat16*)x, T, K, xb, xs,
+                               dbg_q, dbg_s, (const uint8_t*)packed, N, flag);
     count_launches(1);
     if (e != cudaSuccess) return e;
     const int grid = fp8_grid();
     if (grid <= 0) return cudaErrorInvalidConfiguration;
-    F8Args a{(const uint8_t*)packed + kFp8HeaderBytes, xb, xs, T, N, K, (__nv_bfloat16*)y, flag, wait_ns};
+    // split the K range when one token tile leaves most SMs without a tile
+    const int RB = N / F8_BM, KG = K / 128;
+    int S = 1;
+    // (up to two items per CTA: its two pipes stream them at the same time)
+    if (T <= kFp8SplitMaxT && RB < grid) S = std::max(1, std::min({2 * grid / RB, kFp8MaxSplits, KG}));
+    float* part = (float*)((uint8_t*)ws + fp8_part_offset(T, K));
+    F8Args a{(const uint8_t*)packed + kFp8HeaderBytes, xb, xs, T, N, K, (__nv_bfloat16*)y, flag, wait_ns, S, part};
     e = launch_pdl(k_fp8_gemm, dim3(grid), dim3(F8_THREADS), sizeof(F8Shared), st, a);
+    count_launches(1);
+    if (e != cudaSuccess || S == 1) return e;
+    const size_t n4 = (size_t)T * N / 4;
+    e = launch_pdl(k_fp8_reduce, dim3((unsigned)std::min<size_t>((n4 + 255) / 256, 148 * 8)), dim3(256), 0, st,
+                   (const float*)part, S, T, N, (__nv_bfloat16*)y, (const int32_t*)flag);
     count_launches(1);
     return e;
 }

@@ -203,7 +203,11 @@ struct Fp8Header {
     int32_t flag;  // device error word of the packing
 };
 size_t fp8_packed_bytes(int N, int K);
-size_t fp8_workspace_bytes(int T, int K);
+// Calls of at most kFp8SplitMaxT tokens split each tile's K range over up to
+// kFp8MaxSplits CTAs (fp32 partials in the workspace).
+constexpr int kFp8SplitMaxT = 64;
+constexpr int kFp8MaxSplits = 8;
+size_t fp8_workspace_bytes(int T, int N, int K);
 cudaError_t launch_fp8_pack(int N, int K, const uint8_t* wq, const uint8_t* ws, void* packed, bool fwd,
                             uint8_t* out_wq, uint8_t* out_ws, cudaStream_t st);
 cudaError_t launch_fp8_linear(const void* x, int T, int N, int K, const void* packed, void* y, void* ws,

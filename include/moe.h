@@ -294,12 +294,14 @@ int moe_fp8_pack_weights(int N, int K, const uint8_t *w_codes, const uint8_t *w_
 int moe_fp8_unpack_weights(int N, int K, const void *packed, uint8_t *w_codes, uint8_t *w_scales,
                            cudaStream_t stream);
 
-/* Workspace of moe_fp8_linear for up to T_max tokens of K inputs (the
- * quantised activations in the GEMM's tile order; error word first). */
-size_t moe_fp8_workspace_bytes(int T_max, int K);
+/* Workspace of moe_fp8_linear for up to T_max tokens, N outputs and K inputs
+ * (error word first; the quantised activations in the GEMM's tile order; for
+ * calls of at most 64 tokens, whose tiles' K ranges are split over several
+ * CTAs, the fp32 partial sums).  0 for invalid dims. */
+size_t moe_fp8_workspace_bytes(int T_max, int N, int K);
 
 /* y [T, N] bf16 = the projection of x [T, K] bf16 (16-byte aligned) by the
- * packed weights.  ws: moe_fp8_workspace_bytes(T_max, K) bytes, 256-byte
+ * packed weights.  ws: moe_fp8_workspace_bytes(T_max, N, K) bytes, 256-byte
  * aligned, T <= T_max; its first int32 is the device error word (cleared by
  * this call; MOE_FLAG_LAYOUT when `packed` was built for other N, K; the GEMM
  * then leaves y untouched; MOE_FLAG_TIMEOUT as in moe_forward).  dbg_q

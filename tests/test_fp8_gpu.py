@@ -2,7 +2,9 @@
 through the C ABI.
 
 Bit-exact: the packed-layout round trip, the E4M3 codes and UE8M0 bytes of the
-quantised activations.  Tolerance on the bf16 output (the layer's bar:
+quantised activations.  Calls of at most 64 tokens split each tile's K range
+over several CTAs (fp32 partial sums added in a fixed order): the same bound
+holds.  Tolerance on the bf16 output (the layer's bar:
 max|dy| <= 2e-2 max|y_oracle|, relative Frobenius error <= 5e-3), and per
 element |y - y_exact| <= one bf16 ulp + 2^-12 * sum_k |terms| (fp32 tensor-core
 accumulation of up to K exact products, then one bf16 rounding).
@@ -38,7 +40,7 @@ def _run(moe, d, N, tok=None):
     packed = moe.moe_fp8_pack_weights(cu(d["w_codes"]), cu(d["w_scales"]))
     dbg = dict(q=torch.empty((T, K), dtype=torch.uint8, device="cuda"),
                s=torch.empty((T, K // 128), dtype=torch.uint8, device="cuda"))
-    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(T, K), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(T, N, K), dtype=torch.uint8, device="cuda")
     ybuf = torch.full((T + 2, N), 3.0, dtype=torch.bfloat16, device="cuda")
     y = ybuf[1:T + 1]
     moe.moe_fp8_linear(x, packed, N, ws=ws, y=y, debug=dbg)
@@ -85,7 +87,10 @@ def test_fp8_pack_round_trip(moe):
     (130, 256, 384, 2),      # two token tiles, the second with 2 rows; 3 stages
     (300, 384, 512, 3),      # ragged: 44 rows in the last token tile
     (128, 128, 4096, 4),     # a full tile, 32 stages
-    (37, 512, 256, 5),
+    (37, 512, 256, 5),       # (calls of at most 64 tokens split the K range: here 2 ways)
+    (8, 1024, 2048, 6),      # 8 weight tiles, K split 8 ways
+    (64, 256, 384, 7),       # K split 3 ways over 3 stages: one stage each
+    (65, 256, 512, 8),       # one token more: no split
 ])
 def test_fp8_linear_shapes(moe, T, N, K, seed):
     d = dict(x=synth.x_bf16(seed, T, K))
@@ -119,7 +124,7 @@ def test_fp8_layout_mismatch_flag(moe):
     d.update(synth.fp8_weights(7, 256, 256))
     packed = moe.moe_fp8_pack_weights(cu(d["w_codes"]), cu(d["w_scales"]))
     x = cu(d["x"]).view(torch.bfloat16)
-    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(16, 256), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(moe.lib.moe_fp8_workspace_bytes(16, 128, 256), dtype=torch.uint8, device="cuda")
     y = torch.full((16, 128), 5.0, dtype=torch.bfloat16, device="cuda")
     moe.moe_fp8_linear(x, packed, 128, ws=ws, y=y)           # packed for N = 256
     assert moe.moe_check_device_flag(ws) & moe.FLAG_LAYOUT
