@@ -348,18 +348,20 @@ def run_fp8_dense(name: str, steps: int, warmup: int, dist: Dist, peaks: dict, w
     line = {"workload": name, "T": w.T, "N": w.N, "K": w.K, "steps": steps,
             "value": round(whole_job_value(dist.world, w.T, steps, ms * steps), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 5), "clocks": clk,
-            "kernels": "k_fp8_quant_act + k_fp8_gemm (tcgen05 kind::mxf8f6f4 block-scaled); the step times both"}
+            "kernels": "k_fp8_quant_act + k_fp8_gemm (tcgen05 kind::mxf8f6f4 block-scaled) + k_fp8_reduce "
+                       "(calls of at most 64 tokens: the split K ranges' partial sums); the step times them all"}
+    traffic = profiled_traffic(f"k_fp8_gemm_{name}.md")
     if w.T >= 1024:
         tf = flop / (ms * 1e-3) / 1e12
         fp8_peak = 2.0 * peaks["bf16_tflops"]
         line["roofline"] = {"bound": "tensor", "achieved": round(tf, 2), "unit": "TFLOP/s", "peak": fp8_peak,
                             "frac": round(tf / fp8_peak, 5),
-                            "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)", "traffic": None}
+                            "peak_source": peaks["source"] + " bf16 x 2 (fp8/bf16 nominal ratio)", "traffic": traffic}
     else:
         gbs = wbytes / (ms * 1e-3) / 1e9
         line["roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
                             "frac": round(gbs / peaks["hbm_gbs"], 4), "alg_bytes_per_launch": wbytes,
-                            "peak_source": peaks["source"] + " (hbm_gbs: stream copy)", "traffic": None}
+                            "peak_source": peaks["source"] + " (hbm_gbs: stream copy)", "traffic": traffic}
     del packed, ws
     torch.cuda.empty_cache()
     return line
