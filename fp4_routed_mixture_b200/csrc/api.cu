@@ -382,7 +382,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     const int32_t* gemv_soff = logits ? offsets : soff;
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, xq, xinit, perm, k, offsets,
-                                 uoff1, gemv_soff, E, gacc, flag, I, P, group, stream), "W1");
+                                 uoff1, gemv_soff, E, gacc, flag, I, P, group, false, stream), "W1");
     if (use_tc && tc_tn1)
         MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w1, PL.w1_expert_bytes, H, 2 * I, I, px, L.plane_rows, poff, P,
                                        offsets, toff1, E, flag, sx, perm, k, hbuf, opt.wait_ns, withhold, stream),
@@ -399,7 +399,7 @@ int forward_impl(const Options& opt, const moe_dims* d, const float* logits, con
     if (ev && ev[2]) MOE_TRY(cudaEventRecord(ev[2], stream), "event");
     if (use_gemv)
         MOE_TRY(moe::launch_gemv(pk + PL.w2, PL.w2_expert_bytes, I, H, hq, hinit, perm, 0, offsets,
-                                 uoff2, gemv_soff, E, yacc, flag, 0, P, group, stream), "W2");
+                                 uoff2, gemv_soff, E, yacc, flag, 0, P, group, true, stream), "W2");
     if (use_tc && tc_tn2)
         MOE_TRY(moe::launch_tc_gemm_tn(pk + PL.w2, PL.w2_expert_bytes, I, H, 0, ph, L.plane_rows, poff, P,
                                        offsets, toff2, E, flag, sh, perm, 0, yf, opt.wait_ns, 0, stream),

@@ -18,7 +18,10 @@ namespace moe {
 // the compact streaming row come from per-expert tables (expert_tc, offsets,
 // stream_off: E entries, cache-resident), not from the per-row slot table, so
 // a slot costs no extra dependent miss.  With expert_tc == NULL every row is a
-// streaming row stored at its sorted row.
+// streaming row stored at its sorted row.  These tables come from the route,
+// sort and plan, launches before the h quant (which always runs between them
+// and the W2 GEMMs in front of this launch), so they are read before waiting
+// on the W2 GEMMs; Y, the fp64 sums and the h scales are read after.
 template <int KMAX>
 __global__ void __launch_bounds__(256)
     k_combine(const double* __restrict__ yacc, const float* __restrict__ yf,
@@ -26,7 +29,6 @@ __global__ void __launch_bounds__(256)
               const int32_t* __restrict__ stream_off, const int32_t* __restrict__ topk_idx, int E,
               int stream_rows, const float* __restrict__ sh, const float* __restrict__ gates,
               const int32_t* __restrict__ pos, int P, int k, int H, uint2* __restrict__ y, int32_t* flag) {
-    pdl_begin();
     const int t = blockIdx.y;
     const int n4 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 4 columns
     if (4 * n4 >= H) return;
@@ -49,6 +51,7 @@ __global__ void __launch_bounds__(256)
             }
         }
     }
+    pdl_begin();
     float4 v[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {

@@ -47,7 +47,11 @@ namespace moe {
 // one-tile variants with more or fewer registers, and TMA bulk copies in place
 // of the per-lane 16-byte copies were all slower.  The kernel is bound by
 // integer issue (the nibble decode), at about 0.65 of the measured copy
-// bandwidth.
+// bandwidth.  With the equal split the warps of a launch finish over a wide
+// window (decode T = 8, W1: 32-81 us after the wait, in the order of their
+// issue priority on the SM's schedulers); dynamic chunks from an atomic
+// counter, a split weighted by priority, and an L2 prefetch a few items ahead
+// all measured slower than the equal split.
 // One warp per CTA, 32 CTAs per SM: every warp runs its own pipeline anyway,
 // and single-warp CTAs measured ~10% faster than 8-warp CTAs at the same 32
 // warps per SM (decode_T8: 3.58 -> 3.96 TB/s; 4 warps/CTA: 3.70).
@@ -146,6 +150,7 @@ struct GemvArgs {
     const int32_t* flag;       // device error word: a layout mismatch stops the kernel
     int gate_up_half;          // > 0 (= I) for W1: device rows interleave gate and up rows
     int P;                     // pairs (rows of the sorted tables)
+    int pre_wait;              // 1: the tables were written at least two launches back (see k_gemv)
     uint32_t zero;             // always 0 (see Tables)
 };
 
@@ -163,6 +168,13 @@ struct Unit {
 
 template <int G>
 __device__ __forceinline__ Unit unit_at(const GemvArgs& a, int unit) {
+    // (callers stay inside the launch's units; a unit past them would address
+    // memory outside the tables and weights, so it is flagged and clamped)
+    const int units = __ldg(a.unit_off + a.E);
+    if (unit >= units) {
+        raise_flag(const_cast<int32_t*>(a.flag), FLAG_BOUNDS);
+        unit = units - 1;
+    }
     int lo = 0, hi = a.E;  // last e with unit_off[e] <= unit
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -232,7 +244,14 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
     constexpr int kGroup = G;
     using Slot = moe::Slot<G>;
     constexpr int kSlotBytes = slot_bytes<G>();
-    pdl_begin();
+    // pre_wait: the launch in front of this one (the h quant, in front of W2)
+    // writes only the activations, and the unit tables and the error word's
+    // FLAG_LAYOUT bit come from launches before it, which had completed when
+    // that launch passed its own wait.  So the weights of the warp's first item
+    // go into the ring while the launch in front still runs, and the
+    // activations are copied after the wait.  (Also prefetching the next items'
+    // weights into L2 there measured slower: it delayed the h quant.)
+    if (!a.pre_wait) pdl_begin();
     extern __shared__ __align__(16) uint8_t smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // packed weights built for other dims may be smaller than the offsets used here
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
               kg * 4;
     };
     start_unit(f_kg);
-    auto issue = [&]() {
+    auto issue_w = [&]() {  // the item's weights
         const uint32_t sb = ring_s + f_slot * kSlotBytes;
         if (TP == 4) cp_async16(sb + o_sc, f_w + g_sc);
         else if (TP == 2) cp_async8(sb + o_sc, f_w + g_sc);
@@ -284,9 +303,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
 #pragma unroll
             for (int u = 0; u < TP; ++u)
                 cp_async16(sb + o_code + (bb * TP + u) * 512, f_w + g_code + bb * 2048 + u * 512);
+    };
+    auto issue_x = [&]() {  // the item's activation bytes and block terms
+        const uint32_t sb = ring_s + f_slot * kSlotBytes;
         if ((lane >> 3) < fu.mc) cp_async16(sb + o_x, f_x);
         if (lane < fu.mc) cp_async16(sb + o_init, f_i);
-        cp_async_commit();
+    };
+    auto advance = [&]() {  // to the next item of the warp's range
         --f_left;
         f_slot = (f_slot + 1 == kStages) ? 0 : f_slot + 1;
         if (++f_kg == KG) {
@@ -301,11 +324,23 @@ __global__ void __launch_bounds__(kGemvWarps * 32, G == 2 ? 25 : kMinBlocks) k_g
             f_i += 4;
         }
     };
+    auto issue = [&]() {
+        issue_w();
+        issue_x();
+        cp_async_commit();
+        advance();
+    };
 
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        if (f_left > 0) issue();
-        else cp_async_commit();
+    static_assert(kStages == 2, "the prologue fills one slot");
+    if (a.pre_wait) {  // (f_left > 0 here)
+        issue_w();
+        cp_async_commit();
+        pdl_begin();
+        issue_x();
+        cp_async_commit();
+        advance();
+    } else {
+        issue();
     }
 
     // ---- compute side ----
@@ -405,9 +440,10 @@ static int gemv_grid() {
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, const int32_t* stream_off, int E,
-                        double* out, const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st) {
+                        double* out, const int32_t* flag, int gate_up_half, int P, int group, bool pre_wait,
+                        cudaStream_t st) {
     GemvArgs a{w, expert_bytes, K, N, act, act_init, perm, k_div, offsets, unit_off, stream_off, E, out, flag,
-               gate_up_half, P, 0u};
+               gate_up_half, P, pre_wait ? 1 : 0, 0u};
     const int grid = group == 2 ? gemv_grid<2>() : gemv_grid<4>();
     if (grid <= 0) return cudaErrorInvalidConfiguration;
     const cudaError_t e =

@@ -159,7 +159,8 @@ cudaError_t launch_quant_rows(const float* v, int rows, int cols, int8_t* q, flo
 cudaError_t launch_gemv(const uint8_t* w, size_t expert_bytes, int K, int N, const int8_t* act,
                         const int32_t* act_init, const int32_t* perm, int k_div,
                         const int32_t* offsets, const int32_t* unit_off, const int32_t* stream_off, int E,
-                        double* out, const int32_t* flag, int gate_up_half, int P, int group, cudaStream_t st);
+                        double* out, const int32_t* flag, int gate_up_half, int P, int group, bool pre_wait,
+                        cudaStream_t st);
 
 size_t tc_smem_bytes();
 // Digit planes, per 128-input stage g and group of 8 plane rows, hold

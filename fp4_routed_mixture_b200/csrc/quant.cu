@@ -57,7 +57,6 @@ __global__ void __launch_bounds__(kQThreads)
              int stream_rows, uint8_t* __restrict__ planes, int P, int k, int I, int8_t* __restrict__ hq,
              float* __restrict__ sh, int32_t* __restrict__ hinit, int8_t* __restrict__ dbg_hq,
              float* __restrict__ dbg_sh, int32_t* flag) {
-    pdl_begin();
     static_assert(R == 32 || R == kQThreads, "a warp or a CTA per row");
     float4 keep[KEEP > 0 ? KEEP : 1];
     __shared__ uint16_t lut[256];
@@ -67,10 +66,26 @@ __global__ void __launch_bounds__(kQThreads)
     const int l = threadIdx.x % R;
     const int rows_per_cta = kQThreads / R;
     const int steps = I / (4 * R);          // I % 128 == 0; for R = 256 also I % 1024 == 0 (checked by the launcher)
+    // A row's slot, pair and x scale come from the plan, sort and x quant,
+    // launches before the W1 GEMM in front of this one (which had completed
+    // when that GEMM passed its own wait): the first row's are read before
+    // waiting on the GEMM, whose output (the W1 sums or h) is read after.
+    auto row_slot = [&](int i) { return i < P ? plane_row[i] : kNoRow; };
+    int pre_slot = row_slot(blockIdx.x * rows_per_cta + (int)threadIdx.x / R), pre_p = 0;
+    float pre_sx = 0.0f;
+    {
+        const int i = blockIdx.x * rows_per_cta + (int)threadIdx.x / R;
+        if (i < P && pre_slot != kNoRow) {
+            pre_p = checked_index(perm[i], P, flag);
+            if (pre_slot < 0) pre_sx = sx[pre_p / k];
+        }
+    }
+    pdl_begin();
     for (int i0 = blockIdx.x * rows_per_cta; i0 < P; i0 += gridDim.x * rows_per_cta) {
+        const bool first = i0 == (int)blockIdx.x * rows_per_cta;
         const int i = i0 + (int)threadIdx.x / R;
         // (R = 256: always in range; a row's R threads take the same branches)
-        const int slot = i < P ? plane_row[i] : kNoRow;
+        const int slot = first ? pre_slot : row_slot(i);
         const bool tc = slot >= 0;
         const int srow = ~slot;              // streaming row (slot < 0)
         const bool slot_ok = tc ? slot < plane_rows : (slot != kNoRow && srow < stream_rows);
@@ -78,7 +93,7 @@ __global__ void __launch_bounds__(kQThreads)
         const bool row_ok = i < P && slot_ok;
         float a = 0.0f;
         int p = 0;
-        if (row_ok) p = checked_index(perm[i], P, flag);
+        if (row_ok) p = first ? pre_p : checked_index(perm[i], P, flag);
         float4* hr = reinterpret_cast<float4*>(hbuf + (size_t)(row_ok ? i : 0) * I);
         // KEEP > 0 and the row fits: pass 1 leaves the row in registers
         const bool use_keep = KEEP > 0 && steps <= KEEP;
@@ -99,7 +114,7 @@ __global__ void __launch_bounds__(kQThreads)
                 }
             }
         } else if (row_ok) {
-            const double s = (double)sx[p / k];
+            const double s = (double)(first ? pre_sx : sx[p / k]);
             const double* gr = gacc + (size_t)srow * 2 * I;
             for (int g = 0; g < steps; ++g) {
                 const int e0 = 4 * (g * R + l);
